@@ -1,0 +1,257 @@
+"""Seeded synthetic inputs for the DSA decode path.
+
+This module draws random numbers and encodes them into the storage formats the
+path consumes (FP8 e4m3 codes, bf16 bits, int32 tables).  It holds none of the
+method's arithmetic: no score, no selection, no attention.  Both the GPU path
+(via tests / bench) and the fp64 oracle read the bytes it produces, so the two
+sides never have to agree on a quantisation step.
+
+Every tensor comes from its own PCG64 stream seeded by
+``SeedSequence([1000 + config_id + seed_offset, stream])`` with these streams:
+  0 context lengths, 1 page permutation, 2 q^I, 3 w, 4 k^I, 5 heavy-tail rows,
+  6 q (attention query), 7 latent KV.
+Encodings: e4m3 via torch's float8_e4m3fn cast after clamping to +-448 (round
+to nearest even, saturating); bf16 via torch's round-to-nearest-even cast.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+from typing import Optional
+
+import numpy as np
+import torch
+
+# Shapes of the five workloads: tiny decode, batched decode at V3.2 shapes,
+# long-context decode (128K), causal prefill (16K) and paged two-token decode.
+CONFIGS = {
+    1: dict(name="tiny_decode_4k", kind="decode", nseq=1, L=4096, h_idx=4, d_idx=64,
+            w_std=0.5, topk=256, h=16, tail=False),
+    2: dict(name="batched_decode_64x32k", kind="decode", nseq=64, L=32768, h_idx=64,
+            d_idx=128, w_std=0.125, topk=2048, h=128, tail=True),
+    3: dict(name="long_decode_16x128k", kind="decode", nseq=16, L=131072, h_idx=64,
+            d_idx=128, w_std=0.125, topk=2048, h=128, tail=True),
+    4: dict(name="causal_prefill_16k", kind="prefill", nseq=1, L=16384, h_idx=64,
+            d_idx=128, w_std=0.125, topk=2048, h=128, tail=False),
+    5: dict(name="paged_mtp_decode_128seq", kind="paged2", nseq=128, L=16384,
+            h_idx=64, d_idx=128, w_std=0.125, topk=2048, h=128, tail=True),
+}
+D_QK = 576
+D_V = 512
+PAGE_SIZE = 64
+
+
+@dataclasses.dataclass
+class Inputs:
+    """One batch of host-side inputs (numpy, storage formats)."""
+    config_id: int
+    name: str
+    kind: str
+    h_idx: int
+    d_idx: int
+    h: int
+    d_qk: int
+    d_v: int
+    topk: int
+    scale: float
+    q_idx: np.ndarray            # [nq, h_idx, d_idx] uint8 e4m3 codes
+    w: np.ndarray                # [nq, h_idx] uint16 bf16 bits
+    kidx: np.ndarray             # [rows, d_idx] uint8 e4m3 codes
+    k_scale: Optional[np.ndarray]  # [rows] float32 or None
+    q: np.ndarray                # [nq, h, d_qk] uint16 bf16 bits
+    kv: np.ndarray               # [rows, d_qk] uint16 bf16 bits
+    q_seq: np.ndarray            # [nq] int32
+    q_n: np.ndarray              # [nq] int32 visible positions per query
+    seq_len: np.ndarray          # [nseq] int32 cache rows per sequence
+    seq_row0: Optional[np.ndarray]   # [nseq] int64 (contiguous layout)
+    page_table: Optional[np.ndarray]  # [nseq, max_pages] int32 (paged layout)
+    page_size: int
+    q_per_seq: int
+
+    @property
+    def nq(self) -> int:
+        return int(self.q_n.shape[0])
+
+    @property
+    def nseq(self) -> int:
+        return int(self.seq_len.shape[0])
+
+    @property
+    def rows(self) -> int:
+        return int(self.kidx.shape[0])
+
+    @property
+    def max_n(self) -> int:
+        return int(self.q_n.max()) if self.nq else 0
+
+
+def _rng(config_id: int, seed_offset: int, stream: int) -> np.random.Generator:
+    ss = np.random.SeedSequence([1000 + config_id + seed_offset, stream])
+    return np.random.Generator(np.random.PCG64(ss))
+
+
+def encode_e4m3(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).clamp_(-448.0, 448.0)
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def encode_bf16(x: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def _normal_bf16(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.ndarray:
+    """N(0,1) drawn in float32 chunks and stored as bf16 bits."""
+    total = int(np.prod(shape))
+    out = np.empty(total, np.uint16)
+    for start in range(0, total, chunk):
+        n = min(chunk, total - start)
+        out[start:start + n] = encode_bf16(rng.standard_normal(n, dtype=np.float32))
+    return out.reshape(shape)
+
+
+def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = None,
+                L: Optional[int] = None, ragged: bool = False, paged: Optional[bool] = None,
+                lengths: Optional[np.ndarray] = None, with_k_scale: bool = False,
+                topk: Optional[int] = None, h: Optional[int] = None) -> Inputs:
+    """Inputs of workload ``config_id`` (1..5), optionally resized for tests.
+
+    decode  : one query per sequence; query n = L (rows 0..L-1 visible).
+    prefill : one sequence of L tokens; query t sees n = t positions (s < t).
+    paged2  : two queries per sequence (next token + one speculative token)
+              with n = L and L + 1; cache rows L + 1; paged (64-token pages,
+              physical pages a random permutation).
+    ragged  : decode lengths ~ U[1024, L] per sequence, with sequence 0 at
+              2048 and sequence 1 at 2049 (the short-history boundary).
+    """
+    c = dict(CONFIGS[config_id])
+    kind = c["kind"]
+    nseq = c["nseq"] if nseq is None else int(nseq)
+    L = c["L"] if L is None else int(L)
+    h_idx, d_idx = c["h_idx"], c["d_idx"]
+    h = c["h"] if h is None else int(h)
+    k = c["topk"] if topk is None else int(topk)
+    if paged is None:
+        paged = kind == "paged2"
+
+    # context lengths (stream 0)
+    r_len = _rng(config_id, seed_offset, 0)
+    if lengths is not None:
+        seq_ctx = np.asarray(lengths, np.int64).copy()
+        nseq = len(seq_ctx)
+    elif kind == "paged2":
+        z = r_len.standard_normal(nseq)
+        seq_ctx = np.clip(np.round(np.exp(math.log(L) + 1.0 * z)), 512, 131072).astype(np.int64)
+    elif ragged:
+        seq_ctx = r_len.integers(1024, L, size=nseq, endpoint=True).astype(np.int64)
+        if nseq > 0:
+            seq_ctx[0] = min(2048, L)
+        if nseq > 1:
+            seq_ctx[1] = min(2049, L)
+    else:
+        seq_ctx = np.full(nseq, L, np.int64)
+
+    if kind == "prefill":
+        assert nseq == 1
+        q_seq = np.zeros(L, np.int32)
+        q_n = np.arange(L, dtype=np.int32)
+        seq_len = np.array([L], np.int64)
+        q_per_seq = L
+    elif kind == "paged2":
+        q_seq = np.repeat(np.arange(nseq, dtype=np.int32), 2)
+        q_n = np.stack([seq_ctx, seq_ctx + 1], axis=1).reshape(-1).astype(np.int32)
+        seq_len = seq_ctx + 1
+        q_per_seq = 2
+    else:
+        q_seq = np.arange(nseq, dtype=np.int32)
+        q_n = seq_ctx.astype(np.int32)
+        seq_len = seq_ctx.copy()
+        q_per_seq = 1
+    nq = len(q_n)
+
+    # cache layout (stream 1 for the page permutation)
+    if paged:
+        pages = (seq_len + PAGE_SIZE - 1) // PAGE_SIZE
+        total_pages = int(pages.sum())
+        perm = _rng(config_id, seed_offset, 1).permutation(total_pages).astype(np.int32)
+        max_pages = int(pages.max()) if nseq else 1
+        page_table = np.full((nseq, max_pages), -1, np.int32)
+        off = 0
+        for i in range(nseq):
+            page_table[i, :pages[i]] = perm[off:off + pages[i]]
+            off += int(pages[i])
+        rows = total_pages * PAGE_SIZE
+        seq_row0 = None
+        page_size = PAGE_SIZE
+    else:
+        seq_row0 = np.concatenate([[0], np.cumsum(seq_len)[:-1]]).astype(np.int64) if nseq else np.zeros(0, np.int64)
+        rows = int(seq_len.sum())
+        page_table = None
+        page_size = 0
+
+    # indexer query and head weights (streams 2, 3)
+    q_idx = encode_e4m3(_rng(config_id, seed_offset, 2).standard_normal(
+        (nq, h_idx, d_idx), dtype=np.float32))
+    w = encode_bf16(_rng(config_id, seed_offset, 3).standard_normal(
+        (nq, h_idx), dtype=np.float32) * np.float32(c["w_std"]))
+
+    # index-K cache (stream 4), heavy tail (stream 5): per sequence, ceil(1% of
+    # its rows) distinct positions scaled x3 before quantising.
+    kf = _rng(config_id, seed_offset, 4).standard_normal((rows, d_idx), dtype=np.float32)
+    if c["tail"]:
+        r_tail = _rng(config_id, seed_offset, 5)
+        for i in range(nseq):
+            n_i = int(seq_len[i])
+            cnt = int(math.ceil(0.01 * n_i))
+            pos = r_tail.choice(n_i, size=cnt, replace=False)
+            if paged:
+                phys = page_table[i, pos // PAGE_SIZE].astype(np.int64) * PAGE_SIZE + pos % PAGE_SIZE
+            else:
+                phys = seq_row0[i] + pos
+            kf[phys] *= np.float32(3.0)
+    kidx = encode_e4m3(kf)
+    del kf
+    k_scale = None
+    if with_k_scale:
+        # powers of two in [1/4, 4] (e8m0-style block scales)
+        k_scale = np.exp2(_rng(config_id, seed_offset, 5).integers(-2, 3, size=rows)).astype(np.float32)
+
+    # attention query and latent cache (streams 6, 7)
+    q = _normal_bf16(_rng(config_id, seed_offset, 6), (nq, h, D_QK))
+    kv = _normal_bf16(_rng(config_id, seed_offset, 7), (rows, D_QK))
+
+    return Inputs(config_id=config_id, name=c["name"], kind=kind, h_idx=h_idx,
+                  d_idx=d_idx, h=h, d_qk=D_QK, d_v=D_V, topk=k,
+                  scale=float(D_QK) ** -0.5, q_idx=q_idx, w=w, kidx=kidx,
+                  k_scale=k_scale, q=q, kv=kv, q_seq=q_seq, q_n=q_n,
+                  seq_len=seq_len.astype(np.int32), seq_row0=seq_row0,
+                  page_table=page_table, page_size=page_size, q_per_seq=q_per_seq)
+
+
+def to_paged(inp: Inputs, *, config_id: Optional[int] = None, seed_offset: int = 7,
+             page_size: int = PAGE_SIZE) -> Inputs:
+    """The same logical caches re-laid out in pages (random permutation)."""
+    assert inp.page_table is None
+    nseq = inp.nseq
+    pages = (inp.seq_len.astype(np.int64) + page_size - 1) // page_size
+    total = int(pages.sum())
+    perm = _rng(config_id or inp.config_id, seed_offset, 1).permutation(total).astype(np.int32)
+    max_pages = int(pages.max()) if nseq else 1
+    pt = np.full((nseq, max_pages), -1, np.int32)
+    off = 0
+    kidx = np.zeros((total * page_size, inp.d_idx), np.uint8)
+    kv = np.zeros((total * page_size, inp.d_qk), np.uint16)
+    ks = None if inp.k_scale is None else np.ones(total * page_size, np.float32)
+    for i in range(nseq):
+        pt[i, :pages[i]] = perm[off:off + pages[i]]
+        off += int(pages[i])
+        n_i = int(inp.seq_len[i])
+        pos = np.arange(n_i)
+        phys = pt[i, pos // page_size].astype(np.int64) * page_size + pos % page_size
+        src = inp.seq_row0[i] + pos
+        kidx[phys] = inp.kidx[src]
+        kv[phys] = inp.kv[src]
+        if ks is not None:
+            ks[phys] = inp.k_scale[src]
+    return dataclasses.replace(inp, kidx=kidx, kv=kv, k_scale=ks, seq_row0=None,
+                               page_table=pt, page_size=page_size)

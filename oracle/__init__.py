@@ -1,0 +1,216 @@
+"""fp64 CPU oracle for the DSA decode path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
+``bench.py`` may import this package.  The GPU library never imports it, and
+this package imports nothing from the GPU library.
+
+The arithmetic lives in ``dsa_oracle.c`` (plain C, fp64).  This module only
+compiles it with gcc and marshals numpy arrays into its entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsa_oracle.c")
+_LIB = os.path.join(_HERE, "libdsa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+_I64 = ctypes.c_int64
+_F64 = ctypes.c_double
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libdsa_oracle.so`` (gcc, OpenMP).
+
+    -ffp-contract=off keeps every multiply and add separately rounded, so the
+    fp64 sums follow the order written in the C source.
+    """
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        cmd = ["gcc", "-std=c11", "-O2", "-ffp-contract=off", "-fno-fast-math",
+               "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            lib.dsa_oracle_e4m3_to_f64.restype = _F64
+            lib.dsa_oracle_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            lib.dsa_oracle_bf16_to_f64.restype = _F64
+            lib.dsa_oracle_bf16_to_f64.argtypes = [ctypes.c_uint16]
+            lib.dsa_oracle_max_threads.restype = _I32
+            lib.dsa_oracle_indexer_scores.restype = ctypes.c_int
+            lib.dsa_oracle_indexer_scores.argtypes = [
+                _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I32, _I32,
+                _P, _P, _I64, _I32]
+            lib.dsa_oracle_topk.restype = ctypes.c_int
+            lib.dsa_oracle_topk.argtypes = [_I64, _P, _I32, _P, _P]
+            lib.dsa_oracle_sparse_mla.restype = ctypes.c_int
+            lib.dsa_oracle_sparse_mla.argtypes = [
+                _I32, _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P,
+                _I32, _I32, _P, _I32, _P, _P, _I32]
+            lib.dsa_oracle_dense_mla.restype = ctypes.c_int
+            lib.dsa_oracle_dense_mla.argtypes = [
+                _I32, _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P,
+                _I32, _I32, _P, _P, _I32]
+            lib.dsa_oracle_forward.restype = ctypes.c_int
+            lib.dsa_oracle_forward.argtypes = [
+                _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F64, _P, _P, _P, _P,
+                _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32]
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    """Contiguous array of the given dtype (None passes through)."""
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def max_threads() -> int:
+    return int(_load().dsa_oracle_max_threads())
+
+
+def e4m3_to_f64(code: int) -> float:
+    return float(_load().dsa_oracle_e4m3_to_f64(int(code)))
+
+
+def bf16_to_f64(bits: int) -> float:
+    return float(_load().dsa_oracle_bf16_to_f64(int(bits)))
+
+
+def _kv_args(q_seq, q_n, seq_row0, page_table, page_size):
+    q_seq = _c(q_seq, np.int32)
+    q_n = _c(q_n, np.int32)
+    if page_table is not None:
+        page_table = _c(page_table, np.int32)
+        if page_table.ndim != 2:
+            raise ValueError("page_table must be [nseq, max_pages]")
+        return q_seq, q_n, None, page_table, page_table.shape[1], int(page_size)
+    return q_seq, q_n, _c(seq_row0, np.int64), None, 0, 0
+
+
+def indexer_scores(q_idx, w, kidx, q_seq, q_n, *, seq_row0=None, page_table=None,
+                   page_size=0, k_scale=None, ld=None, with_abs=False, nthreads=0):
+    """I[q, s] for s < q_n[q] (fp64); -inf beyond.  Shapes:
+    q_idx [nq, H_I, d_I] uint8 (e4m3 codes), w [nq, H_I] uint16 (bf16 bits),
+    kidx [rows, d_I] uint8, k_scale [rows] float32 or None."""
+    q_idx = _c(q_idx, np.uint8)
+    nq, h_idx, d_idx = q_idx.shape
+    w = _c(w, np.uint16)
+    kidx = _c(kidx, np.uint8)
+    k_scale = _c(k_scale, np.float32)
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    if ld is None:
+        ld = int(q_n.max()) if nq else 0
+    scores = np.empty((nq, ld), np.float64)
+    absv = np.empty((nq, ld), np.float64) if with_abs else None
+    rc = _load().dsa_oracle_indexer_scores(
+        nq, h_idx, d_idx, _ptr(q_idx), _ptr(w), _ptr(kidx), _ptr(k_scale),
+        _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+        page_size, _ptr(scores), _ptr(absv), ld, nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_indexer_scores failed: %d" % rc)
+    return (scores, absv) if with_abs else scores
+
+
+def topk(scores, k, n=None):
+    """Selected positions (rank order) padded with -1 to length k, and nsel."""
+    scores = _c(scores, np.float64)
+    if n is None:
+        n = scores.shape[0]
+    idx = np.empty(k, np.int32)
+    nsel = np.zeros(1, np.int32)
+    rc = _load().dsa_oracle_topk(int(n), _ptr(scores), int(k), _ptr(idx), _ptr(nsel))
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_topk failed: %d" % rc)
+    return idx, int(nsel[0])
+
+
+def sparse_mla(q, kv, idx, q_seq, q_n, *, scale, d_v=512, seq_row0=None,
+               page_table=None, page_size=0, nthreads=0):
+    """out [nq, H, d_v] fp64, lse [nq, H] fp64.  q [nq, H, d_qk] uint16,
+    kv [rows, d_qk] uint16 (bf16 bits), idx [nq, k] int32."""
+    q = _c(q, np.uint16)
+    nq, h, d_qk = q.shape
+    kv = _c(kv, np.uint16)
+    idx = _c(idx, np.int32)
+    k = idx.shape[1] if idx.ndim == 2 else 0
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    out = np.empty((nq, h, d_v), np.float64)
+    lse = np.empty((nq, h), np.float64)
+    rc = _load().dsa_oracle_sparse_mla(
+        nq, h, d_qk, d_v, float(scale), _ptr(q), _ptr(kv), kv.shape[1],
+        _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+        page_size, _ptr(idx), k, _ptr(out), _ptr(lse), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_sparse_mla failed: %d" % rc)
+    return out, lse
+
+
+def dense_mla(q, kv, q_seq, q_n, *, scale, d_v=512, seq_row0=None,
+              page_table=None, page_size=0, nthreads=0):
+    """Textbook attention over all visible positions (no index list)."""
+    q = _c(q, np.uint16)
+    nq, h, d_qk = q.shape
+    kv = _c(kv, np.uint16)
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    out = np.empty((nq, h, d_v), np.float64)
+    lse = np.empty((nq, h), np.float64)
+    rc = _load().dsa_oracle_dense_mla(
+        nq, h, d_qk, d_v, float(scale), _ptr(q), _ptr(kv), kv.shape[1],
+        _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+        page_size, _ptr(out), _ptr(lse), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_dense_mla failed: %d" % rc)
+    return out, lse
+
+
+def forward(q_idx, w, kidx, q, kv, q_seq, q_n, *, k, scale, d_v=512,
+            seq_row0=None, page_table=None, page_size=0, k_scale=None,
+            nthreads=0):
+    """Score -> TopK -> sparse attention.  Returns (idx [nq,k], out, lse)."""
+    q_idx = _c(q_idx, np.uint8)
+    nq, h_idx, d_idx = q_idx.shape
+    w = _c(w, np.uint16)
+    kidx = _c(kidx, np.uint8)
+    k_scale = _c(k_scale, np.float32)
+    q = _c(q, np.uint16)
+    _, h, d_qk = q.shape
+    kv = _c(kv, np.uint16)
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    idx = np.empty((nq, k), np.int32)
+    out = np.empty((nq, h, d_v), np.float64)
+    lse = np.empty((nq, h), np.float64)
+    rc = _load().dsa_oracle_forward(
+        nq, h_idx, d_idx, h, d_qk, d_v, int(k), float(scale), _ptr(q_idx),
+        _ptr(w), _ptr(kidx), _ptr(k_scale), _ptr(q), _ptr(kv), kv.shape[1],
+        _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+        page_size, _ptr(idx), _ptr(out), _ptr(lse), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_forward failed: %d" % rc)
+    return idx, out, lse

@@ -1,0 +1,399 @@
+/*
+ * dsa_oracle.c -- plain, slow fp64 CPU oracle for the DeepSeek Sparse Attention
+ * (DSA) decode path: lightning-indexer scores, per-query TopK, and sparse
+ * MQA-mode MLA attention over the selected latent rows.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the package smoke check and
+ * the benchmark's CPU-baseline leg may load this library.  The GPU library
+ * shares no code with it and never calls it.
+ *
+ * Every function is the plain definition of one step, written in the pages'
+ * notation, with no blocking, fusion or reordering beyond what the definition
+ * states.  Loops over independent outputs may run in parallel (OpenMP); every
+ * single output is summed in a fixed sequential order.
+ *
+ * Sources (web pages on DeepSeek-V3.2 DSA):
+ *   [marsggbo]  "arXiv'25 | DSA lets DeepSeek-V3.2's long-context attention read
+ *               less KV" (marsggbo.github.io), section 2 (toy example),
+ *               section 3 (index score, TopK and attention equations),
+ *               section 4 (MQA mode).
+ *   [yuyanqi]   "DeepSeekV3.2之DSA" (yuyanqi.com), section 3.1 (symbol table),
+ *               section 3.3 (TopK and the short-history rule), section 4.3
+ *               (FP8 kernel comment: fp8 q.k -> relu * weights -> head sum ->
+ *               * k_s), section 4.4 (topk(min(topk, end_pos)) returns indices),
+ *               section 4.5 (skip scoring when the history fits in k),
+ *               section 5.1 (softmax(q.[c_kv; k_pe]^T).c_kv).
+ *
+ * Where the pages leave a step open, the reading taken is stated at the
+ * function.  Parity is pinned by the tests under tests/ (toy example, brute
+ * force, closed forms, library routines), not by this file.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------- */
+/* Number formats                                                              */
+/* ------------------------------------------------------------------------- */
+
+/* FP8 E4M3 as used by the indexer ("FP8" in [marsggbo] section 3 and the
+ * e4m3 operands of the kernel comment in [yuyanqi] section 4.3).  Decoded from
+ * the OCP 8-bit floating point definition of E4M3: 1 sign bit, 4 exponent bits
+ * with bias 7, 3 mantissa bits; exponent field 0 is subnormal
+ * (value = mantissa * 2^-9); exponent 15 with mantissa 7 is NaN; there are no
+ * infinities, so the largest finite magnitude is 1.75 * 2^8 = 448. */
+double dsa_oracle_e4m3_to_f64(uint8_t code)
+{
+    int sign = (code >> 7) & 1;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);               /* m/8 * 2^(1-7) */
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* bfloat16: the upper 16 bits of an IEEE-754 binary32.  Widening is exact. */
+double dsa_oracle_bf16_to_f64(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Where logical position s of a query's history lives in a cache              */
+/* ------------------------------------------------------------------------- */
+
+/* Both caches (the FP8 index-K cache and the bf16 latent cache) are indexed by
+ * the same token positions ([yuyanqi] section 5.2, item 3).  A query q belongs
+ * to sequence q_seq[q]; position s of that sequence is
+ *   contiguous layout: row seq_row0[seq] + s
+ *   paged layout:      row page_table[seq][s / page_size] * page_size
+ *                          + s % page_size
+ * (paged KV as named in [yuyanqi] section 4.4, "_get_topk_paged"). */
+static int64_t cache_row(int32_t seq, int64_t s, const int64_t *seq_row0,
+                         const int32_t *page_table, int32_t max_pages,
+                         int32_t page_size)
+{
+    if (page_table != NULL) {
+        int64_t page = page_table[(int64_t)seq * max_pages + s / page_size];
+        return page * page_size + s % page_size;
+    }
+    return seq_row0[seq] + s;
+}
+
+static void set_threads(int32_t nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int32_t dsa_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 1: lightning-indexer score                                             */
+/* ------------------------------------------------------------------------- */
+
+/* I[t,s] = sum_{j=1..H_I} w[t,j] * ReLU(q^I[t,j] . k^I[s])
+ *   -- the index-score equation of [marsggbo] section 3, with the symbol
+ *      table of [yuyanqi] section 3.1 (k^I has one head shared by all H_I
+ *      indexer heads; w comes from the query token).
+ * The FP8 kernel of [yuyanqi] section 4.3 multiplies the head sum by a
+ * per-key dequantisation scale k_s; k_scale[row] plays that role here
+ * (NULL means 1).
+ * Reading taken: w is used exactly as given (every constant factor of
+ * [yuyanqi] section 4.3 -- n_heads^-1/2, q scale, d_I^-1/2 -- is already folded
+ * into it by the caller); no further scale is applied.
+ *
+ * Output: scores[q*ld + s] for s < q_n[q]; entries q_n[q] <= s < ld are -inf.
+ * abs_scores (optional) receives sum_j |w| * ReLU(q.k) * |k_s|, the magnitude
+ * against which a rounding error of the sum is measured. */
+int dsa_oracle_indexer_scores(int32_t nq, int32_t h_idx, int32_t d_idx,
+                              const uint8_t *q_idx, const uint16_t *w,
+                              const uint8_t *kidx, const float *k_scale,
+                              const int32_t *q_seq, const int32_t *q_n,
+                              const int64_t *seq_row0,
+                              const int32_t *page_table, int32_t max_pages,
+                              int32_t page_size, double *scores,
+                              double *abs_scores, int64_t ld, int32_t nthreads)
+{
+    if (nq < 0 || h_idx <= 0 || d_idx <= 0 || ld < 0) return -1;
+    for (int32_t q = 0; q < nq; ++q)
+        if (q_n[q] < 0 || q_n[q] > ld) return -1;
+    set_threads(nthreads);
+
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int32_t q = 0; q < nq; ++q) {
+        for (int64_t s = 0; s < ld; ++s) {
+            double *out = &scores[(int64_t)q * ld + s];
+            double *aout = abs_scores ? &abs_scores[(int64_t)q * ld + s] : NULL;
+            if (s >= q_n[q]) {
+                *out = -INFINITY;
+                if (aout) *aout = 0.0;
+                continue;
+            }
+            int64_t row = cache_row(q_seq[q], s, seq_row0, page_table,
+                                    max_pages, page_size);
+            const uint8_t *k = kidx + row * (int64_t)d_idx;
+            double ks = k_scale ? (double)k_scale[row] : 1.0;
+            double total = 0.0, total_abs = 0.0;
+            for (int32_t j = 0; j < h_idx; ++j) {
+                const uint8_t *qj = q_idx + ((int64_t)q * h_idx + j) * d_idx;
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_idx; ++d)
+                    dot += dsa_oracle_e4m3_to_f64(qj[d]) *
+                           dsa_oracle_e4m3_to_f64(k[d]);
+                double relu = dot > 0.0 ? dot : 0.0;
+                double wj = dsa_oracle_bf16_to_f64(w[(int64_t)q * h_idx + j]);
+                total += wj * relu;
+                total_abs += fabs(wj) * relu;
+            }
+            *out = total * ks;
+            if (aout) *aout = total_abs * fabs(ks);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 2: TopK with the short-history rule                                    */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    double score;
+    int64_t pos;
+} scored_pos;
+
+/* Larger score first; among equal scores the lower position first
+ * (the tie rule: lower index wins). -0.0 and +0.0 compare equal. */
+static int by_score_then_pos(const void *a, const void *b)
+{
+    const scored_pos *x = (const scored_pos *)a, *y = (const scored_pos *)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    if (x->pos < y->pos) return -1;
+    if (x->pos > y->pos) return 1;
+    return 0;
+}
+
+/* I_t = TopK(I[t, s] over the visible history) -- [marsggbo] section 3; the
+ * positions, not the scores, are the result ([yuyanqi] section 4.4,
+ * "topk(...)[1]").  When the history has at most k positions every position
+ * is kept ([yuyanqi] section 3.3 and section 4.5; topk(min(topk, end_pos))).
+ *
+ * n positions 0..n-1 with scores[0..n-1]; writes idx[0..k-1]: the min(k, n)
+ * selected positions in rank order (score descending, position ascending),
+ * then -1.  *nsel (optional) = min(k, n).  A full sort is used. */
+int dsa_oracle_topk(int64_t n, const double *scores, int32_t k, int32_t *idx,
+                    int32_t *nsel)
+{
+    if (n < 0 || k <= 0) return -1;
+    int64_t keep = n < k ? n : k;
+    if (n <= k) {
+        for (int64_t i = 0; i < n; ++i) idx[i] = (int32_t)i;
+    } else {
+        scored_pos *all = (scored_pos *)malloc((size_t)n * sizeof(scored_pos));
+        if (!all) return -2;
+        for (int64_t s = 0; s < n; ++s) {
+            all[s].score = scores[s];
+            all[s].pos = s;
+        }
+        qsort(all, (size_t)n, sizeof(scored_pos), by_score_then_pos);
+        for (int64_t i = 0; i < keep; ++i) idx[i] = (int32_t)all[i].pos;
+        free(all);
+    }
+    for (int64_t i = keep; i < k; ++i) idx[i] = -1;
+    if (nsel) *nsel = (int32_t)keep;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Step 3: sparse MQA-mode MLA attention over the selected latent rows          */
+/* ------------------------------------------------------------------------- */
+
+/* u_t = Attn(h_t, {c_s : s in I_t})            -- [marsggbo] section 3
+ * In MQA mode every query head shares the one latent row c_s
+ * ([marsggbo] section 4).  With weight absorption the attention is
+ * softmax(q . [c_kv; k_pe]^T) . c_kv ([yuyanqi] section 5.1): the key is the
+ * whole d_qk-wide row (512 latent + 64 rope), the value its first d_v columns.
+ *
+ * For every query q and head h, with the valid entries s_i of idx[q, :]
+ * (entries that are -1 or >= q_n[q] are skipped; a position listed twice is
+ * counted twice):
+ *   S_i   = scale * sum_{d < d_qk} q[q,h,d] * c[s_i, d]
+ *   m     = max_i S_i
+ *   out   = sum_i exp(S_i - m) * c[s_i, 0:d_v] / sum_i exp(S_i - m)
+ *   lse   = m + ln sum_i exp(S_i - m)
+ * With no valid entry: out = 0 and lse = -inf.
+ * kv row r starts at kv + r * kv_row_stride (elements). */
+int dsa_oracle_sparse_mla(int32_t nq, int32_t h, int32_t d_qk, int32_t d_v,
+                          double scale, const uint16_t *q, const uint16_t *kv,
+                          int64_t kv_row_stride, const int32_t *q_seq,
+                          const int32_t *q_n, const int64_t *seq_row0,
+                          const int32_t *page_table, int32_t max_pages,
+                          int32_t page_size, const int32_t *idx, int32_t k,
+                          double *out, double *lse, int32_t nthreads)
+{
+    if (nq < 0 || h <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk || k < 0)
+        return -1;
+    set_threads(nthreads);
+    int bad = 0;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) reduction(| : bad)
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        for (int32_t hh = 0; hh < h; ++hh) {
+            const uint16_t *qv = q + ((int64_t)qi * h + hh) * d_qk;
+            double *o = out + ((int64_t)qi * h + hh) * d_v;
+            double *S = (double *)malloc((size_t)(k > 0 ? k : 1) * sizeof(double));
+            int64_t *rows = (int64_t *)malloc((size_t)(k > 0 ? k : 1) * sizeof(int64_t));
+            if (!S || !rows) { bad |= 1; free(S); free(rows); continue; }
+            int32_t cnt = 0;
+            for (int32_t i = 0; i < k; ++i) {
+                int32_t s = idx[(int64_t)qi * k + i];
+                if (s < 0 || s >= q_n[qi]) continue;
+                rows[cnt++] = cache_row(q_seq[qi], s, seq_row0, page_table,
+                                        max_pages, page_size);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] = 0.0;
+            if (cnt == 0) {
+                lse[(int64_t)qi * h + hh] = -INFINITY;
+                free(S); free(rows);
+                continue;
+            }
+            double m = -INFINITY;
+            for (int32_t i = 0; i < cnt; ++i) {
+                const uint16_t *c = kv + rows[i] * kv_row_stride;
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_qk; ++d)
+                    dot += dsa_oracle_bf16_to_f64(qv[d]) * dsa_oracle_bf16_to_f64(c[d]);
+                S[i] = scale * dot;
+                if (S[i] > m) m = S[i];
+            }
+            double denom = 0.0;
+            for (int32_t i = 0; i < cnt; ++i) {
+                double p = exp(S[i] - m);
+                const uint16_t *c = kv + rows[i] * kv_row_stride;
+                denom += p;
+                for (int32_t d = 0; d < d_v; ++d) o[d] += p * dsa_oracle_bf16_to_f64(c[d]);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] /= denom;
+            lse[(int64_t)qi * h + hh] = m + log(denom);
+            free(S);
+            free(rows);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/* Dense attention over the whole visible history 0..q_n-1, with no index
+ * list: the textbook MQA softmax attention.  When the history has at most k
+ * positions DSA keeps all of them ([yuyanqi] section 3.3), so the sparse path
+ * must reproduce this. */
+int dsa_oracle_dense_mla(int32_t nq, int32_t h, int32_t d_qk, int32_t d_v,
+                         double scale, const uint16_t *q, const uint16_t *kv,
+                         int64_t kv_row_stride, const int32_t *q_seq,
+                         const int32_t *q_n, const int64_t *seq_row0,
+                         const int32_t *page_table, int32_t max_pages,
+                         int32_t page_size, double *out, double *lse,
+                         int32_t nthreads)
+{
+    if (nq < 0 || h <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk) return -1;
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) reduction(| : bad)
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        for (int32_t hh = 0; hh < h; ++hh) {
+            int64_t n = q_n[qi];
+            const uint16_t *qv = q + ((int64_t)qi * h + hh) * d_qk;
+            double *o = out + ((int64_t)qi * h + hh) * d_v;
+            for (int32_t d = 0; d < d_v; ++d) o[d] = 0.0;
+            if (n <= 0) { lse[(int64_t)qi * h + hh] = -INFINITY; continue; }
+            double *logit = (double *)malloc((size_t)n * sizeof(double));
+            if (!logit) { bad |= 1; continue; }
+            for (int64_t s = 0; s < n; ++s) {
+                const uint16_t *c = kv + cache_row(q_seq[qi], s, seq_row0, page_table,
+                                                   max_pages, page_size) * kv_row_stride;
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_qk; ++d)
+                    dot += dsa_oracle_bf16_to_f64(qv[d]) * dsa_oracle_bf16_to_f64(c[d]);
+                logit[s] = scale * dot;
+            }
+            double m = logit[0];
+            for (int64_t s = 1; s < n; ++s) if (logit[s] > m) m = logit[s];
+            double z = 0.0;
+            for (int64_t s = 0; s < n; ++s) {
+                const uint16_t *c = kv + cache_row(q_seq[qi], s, seq_row0, page_table,
+                                                   max_pages, page_size) * kv_row_stride;
+                double p = exp(logit[s] - m);
+                z += p;
+                for (int32_t d = 0; d < d_v; ++d) o[d] += p * dsa_oracle_bf16_to_f64(c[d]);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] /= z;
+            lse[(int64_t)qi * h + hh] = m + log(z);
+            free(logit);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* The three steps composed (one decode step of the attention layer)           */
+/* ------------------------------------------------------------------------- */
+
+/* Score -> TopK -> sparse attention, in the order of the decode data flow of
+ * [yuyanqi] section 5.1.  A query whose history fits in k skips scoring and
+ * keeps every position ([yuyanqi] section 4.5).  idx_out: [nq, k]. */
+int dsa_oracle_forward(int32_t nq, int32_t h_idx, int32_t d_idx, int32_t h,
+                       int32_t d_qk, int32_t d_v, int32_t k, double scale,
+                       const uint8_t *q_idx, const uint16_t *w,
+                       const uint8_t *kidx, const float *k_scale,
+                       const uint16_t *q, const uint16_t *kv,
+                       int64_t kv_row_stride, const int32_t *q_seq,
+                       const int32_t *q_n, const int64_t *seq_row0,
+                       const int32_t *page_table, int32_t max_pages,
+                       int32_t page_size, int32_t *idx_out, double *out,
+                       double *lse, int32_t nthreads)
+{
+    if (nq < 0 || k <= 0) return -1;
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        int64_t n = q_n[qi];
+        int32_t *row_idx = idx_out + (int64_t)qi * k;
+        if (n <= k) {
+            if (dsa_oracle_topk(n, NULL, k, row_idx, NULL) != 0) return -1;
+            continue;
+        }
+        double *sc = (double *)malloc((size_t)n * sizeof(double));
+        if (!sc) return -2;
+        int rc = dsa_oracle_indexer_scores(1, h_idx, d_idx,
+                                           q_idx + (int64_t)qi * h_idx * d_idx,
+                                           w + (int64_t)qi * h_idx, kidx, k_scale,
+                                           q_seq + qi, q_n + qi, seq_row0,
+                                           page_table, max_pages, page_size, sc,
+                                           NULL, n, nthreads);
+        if (rc == 0) rc = dsa_oracle_topk(n, sc, k, row_idx, NULL);
+        free(sc);
+        if (rc != 0) return rc;
+    }
+    return dsa_oracle_sparse_mla(nq, h, d_qk, d_v, scale, q, kv, kv_row_stride,
+                                 q_seq, q_n, seq_row0, page_table, max_pages,
+                                 page_size, idx_out, k, out, lse, nthreads);
+}
