@@ -1,0 +1,224 @@
+/*
+ * dsa.h -- C ABI of the B200 (sm_100a) DeepSeek Sparse Attention decode path.
+ *
+ * The path has three steps (DSA blog by marsggbo, section 3; "DeepSeekV3.2之DSA"
+ * by yuyanqi, sections 3-5):
+ *   1. lightning-indexer score  I[t,s] = sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])
+ *   2. per-query TopK of I[t, 0..n-1]; every position when n <= k
+ *   3. MQA-mode MLA attention of all query heads over the selected latent rows,
+ *      softmax(q . [c_kv; k_pe]^T) . c_kv
+ *
+ * Conventions shared by every call
+ *   - Pointers.  Every tensor argument is a DEVICE pointer owned by the caller.
+ *     The library allocates no device memory; scratch comes from the caller's
+ *     `ws` buffer of at least dsa_workspace_size() bytes, 256-byte aligned.
+ *     `dsa_params` and `dsa_kv` themselves are host structs (their pointer
+ *     members are device pointers).
+ *   - Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy
+ *     default stream).  Calls only enqueue work and return; nothing
+ *     synchronises implicitly.
+ *   - Errors.  Every call returns a dsa_status.  Host-side validation failures
+ *     launch nothing.  Problems only the device can see (an index >= n, a
+ *     bounded wait that expired) are recorded in a status word inside `ws`;
+ *     dsa_check_status() synchronises the stream and returns (then clears) it.
+ *     dsa_last_error() gives a thread-local message for the last failure.
+ *   - Threads.  Calls are stateless and re-entrant; concurrent calls must use
+ *     distinct workspaces.
+ *   - Layouts.  Row-major, innermost dimension last, densely packed unless a
+ *     stride argument says otherwise.  FP8 is OCP E4M3 ("fn": max 448, no inf),
+ *     bf16 is the upper half of binary32.
+ */
+#ifndef DSA_B200_H
+#define DSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = -1,  /* a pointer, size or shape is invalid; nothing launched */
+    DSA_ERR_UNSUPPORTED = -2,  /* valid but outside what this build implements */
+    DSA_ERR_CUDA = -3,         /* a CUDA runtime/driver call failed */
+    DSA_ERR_WORKSPACE = -4,    /* ws is NULL, misaligned or smaller than required */
+    DSA_ERR_TIMEOUT = -5,      /* device: a bounded wait expired (the work was abandoned) */
+    DSA_ERR_DEVICE_CHECK = -6  /* device: an input failed a check (e.g. index >= n) */
+} dsa_status;
+
+/* Problem shape.
+ *   nq         query tokens in the batch (>= 0)
+ *   h_idx      indexer heads H_I, 1..64 ("index_n_heads", yuyanqi section 3.1)
+ *   d_idx      indexer head dim d_I: 64 or 128
+ *   h          attention heads, 1..128 (all share one latent row: MQA mode,
+ *              marsggbo section 4)
+ *   d_qk       key width: 576 (512 latent + 64 rope, yuyanqi section 5.1)
+ *   d_v        value width: 512 (the first d_v columns of the same row)
+ *   topk       k, 1..2048 (DeepSeek-V3.2 uses 2048, marsggbo section 3)
+ *   max_n      an upper bound of every q_n (host-known; sizes the launch grid
+ *              and the workspace); 0 <= q_n[i] <= max_n <= 2^27
+ *   q_per_seq  queries are in blocks of q_per_seq consecutive queries that
+ *              read the same sequence (1 for plain decode, 2 for next token +
+ *              one speculative token, L for a prefill of L tokens); the
+ *              indexer shares each k^I tile among the queries of a block
+ *   scale      softmax scale applied to q . c (576^-0.5 in the workloads)
+ */
+typedef struct {
+    int32_t nq;
+    int32_t h_idx;
+    int32_t d_idx;
+    int32_t h;
+    int32_t d_qk;
+    int32_t d_v;
+    int32_t topk;
+    int32_t max_n;
+    int32_t q_per_seq;
+    float scale;
+} dsa_params;
+
+/* Where each query's history lives.  The FP8 index-K cache and the bf16
+ * latent cache are indexed by the same token positions (yuyanqi section 5.2,
+ * item 3): logical position s of sequence b is cache row
+ *   contiguous (page_table == NULL):  seq_row0[b] + s
+ *   paged      (page_table != NULL):  page_table[b * max_pages + s / page_size]
+ *                                        * page_size + s % page_size
+ *   q_seq      [nq] int32, device: sequence of each query
+ *   q_n        [nq] int32, device: visible positions n of each query; the
+ *              query sees positions 0..n-1 (s < t of marsggbo section 3 when
+ *              the caller sets n = t)
+ *   seq_row0   [nseq] int64, device (contiguous layout) or NULL
+ *   page_table [nseq, max_pages] int32, device (paged layout) or NULL
+ *   max_pages  columns of page_table
+ *   page_size  tokens per page: 64 or 128 (paged layout); ignored otherwise
+ *   cache_rows rows in each cache (bounds every cache access)
+ */
+typedef struct {
+    const int32_t *q_seq;
+    const int32_t *q_n;
+    const int64_t *seq_row0;
+    const int32_t *page_table;
+    int32_t max_pages;
+    int32_t page_size;
+    int64_t cache_rows;
+} dsa_kv;
+
+/* Operation selector for dsa_workspace_size(). */
+typedef enum {
+    DSA_OP_INDEXER_SCORES = 0,
+    DSA_OP_TOPK = 1,
+    DSA_OP_INDEXER_TOPK = 2,
+    DSA_OP_SPARSE_MLA_DECODE = 3,
+    DSA_OP_SPARSE_MLA_PREFILL = 4,
+    DSA_OP_FORWARD = 5
+} dsa_op;
+
+/* Bytes of scratch `ws` the given operation needs for this shape (host only,
+ * no CUDA call).  `kv` may be NULL for DSA_OP_TOPK.  Returns
+ * DSA_ERR_INVALID_ARG for a shape the operation rejects. */
+int dsa_workspace_size(const dsa_params *p, const dsa_kv *kv, int op, size_t *bytes);
+
+/* Step 1 alone: the lightning-indexer score of every visible position,
+ * written to HBM (index-score equation, marsggbo section 3; FP8 kernel
+ * comment of yuyanqi section 4.3: fp8 q.k -> fp32 logits, ReLU, * weights,
+ * sum over heads, * k_s).
+ *   q_idx      [nq, h_idx, d_idx] e4m3
+ *   w          [nq, h_idx] bf16; every constant factor (H_I^-1/2, the q
+ *              quantisation scale, d_I^-1/2; yuyanqi section 4.3) must already
+ *              be folded in: the library applies none
+ *   kidx_cache [cache_rows, d_idx] e4m3 index-K cache (one head shared by all
+ *              indexer heads), rows 16-byte aligned
+ *   k_scale    [cache_rows] fp32 per-row dequantisation scale, or NULL (= 1)
+ *   scores     [nq, ld_scores] fp32 output: scores[i, s] for s < q_n[i];
+ *              -inf for q_n[i] <= s < ld_scores.  ld_scores >= max_n.
+ * Arithmetic: FP8 products are exact; the d_I-term dot products are
+ * accumulated in fp32 by the tensor cores; ReLU, * w and the head sum in fp32. */
+int dsa_indexer_scores(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
+                       const void *w, const void *kidx_cache, const float *k_scale,
+                       float *scores, int64_t ld_scores, void *ws, size_t ws_bytes,
+                       void *stream);
+
+/* Step 2 alone: per-query TopK of scores already in HBM (marsggbo section 3;
+ * indices, not values, as in yuyanqi section 4.4).  For query i with n = q_n[i]:
+ * if n <= topk the result is every position 0..n-1 (yuyanqi section 3.3);
+ * otherwise the topk positions with the largest score, ties broken toward
+ * the lower position.  -0.0 and +0.0 are equal.  Scores must not be NaN.
+ *   scores  [nq, ld_scores] fp32 (entries s >= q_n[i] are not read)
+ *   q_n     [nq] int32 device
+ *   idx     [nq, topk] int32 output: the min(topk, n) selected positions in
+ *           unspecified order, then -1
+ *   nsel    [nq] int32 output min(topk, n), or NULL
+ * The result is exact: identical scores give identical sets. */
+int dsa_topk(const dsa_params *p, const float *scores, int64_t ld_scores,
+             const int32_t *q_n, int32_t *idx, int32_t *nsel, void *ws,
+             size_t ws_bytes, void *stream);
+
+/* Steps 1 + 2 fused: the scores of a query never leave on-chip memory; only
+ * the selected positions reach HBM (the fused logits + TopK path of yuyanqi
+ * section 4.4).  Queries with q_n <= topk skip scoring (yuyanqi section 4.5).
+ * Arguments as dsa_indexer_scores and dsa_topk.  The selected set is the one
+ * dsa_topk returns on the scores dsa_indexer_scores writes, bit for bit. */
+int dsa_indexer_topk(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
+                     const void *w, const void *kidx_cache, const float *k_scale,
+                     int32_t *idx, int32_t *nsel, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/* Step 3: sparse MQA-mode MLA attention (u_t = Attn(h_t, {c_s : s in I_t}),
+ * marsggbo section 3; softmax(q . [c_kv; k_pe]^T) . c_kv, yuyanqi section 5.1).
+ * For every query i and head h, over the valid entries s of idx[i, :]:
+ *   S_s = scale * q[i,h,:] . c[s, 0:d_qk];   P = softmax(S)
+ *   out[i,h,:] = sum_s P_s c[s, 0:d_v];      lse[i,h] = ln sum_s exp(S_s)
+ *   q            [nq, h, d_qk] bf16
+ *   kv_cache     latent cache, bf16 rows of d_qk values, row r at element
+ *                offset r * kv_row_stride (kv_row_stride >= d_qk, multiple of 8)
+ *   idx          [nq, topk] int32 logical positions; -1 entries are skipped;
+ *                entries >= q_n[i] are skipped and flag DSA_ERR_DEVICE_CHECK;
+ *                a position listed twice counts twice
+ *   out          [nq, h, d_v] bf16;  lse [nq, h] fp32 (natural log)
+ * A query with no valid entry gets out = 0 and lse = -inf.
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation; softmax in
+ * fp32; P rounded to bf16 for the P.V product. */
+int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q,
+                          const void *kv_cache, int64_t kv_row_stride,
+                          const int32_t *idx, void *out, float *lse, void *ws,
+                          size_t ws_bytes, void *stream);
+
+/* Step 3 scheduled for many queries of one sequence (causal prefill, where
+ * token t sees n = t positions).  Same arguments and results as
+ * dsa_sparse_mla_decode. */
+int dsa_sparse_mla_prefill(const dsa_params *p, const dsa_kv *kv, const void *q,
+                           const void *kv_cache, int64_t kv_row_stride,
+                           const int32_t *idx, void *out, float *lse, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/* Steps 1-3 in one call: fused indexer + TopK, then sparse attention, as in
+ * the decode data flow of yuyanqi section 5.1.  idx_out [nq, topk] receives
+ * the selected positions (or NULL: they stay in ws).  Arguments as above;
+ * page_table may be set (paged caches) or NULL (contiguous caches). */
+int dsa_forward(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
+                const void *w, const void *kidx_cache, const float *k_scale,
+                const void *q, const void *kv_cache, int64_t kv_row_stride,
+                void *out, float *lse, int32_t *idx_out, void *ws,
+                size_t ws_bytes, void *stream);
+
+/* dsa_forward over paged caches (sglang's paged TopK path named in yuyanqi
+ * section 4.4): kv->page_table must be non-NULL. */
+int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
+                      const void *w, const void *kidx_cache, const float *k_scale,
+                      const void *q, const void *kv_cache, int64_t kv_row_stride,
+                      void *out, float *lse, int32_t *idx_out, void *ws,
+                      size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, return the device status word stored in `ws`
+ * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK) and clear it. */
+int dsa_check_status(void *ws, void *stream);
+
+/* Message describing the last failure on this thread ("" if none). */
+const char *dsa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_B200_H */

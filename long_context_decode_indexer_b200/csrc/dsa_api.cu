@@ -1,0 +1,578 @@
+// dsa_api.cu -- the C ABI declared in include/dsa.h: argument validation,
+// work planning, workspace carving, TMA descriptor encoding and launches.
+// Every step of the computation runs in the kernels of indexer.cu and
+// sparse_mla.cu; this file only decides shapes and enqueues them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "dsa.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *what) {
+    return fail(DSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- TMA maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+int make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_t inner,
+                uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return DSA_OK;
+}
+
+int num_sms() {
+    static int sms = 0;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess)
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    });
+    return sms;
+}
+
+// --------------------------------------------------------------- validation
+int check_params(const dsa_params *p) {
+    if (!p) return fail(DSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->nq < 0) return fail(DSA_ERR_INVALID_ARG, "nq < 0");
+    if (p->h_idx < 1 || p->h_idx > 64) return fail(DSA_ERR_INVALID_ARG, "h_idx must be in [1, 64]");
+    if (p->d_idx != 64 && p->d_idx != 128) return fail(DSA_ERR_INVALID_ARG, "d_idx must be 64 or 128");
+    if (p->h < 1 || p->h > 128) return fail(DSA_ERR_INVALID_ARG, "h must be in [1, 128]");
+    if (p->d_qk != 576 || p->d_v != 512)
+        return fail(DSA_ERR_UNSUPPORTED, "only d_qk = 576 and d_v = 512 are implemented");
+    if (p->topk < 1 || p->topk > 2048) return fail(DSA_ERR_INVALID_ARG, "topk must be in [1, 2048]");
+    if (p->max_n < 0 || p->max_n > (1 << 27)) return fail(DSA_ERR_INVALID_ARG, "max_n must be in [0, 2^27]");
+    if (p->q_per_seq < 1) return fail(DSA_ERR_INVALID_ARG, "q_per_seq must be >= 1");
+    if (!isfinite(p->scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite");
+    return DSA_OK;
+}
+
+int check_kv(const dsa_params *p, const dsa_kv *kv) {
+    if (!kv) return fail(DSA_ERR_INVALID_ARG, "kv is NULL");
+    if (p->nq > 0 && (!kv->q_seq || !kv->q_n)) return fail(DSA_ERR_INVALID_ARG, "q_seq / q_n are NULL");
+    if ((kv->seq_row0 == nullptr) == (kv->page_table == nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "exactly one of seq_row0 and page_table must be set");
+    if (kv->page_table) {
+        if (kv->page_size != 64 && kv->page_size != 128)
+            return fail(DSA_ERR_UNSUPPORTED, "page_size must be 64 or 128");
+        if (kv->max_pages < 1 || static_cast<int64_t>(kv->max_pages) * kv->page_size < p->max_n)
+            return fail(DSA_ERR_INVALID_ARG, "max_pages * page_size < max_n");
+    }
+    if (kv->cache_rows < 1 || kv->cache_rows >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "cache_rows must be in [1, 2^31)");
+    return DSA_OK;
+}
+
+// ----------------------------------------------------------------- planning
+struct IndexerPlan {
+    int hp, qg, gpb, n_groups, P, chunk;
+    uint32_t tmem_cols;
+    size_t smem;
+};
+
+int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
+    pl.hp = p->h_idx <= 16 ? 16 : 64;
+    if (mode == dsa::kModeTopk) {
+        pl.qg = 1;
+        pl.gpb = 1;
+        pl.n_groups = p->nq;
+    } else {
+        pl.qg = p->q_per_seq < dsa::kMaxGroupQueries ? p->q_per_seq : dsa::kMaxGroupQueries;
+        pl.gpb = (p->q_per_seq + pl.qg - 1) / pl.qg;
+        const int nblocks = (p->nq + p->q_per_seq - 1) / p->q_per_seq;
+        const int64_t ng = static_cast<int64_t>(nblocks) * pl.gpb;
+        if (ng > (int64_t(1) << 24)) return fail(DSA_ERR_UNSUPPORTED, "too many query groups");
+        pl.n_groups = static_cast<int>(ng);
+    }
+    const int64_t sp = span > 0 ? span : 1;
+    int64_t chunk_max;
+    if (mode == dsa::kModeScores)
+        chunk_max = 1 << 20;
+    else
+        chunk_max = (dsa::kKeysBudget / (4 * pl.qg)) / 128 * 128;
+    const int64_t p_min = (sp + chunk_max - 1) / chunk_max;
+    const int64_t p_fill = pl.n_groups > 0 ? (num_sms() / pl.n_groups > 1 ? num_sms() / pl.n_groups : 1) : 1;
+    const int64_t p_small = (sp + 1023) / 1024;  // no chunk below 1024 positions
+    int64_t P = p_fill < p_small ? p_fill : p_small;
+    if (P < p_min) P = p_min;
+    if (P < 1) P = 1;
+    if (mode != dsa::kModeScores) {
+        // the merge list (P * topk composites) must fit on chip
+        const int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
+        if (P > p_cap) {
+            if (p_min > p_cap) return fail(DSA_ERR_UNSUPPORTED, "history too long for topk=%d (max_n=%d)", p->topk, p->max_n);
+            P = p_cap;
+        }
+    }
+    int64_t chunk = (sp + P - 1) / P;
+    chunk = (chunk + 127) / 128 * 128;
+    if (chunk > chunk_max) chunk = chunk_max;
+    P = (sp + chunk - 1) / chunk;
+    pl.P = static_cast<int>(P);
+    pl.chunk = static_cast<int>(chunk);
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(2 * pl.qg * pl.hp)) cols <<= 1;
+    pl.tmem_cols = cols;
+    const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk);
+    pl.smem = L.total;
+    if (pl.smem > 232448) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
+    return DSA_OK;
+}
+
+struct MlaPlan {
+    int splits, rows_per_split, wave;
+};
+
+constexpr size_t kPartialBudget = size_t(1) << 30;  // bytes of split partials per wave
+
+MlaPlan plan_mla(const dsa_params *p) {
+    MlaPlan m;
+    const int k = p->topk;
+    const int s_min = (k + dsa::kMlaMaxRows - 1) / dsa::kMlaMaxRows;
+    int s_fill = p->nq > 0 ? num_sms() / p->nq : 1;
+    const int s_small = (k + 63) / 64;
+    int s = s_fill < s_small ? s_fill : s_small;
+    if (s < s_min) s = s_min;
+    if (s < 1) s = 1;
+    int rps = (k + s - 1) / s;
+    rps = (rps + 15) / 16 * 16;
+    if (rps > dsa::kMlaMaxRows) rps = dsa::kMlaMaxRows;
+    m.rows_per_split = rps;
+    m.splits = (k + rps - 1) / rps;
+    if (m.splits == 1) {
+        m.wave = p->nq;
+    } else {
+        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv + 1) * 4;
+        size_t w = kPartialBudget / per_q;
+        if (w < 1) w = 1;
+        m.wave = p->nq < static_cast<int>(w) ? p->nq : static_cast<int>(w);
+    }
+    return m;
+}
+
+// -------------------------------------------------------------- workspace
+struct WsLayout {
+    size_t status, ghist, cand, cand_cnt, done, idx, part_o, part_lse, total;
+    size_t zero_begin, zero_end;  // cleared at the start of every call
+};
+
+size_t indexer_ws(const dsa_params *p, const IndexerPlan &pl, int mode, size_t off, WsLayout &w) {
+    w.ghist = w.cand = w.cand_cnt = w.done = off;
+    if (mode == dsa::kModeScores || pl.P <= 1) return off;
+    w.zero_begin = off;
+    w.ghist = off;
+    off = up(off + static_cast<size_t>(p->nq) * 2048 * 4, 256);
+    w.done = off;
+    off = up(off + static_cast<size_t>(pl.n_groups) * 4, 256);
+    w.zero_end = off;
+    w.cand = off;
+    off = up(off + static_cast<size_t>(p->nq) * pl.P * p->topk * 8, 256);
+    w.cand_cnt = off;
+    off = up(off + static_cast<size_t>(p->nq) * pl.P * 4, 256);
+    return off;
+}
+
+size_t mla_ws(const dsa_params *p, const MlaPlan &m, size_t off, WsLayout &w) {
+    w.part_o = w.part_lse = off;
+    if (m.splits <= 1) return off;
+    w.part_o = off;
+    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * dsa::kDv * 4, 256);
+    w.part_lse = off;
+    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 4, 256);
+    return off;
+}
+
+int layout_for(const dsa_params *p, int op, WsLayout &w, IndexerPlan *ipl, MlaPlan *mpl,
+               int64_t ld_scores) {
+    memset(&w, 0, sizeof w);
+    size_t off = 256;  // status word
+    w.status = 0;
+    IndexerPlan pl{};
+    MlaPlan m{};
+    int rc;
+    switch (op) {
+    case DSA_OP_INDEXER_SCORES:
+        rc = plan_indexer(p, dsa::kModeScores, ld_scores > p->max_n ? ld_scores : p->max_n, pl);
+        if (rc) return rc;
+        off = indexer_ws(p, pl, dsa::kModeScores, off, w);
+        break;
+    case DSA_OP_TOPK:
+        rc = plan_indexer(p, dsa::kModeTopk, p->max_n, pl);
+        if (rc) return rc;
+        off = indexer_ws(p, pl, dsa::kModeTopk, off, w);
+        break;
+    case DSA_OP_INDEXER_TOPK:
+        rc = plan_indexer(p, dsa::kModeFused, p->max_n, pl);
+        if (rc) return rc;
+        off = indexer_ws(p, pl, dsa::kModeFused, off, w);
+        break;
+    case DSA_OP_SPARSE_MLA_DECODE:
+    case DSA_OP_SPARSE_MLA_PREFILL:
+        m = plan_mla(p);
+        off = mla_ws(p, m, off, w);
+        break;
+    case DSA_OP_FORWARD:
+        rc = plan_indexer(p, dsa::kModeFused, p->max_n, pl);
+        if (rc) return rc;
+        off = indexer_ws(p, pl, dsa::kModeFused, off, w);
+        w.idx = off;
+        off = up(off + static_cast<size_t>(p->nq) * p->topk * 4, 256);
+        m = plan_mla(p);
+        off = mla_ws(p, m, off, w);
+        break;
+    default:
+        return fail(DSA_ERR_INVALID_ARG, "unknown op %d", op);
+    }
+    w.total = off;
+    if (ipl) *ipl = pl;
+    if (mpl) *mpl = m;
+    return DSA_OK;
+}
+
+int check_ws(void *ws, size_t ws_bytes, const WsLayout &w) {
+    if (!ws) return fail(DSA_ERR_WORKSPACE, "ws is NULL");
+    if (!aligned(ws, 256)) return fail(DSA_ERR_WORKSPACE, "ws must be 256-byte aligned");
+    if (ws_bytes < w.total) return fail(DSA_ERR_WORKSPACE, "ws_bytes %zu < required %zu", ws_bytes, w.total);
+    return DSA_OK;
+}
+
+template <class T>
+T *at(void *ws, size_t off) {
+    return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+// ------------------------------------------------------------ enqueue steps
+int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_idx, const void *w,
+                const void *kidx_cache, const float *k_scale, float *scores, int64_t ld,
+                int32_t *idx, int32_t *nsel, void *ws, const WsLayout &wl, const IndexerPlan &pl,
+                cudaStream_t st) {
+    dsa::K1Params a;
+    memset(&a, 0, sizeof a);
+    a.q_idx = static_cast<const uint8_t *>(q_idx);
+    a.w = static_cast<const uint16_t *>(w);
+    a.k_scale = k_scale;
+    a.nq = p->nq;
+    a.h_idx = p->h_idx;
+    a.d_idx = p->d_idx;
+    a.topk = p->topk;
+    a.q_per_seq = p->q_per_seq;
+    a.qg = pl.qg;
+    a.groups_per_block = pl.gpb;
+    a.n_groups = pl.n_groups;
+    a.P = pl.P;
+    a.chunk = pl.chunk;
+    a.tmem_cols = pl.tmem_cols;
+    a.scores = scores;
+    a.ld = ld;
+    a.idx = idx;
+    a.nsel = nsel;
+    a.status = at<int>(ws, wl.status);
+    if (mode != dsa::kModeScores && pl.P > 1) {
+        a.ghist = at<uint32_t>(ws, wl.ghist);
+        a.done = at<uint32_t>(ws, wl.done);
+        a.cand = at<uint64_t>(ws, wl.cand);
+        a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
+        cudaError_t e = cudaMemsetAsync(static_cast<uint8_t *>(ws) + wl.zero_begin, 0,
+                                        wl.zero_end - wl.zero_begin, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    }
+    if (p->nq == 0) return DSA_OK;
+    cudaError_t e;
+    if (mode == dsa::kModeTopk) {
+        a.q_n = kv ? kv->q_n : nullptr;
+        e = dsa::launch_topk(a, st);
+        if (e != cudaSuccess) return cuda_fail(e, "TopK launch");
+        return DSA_OK;
+    }
+    a.q_seq = kv->q_seq;
+    a.q_n = kv->q_n;
+    a.seq_row0 = kv->seq_row0;
+    a.page_table = kv->page_table;
+    a.max_pages = kv->max_pages;
+    a.page_size = kv->page_table ? kv->page_size : 0;
+    a.cache_rows = kv->cache_rows;
+    CUtensorMap kmap;
+    const uint32_t box_rows = kv->page_table ? static_cast<uint32_t>(kv->page_size) : 128u;
+    int rc = make_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, kidx_cache, p->d_idx, kv->cache_rows,
+                         p->d_idx, p->d_idx, box_rows,
+                         p->d_idx == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+    if (rc) return rc;
+    e = dsa::launch_indexer(mode, pl.hp, p->d_idx, kmap, a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
+    return DSA_OK;
+}
+
+int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
+            int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
+            const WsLayout &wl, const MlaPlan &m, cudaStream_t st) {
+    if (p->nq == 0) return DSA_OK;
+    CUtensorMap qmap, kvmap;
+    const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
+    int rc = make_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dsa::kDqk,
+                         static_cast<uint64_t>(p->nq) * p->h, dsa::kDqk * 2, 64, hbox,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    rc = make_map_2d(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_cache, dsa::kDqk, kv->cache_rows,
+                     static_cast<uint64_t>(kv_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    dsa::MlaParams a;
+    memset(&a, 0, sizeof a);
+    a.q_seq = kv->q_seq;
+    a.q_n = kv->q_n;
+    a.seq_row0 = kv->seq_row0;
+    a.page_table = kv->page_table;
+    a.max_pages = kv->max_pages;
+    a.page_size = kv->page_table ? kv->page_size : 0;
+    a.cache_rows = kv->cache_rows;
+    a.idx = idx;
+    a.kv = static_cast<const uint16_t *>(kv_cache);
+    a.kv_row_stride = kv_row_stride;
+    a.nq = p->nq;
+    a.h = p->h;
+    a.topk = p->topk;
+    a.splits = m.splits;
+    a.rows_per_split = m.rows_per_split;
+    a.scale = p->scale;
+    a.scale_log2 = p->scale * 1.4426950408889634f;
+    a.out = static_cast<uint16_t *>(out);
+    a.lse = lse;
+    a.part_o = m.splits > 1 ? at<float>(ws, wl.part_o) : nullptr;
+    a.part_lse = m.splits > 1 ? at<float>(ws, wl.part_lse) : nullptr;
+    a.status = at<int>(ws, wl.status);
+    for (int q0 = 0; q0 < p->nq; q0 += m.wave) {
+        const int nw = (p->nq - q0) < m.wave ? (p->nq - q0) : m.wave;
+        a.q0 = q0;
+        cudaError_t e = dsa::launch_sparse_mla(qmap, kvmap, a, nw, st);
+        if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
+        e = dsa::launch_mla_combine(a, nw, st);
+        if (e != cudaSuccess) return cuda_fail(e, "split combine launch");
+    }
+    return DSA_OK;
+}
+
+int check_indexer_inputs(const dsa_params *p, const void *q_idx, const void *w, const void *kidx) {
+    if (p->nq == 0) return DSA_OK;
+    if (!q_idx || !w || !kidx) return fail(DSA_ERR_INVALID_ARG, "q_idx / w / kidx_cache is NULL");
+    if (!aligned(q_idx, 16) || !aligned(kidx, 16)) return fail(DSA_ERR_INVALID_ARG, "q_idx / kidx_cache must be 16-byte aligned");
+    if (!aligned(w, 2)) return fail(DSA_ERR_INVALID_ARG, "w must be 2-byte aligned");
+    return DSA_OK;
+}
+
+int check_mla_inputs(const dsa_params *p, const void *q, const void *kv_cache, int64_t stride,
+                     const void *idx, const void *out, const void *lse) {
+    if (p->nq == 0) return DSA_OK;
+    if (!q || !kv_cache || !idx || !out || !lse) return fail(DSA_ERR_INVALID_ARG, "q / kv_cache / idx / out / lse is NULL");
+    if (!aligned(q, 16) || !aligned(kv_cache, 16) || !aligned(out, 16))
+        return fail(DSA_ERR_INVALID_ARG, "q / kv_cache / out must be 16-byte aligned");
+    if (stride < 576 || stride % 8 != 0) return fail(DSA_ERR_INVALID_ARG, "kv_row_stride must be >= 576 and a multiple of 8");
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_workspace_size(const dsa_params *p, const dsa_kv *kv, int op, size_t *bytes) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+    if (op != DSA_OP_TOPK) {
+        rc = check_kv(p, kv);
+        if (rc) return rc;
+    }
+    WsLayout w;
+    rc = layout_for(p, op, w, nullptr, nullptr, p->max_n);
+    if (rc) return rc;
+    *bytes = w.total;
+    return DSA_OK;
+}
+
+int dsa_indexer_scores(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,
+                       const void *kidx_cache, const float *k_scale, float *scores, int64_t ld_scores,
+                       void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (!rc) rc = check_indexer_inputs(p, q_idx, w, kidx_cache);
+    if (rc) return rc;
+    if (ld_scores < p->max_n || ld_scores > (int64_t(1) << 27)) return fail(DSA_ERR_INVALID_ARG, "ld_scores must be in [max_n, 2^27]");
+    if (p->nq > 0 && !scores) return fail(DSA_ERR_INVALID_ARG, "scores is NULL");
+    WsLayout wl;
+    IndexerPlan pl;
+    rc = layout_for(p, DSA_OP_INDEXER_SCORES, wl, &pl, nullptr, ld_scores);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    // the score plan covers ld_scores positions
+    rc = plan_indexer(p, dsa::kModeScores, ld_scores > 0 ? ld_scores : 1, pl);
+    if (rc) return rc;
+    return run_indexer(p, kv, dsa::kModeScores, q_idx, w, kidx_cache, k_scale, scores, ld_scores,
+                       nullptr, nullptr, ws, wl, pl, static_cast<cudaStream_t>(stream));
+}
+
+int dsa_topk(const dsa_params *p, const float *scores, int64_t ld_scores, const int32_t *q_n,
+             int32_t *idx, int32_t *nsel, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (rc) return rc;
+    if (p->nq > 0 && (!scores || !q_n || !idx)) return fail(DSA_ERR_INVALID_ARG, "scores / q_n / idx is NULL");
+    if (ld_scores < p->max_n) return fail(DSA_ERR_INVALID_ARG, "ld_scores < max_n");
+    WsLayout wl;
+    IndexerPlan pl;
+    rc = layout_for(p, DSA_OP_TOPK, wl, &pl, nullptr, ld_scores);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    dsa_kv kv;
+    memset(&kv, 0, sizeof kv);
+    kv.q_n = q_n;
+    return run_indexer(p, &kv, dsa::kModeTopk, nullptr, nullptr, nullptr, nullptr,
+                       const_cast<float *>(scores), ld_scores, idx, nsel, ws, wl, pl,
+                       static_cast<cudaStream_t>(stream));
+}
+
+int dsa_indexer_topk(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,
+                     const void *kidx_cache, const float *k_scale, int32_t *idx, int32_t *nsel,
+                     void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (!rc) rc = check_indexer_inputs(p, q_idx, w, kidx_cache);
+    if (rc) return rc;
+    if (p->nq > 0 && !idx) return fail(DSA_ERR_INVALID_ARG, "idx is NULL");
+    WsLayout wl;
+    IndexerPlan pl;
+    rc = layout_for(p, DSA_OP_INDEXER_TOPK, wl, &pl, nullptr, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    return run_indexer(p, kv, dsa::kModeFused, q_idx, w, kidx_cache, k_scale, nullptr, 0, idx, nsel,
+                       ws, wl, pl, static_cast<cudaStream_t>(stream));
+}
+
+static int mla_common(int op, const dsa_params *p, const dsa_kv *kv, const void *q,
+                      const void *kv_cache, int64_t kv_row_stride, const int32_t *idx, void *out,
+                      float *lse, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (!rc) rc = check_mla_inputs(p, q, kv_cache, kv_row_stride, idx, out, lse);
+    if (rc) return rc;
+    WsLayout wl;
+    MlaPlan m;
+    rc = layout_for(p, op, wl, nullptr, &m, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    return run_mla(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, wl, m,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
+                          int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
+                          size_t ws_bytes, void *stream) {
+    return mla_common(DSA_OP_SPARSE_MLA_DECODE, p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws,
+                      ws_bytes, stream);
+}
+
+int dsa_sparse_mla_prefill(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
+                           int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
+                           size_t ws_bytes, void *stream) {
+    return mla_common(DSA_OP_SPARSE_MLA_PREFILL, p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws,
+                      ws_bytes, stream);
+}
+
+int dsa_forward(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,
+                const void *kidx_cache, const float *k_scale, const void *q, const void *kv_cache,
+                int64_t kv_row_stride, void *out, float *lse, int32_t *idx_out, void *ws,
+                size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (!rc) rc = check_indexer_inputs(p, q_idx, w, kidx_cache);
+    if (!rc) rc = check_mla_inputs(p, q, kv_cache, kv_row_stride, q, out, lse);
+    if (rc) return rc;
+    WsLayout wl;
+    IndexerPlan pl;
+    MlaPlan m;
+    rc = layout_for(p, DSA_OP_FORWARD, wl, &pl, &m, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t *idx = idx_out ? idx_out : at<int32_t>(ws, wl.idx);
+    rc = run_indexer(p, kv, dsa::kModeFused, q_idx, w, kidx_cache, k_scale, nullptr, 0, idx, nullptr,
+                     ws, wl, pl, st);
+    if (rc) return rc;
+    return run_mla(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, wl, m, st);
+}
+
+int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,
+                      const void *kidx_cache, const float *k_scale, const void *q,
+                      const void *kv_cache, int64_t kv_row_stride, void *out, float *lse,
+                      int32_t *idx_out, void *ws, size_t ws_bytes, void *stream) {
+    if (!kv || !kv->page_table) return fail(DSA_ERR_INVALID_ARG, "dsa_forward_paged needs kv->page_table");
+    return dsa_forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, out, lse,
+                       idx_out, ws, ws_bytes, stream);
+}
+
+int dsa_check_status(void *ws, void *stream) {
+    if (!ws) return fail(DSA_ERR_WORKSPACE, "ws is NULL");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0;
+    e = cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(status)");
+    if (v != 0) {
+        const int zero = 0;
+        e = cudaMemcpy(ws, &zero, sizeof zero, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(clear status)");
+        fail(v, "device reported status %d", v);
+    }
+    return v;
+}
+
+const char *dsa_last_error(void) { return g_err; }
+
+}  // extern "C"

@@ -1,0 +1,610 @@
+// indexer.cu -- lightning indexer and TopK on sm_100a.
+//
+// Index score (DSA blog by marsggbo, section 3; FP8 kernel comment in
+// "DeepSeekV3.2之DSA" by yuyanqi, section 4.3):
+//   I[t,s] = k_s[s] * sum_j w[t,j] * ReLU(q^I[t,j] . k^I[s])
+// TopK with the short-history rule (marsggbo section 3; yuyanqi sections
+// 3.3, 4.4, 4.5): the min(k, n) largest positions, ties toward the lower one.
+//
+// Work split.  Queries come in groups of up to `qg` that read the same
+// sequence; a group's history [0, span) is cut into P chunks, one CTA each.
+// A CTA streams its chunk of the FP8 index-K cache through a TMA ring, and
+// the tensor cores compute D[128 positions x qg*hp heads] = K_tile . Q^T
+// (tcgen05 kind::f8f6f4, M = 128, N = qg*hp, K = d_I) into TMEM.  Four
+// epilogue warps read D back (one TMEM lane = one position per thread) and
+// apply ReLU, * w, the head sum and * k_s.
+//
+// Fused mode keeps the chunk's scores in shared memory as order-preserving
+// keys.  Exact selection across chunks without a grid barrier:
+//   1. each chunk adds the histogram of its keys' top 11 bits to the query's
+//      global histogram G;
+//   2. it reads G back: any snapshot of G is a lower bound of the final one
+//      bin by bin, so the bin where G's count from the top reaches k is at
+//      most the final threshold bin -- keys in lower bins can never win;
+//   3. it publishes its keys at or above that bin (capped by an exact local
+//      TopK of size k), then bumps the group's done counter;
+//   4. the last CTA of the group takes everything above the final threshold
+//      bin and radix-refines the threshold bin among the candidates.
+// Scores never leave the SM.  With one chunk per group the CTA selects
+// directly.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kTileRows = 128;
+
+struct K1Smem {
+    uint64_t full[kK1Stages];
+    uint64_t empty[kK1Stages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint32_t tmem_base;
+    volatile int32_t abort;
+    int32_t is_last;
+    int32_t n_q[kMaxGroupQueries];
+    uint32_t g_digit[kMaxGroupQueries];  // threshold bin seen in G
+    uint32_t cand_count[kMaxGroupQueries];
+    SelectScratch sel;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// first query and query count of group g
+__device__ __forceinline__ void group_queries(const K1Params &a, int g, int &q0, int &cnt) {
+    const int blk = g / a.groups_per_block, sub = g % a.groups_per_block;
+    q0 = blk * a.q_per_seq + sub * a.qg;
+    int c = a.qg;
+    c = min(c, a.q_per_seq - sub * a.qg);
+    c = min(c, a.nq - q0);
+    cnt = max(c, 0);
+}
+
+// Key of position p's score in the local chunk buffer -> composite.
+struct LocalSrc {
+    const uint32_t *keys;
+    int base;
+    __device__ bool operator()(int i, uint64_t &v) const {
+        v = make_composite(keys[i], static_cast<uint32_t>(base + i));
+        return true;
+    }
+};
+// Candidates staged in shared memory (already composites).
+struct ListSrc {
+    const uint64_t *list;
+    __device__ bool operator()(int i, uint64_t &v) const {
+        v = list[i];
+        return true;
+    }
+};
+
+// Local histogram of the top digit of every key of this chunk.
+__device__ void local_top_hist(const uint32_t *keys, int len, uint32_t *hist) {
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < len; i0 += blockDim.x) {
+        const int i = i0 + threadIdx.x;
+        const bool act = i < len;
+        hist_add(hist, act, act ? top_digit(keys[i]) : 0u);
+    }
+    __syncthreads();
+}
+
+// Everything one query of a chunk does after its keys are in shared memory:
+// direct selection (one chunk), or publishing candidates (several chunks).
+// `keys` holds the chunk's keys for positions [start, start + len).
+__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, const uint32_t *keys,
+                             int start, int len, uint32_t *hist) {
+    const int K = a.topk;
+    const int n = sm.n_q[qi];
+    LocalSrc src{keys, start};
+    if (a.P == 1) {
+        // the whole history is here: n == len > K
+        local_top_hist(keys, len, hist);
+        find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+        const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
+        __syncthreads();
+        const uint32_t need = static_cast<uint32_t>(K) - above;
+        uint64_t thr = (static_cast<uint64_t>(d) << 53);
+        if (bucket != need) thr = radix_refine(src, len, d, 1, need, hist, sm.sel);
+        if (threadIdx.x == 0) sm.sel.counter[0] = 0;
+        __syncthreads();
+        int32_t *out = a.idx + static_cast<int64_t>(q) * K;
+        emit_selected(src, len, [thr](uint64_t v) { return v >= thr; },
+                      [out, K](uint32_t slot, uint64_t v) {
+                          if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
+                      },
+                      sm.sel, 0);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            if (sm.sel.counter[0] != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+            if (a.nsel) a.nsel[q] = K;
+        }
+        (void)n;
+        return;
+    }
+
+    // ---- several chunks: publish this chunk's candidates
+    uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + blockIdx.x % a.P) * K;
+    local_top_hist(keys, len, hist);
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
+        if (hist[b]) atomicAdd(&G[b], hist[b]);
+    __threadfence();
+    __syncthreads();
+    // snapshot of G (a lower bound of the final histogram, bin by bin)
+    uint32_t *snap = hist;
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) snap[b] = __ldcg(&G[b]);
+    __syncthreads();
+    find_digit(snap, kSelBins, static_cast<uint32_t>(K), sm.sel);
+    const uint32_t dlow = sm.sel.res[0];
+    __syncthreads();
+    // how many local keys sit at or above dlow
+    if (threadIdx.x == 0) sm.sel.counter[1] = 0;
+    __syncthreads();
+    {
+        uint32_t c = 0;
+        for (int i = threadIdx.x; i < len; i += blockDim.x) c += (top_digit(keys[i]) >= dlow);
+        c = warp_sum(c);
+        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], c);
+    }
+    __syncthreads();
+    const uint32_t at_or_above = sm.sel.counter[1];
+    uint64_t thr = static_cast<uint64_t>(dlow) << 53;
+    if (at_or_above > static_cast<uint32_t>(K)) {
+        // cap at the exact local TopK: a key beaten by k keys of its own
+        // chunk can never be selected; keep the intersection of both sets
+        local_top_hist(keys, len, hist);
+        find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+        const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
+        __syncthreads();
+        const uint32_t need = static_cast<uint32_t>(K) - above;
+        uint64_t lthr = static_cast<uint64_t>(d) << 53;
+        if (bucket != need) lthr = radix_refine(src, len, d, 1, need, hist, sm.sel);
+        thr = lthr > thr ? lthr : thr;
+    }
+    if (threadIdx.x == 0) sm.sel.counter[0] = 0;
+    __syncthreads();
+    emit_selected(src, len, [thr](uint64_t v) { return v >= thr; },
+                  [cand, K](uint32_t slot, uint64_t v) {
+                      if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
+                  },
+                  sm.sel, 0);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t m = sm.sel.counter[0];
+        if (m > static_cast<uint32_t>(K)) {
+            record_status(a.status, DSA_ERR_DEVICE_CHECK);
+            m = K;
+        }
+        a.cand_cnt[static_cast<int64_t>(q) * a.P + blockIdx.x % a.P] = static_cast<int32_t>(m);
+    }
+    (void)n;
+}
+
+// The last CTA of a group: final selection of query q from all candidates.
+__device__ void group_merge(const K1Params &a, K1Smem &sm, int q, uint32_t *hist, uint64_t *list,
+                            int list_cap) {
+    const int K = a.topk;
+    const uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = __ldcg(&G[b]);
+    __syncthreads();
+    find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+    const uint32_t dstar = sm.sel.res[0], above = sm.sel.res[1];
+    __syncthreads();
+    int32_t *out = a.idx + static_cast<int64_t>(q) * K;
+    if (threadIdx.x == 0) {
+        sm.sel.counter[0] = 0;  // slots in out
+        sm.sel.counter[1] = 0;  // bucket list length
+    }
+    __syncthreads();
+    // pass over all candidates: digit > d* -> selected; digit == d* -> list
+    const uint64_t *cand = a.cand + static_cast<int64_t>(q) * a.P * K;
+    const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * a.P;
+    const int lane = threadIdx.x & 31;
+    for (int c = 0; c < a.P; ++c) {
+        const int m = __ldcg(&cnt[c]);
+        for (int i0 = 0; i0 < m; i0 += blockDim.x) {
+            const int i = i0 + threadIdx.x;
+            uint64_t v = 0;
+            if (i < m) v = __ldcg(&cand[static_cast<int64_t>(c) * K + i]);
+            const uint32_t dg = static_cast<uint32_t>(v >> 53);
+            const bool take = (i < m) && dg > dstar;
+            const bool keep = (i < m) && dg == dstar;
+            unsigned mt = __ballot_sync(0xffffffffu, take);
+            unsigned mk = __ballot_sync(0xffffffffu, keep);
+            uint32_t bt = 0, bk = 0;
+            if (lane == 0) {
+                if (mt) bt = atomicAdd(&sm.sel.counter[0], static_cast<uint32_t>(__popc(mt)));
+                if (mk) bk = atomicAdd(&sm.sel.counter[1], static_cast<uint32_t>(__popc(mk)));
+            }
+            bt = __shfl_sync(0xffffffffu, bt, 0);
+            bk = __shfl_sync(0xffffffffu, bk, 0);
+            const unsigned lt = (1u << lane) - 1u;
+            if (take) {
+                const uint32_t s = bt + __popc(mt & lt);
+                if (s < static_cast<uint32_t>(K)) out[s] = static_cast<int32_t>(composite_pos(v));
+            }
+            if (keep) {
+                const uint32_t s = bk + __popc(mk & lt);
+                if (s < static_cast<uint32_t>(list_cap)) list[s] = v;
+            }
+        }
+    }
+    __syncthreads();
+    const uint32_t taken = sm.sel.counter[0];
+    const uint32_t nlist = sm.sel.counter[1];
+    __syncthreads();
+    if (taken != above || nlist > static_cast<uint32_t>(list_cap) ||
+        nlist < static_cast<uint32_t>(K) - above) {
+        if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        return;
+    }
+    const uint32_t need = static_cast<uint32_t>(K) - above;
+    ListSrc src{list};
+    uint64_t thr = static_cast<uint64_t>(dstar) << 53;
+    if (nlist != need) thr = radix_refine(src, static_cast<int>(nlist), dstar, 1, need, hist, sm.sel);
+    emit_selected(src, static_cast<int>(nlist), [thr](uint64_t v) { return v >= thr; },
+                  [out, K](uint32_t slot, uint64_t v) {
+                      if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
+                  },
+                  sm.sel, 0);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (sm.sel.counter[0] != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        if (a.nsel) a.nsel[q] = K;
+    }
+    __syncthreads();
+}
+
+// Queries whose history fits in k keep every position (no scoring).
+__device__ void write_fallback(const K1Params &a, int q, int n) {
+    const int K = a.topk;
+    int32_t *out = a.idx + static_cast<int64_t>(q) * K;
+    for (int i = threadIdx.x; i < K; i += blockDim.x) out[i] = i < n ? i : -1;
+    if (threadIdx.x == 0 && a.nsel) a.nsel[q] = n;
+}
+
+// After all chunks of a group published: is this CTA the last one?
+__device__ bool arrive_group(const K1Params &a, K1Smem &sm, int g) {
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(&a.done[g], 1u);
+        sm.is_last = (prev == static_cast<uint32_t>(a.P - 1));
+    }
+    __syncthreads();
+    if (sm.is_last) __threadfence();
+    return sm.is_last != 0;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// K1: streaming indexer.  MODE_FUSED (scores stay on chip, TopK written) or
+// MODE_SCORES (scores written to HBM).
+// ---------------------------------------------------------------------------
+template <int MODE, int HP, int DI>
+__global__ void __launch_bounds__(kK1Threads, 1)
+    k1_indexer(const __grid_constant__ CUtensorMap kmap, const K1Params a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk);
+    uint8_t *stages = base + L.stages;
+    uint8_t *qtile = base + L.qtile;
+    uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
+    float *wts = reinterpret_cast<float *>(base + L.wts);
+    K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = blockIdx.x / a.P, c = blockIdx.x % a.P;
+    int q0, nqg;
+    group_queries(a, g, q0, nqg);
+    constexpr int kTileBytes = kTileRows * DI;
+    const int N = a.qg * HP;  // MMA N (columns per accumulator buffer)
+
+    // ---- set-up
+    if (tid == 0) {
+        sm.abort = 0;
+        sm.is_last = 0;
+        for (int s = 0; s < kK1Stages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 4);
+        }
+        fence_mbar_init();
+    }
+    if (tid < kMaxGroupQueries) sm.n_q[tid] = tid < nqg ? a.q_n[q0 + tid] : 0;
+    const int seq = nqg > 0 ? a.q_seq[q0] : 0;
+    // q^I tile (B operand, K-major, swizzled like the TMA tiles) and weights
+    for (int i = tid; i < N * (DI / 16); i += blockDim.x) {
+        const int r = i / (DI / 16), ch = i % (DI / 16);
+        const int qi = r / HP, j = r % HP;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (qi < nqg && j < a.h_idx)
+            v = *reinterpret_cast<const uint4 *>(a.q_idx + (static_cast<int64_t>(q0 + qi) * a.h_idx + j) * DI + ch * 16);
+        const int sw = (DI == 128) ? (ch ^ (r & 7)) : (ch ^ ((r >> 1) & 3));
+        *reinterpret_cast<uint4 *>(qtile + r * DI + sw * 16) = v;
+    }
+    for (int i = tid; i < N; i += blockDim.x) {
+        const int qi = i / HP, j = i % HP;
+        wts[i] = (qi < nqg && j < a.h_idx) ? bf16_bits_to_float(a.w[static_cast<int64_t>(q0 + qi) * a.h_idx + j]) : 0.f;
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, a.tmem_cols);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();  // q tile written by threads, read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    // a query group must read one sequence
+    if (tid < nqg && a.q_seq[q0 + tid] != seq) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+
+    // ---- span of positions this CTA covers
+    int nmax = 0, nscored = 0;
+    for (int i = 0; i < nqg; ++i) {
+        nmax = max(nmax, sm.n_q[i]);
+        if (MODE == kModeScores || sm.n_q[i] > a.topk) nscored = max(nscored, sm.n_q[i]);
+    }
+    const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
+    const int start = c * a.chunk;
+    const int end = min(start + a.chunk, span);
+    const int len = max(end - start, 0);
+    const int ntiles = (len + kTileRows - 1) / kTileRows;
+
+    if (MODE == kModeFused && c == 0)
+        for (int i = 0; i < nqg; ++i)
+            if (sm.n_q[i] <= a.topk) write_fallback(a, q0 + i, sm.n_q[i]);
+
+    // ---- streaming pipeline
+    if (ntiles > 0) {
+        if (warp == 0) {
+            if (lane == 0) {
+                const bool paged = a.page_table != nullptr;
+                const int64_t row0 = paged ? 0 : a.seq_row0[seq];
+                const int box = paged ? a.page_size : kTileRows;
+                for (int t = 0; t < ntiles && !sm.abort; ++t) {
+                    const int s = t % kK1Stages;
+                    const uint32_t ph = (t / kK1Stages) & 1;
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                        break;
+                    }
+                    const int p0 = start + t * kTileRows;
+                    uint32_t bytes = 0;
+                    for (int h = 0; h < kTileRows / box; ++h)
+                        if (p0 + h * box < nmax) bytes += box * DI;
+                    mbar_arrive_expect_tx(&sm.full[s], bytes);
+                    uint8_t *dst = stages + s * kTileBytes;
+                    for (int h = 0; h < kTileRows / box; ++h) {
+                        const int pp = p0 + h * box;
+                        if (pp >= nmax) break;
+                        int64_t row;
+                        if (paged)
+                            row = static_cast<int64_t>(a.page_table[static_cast<int64_t>(seq) * a.max_pages + pp / box]) * box;
+                        else
+                            row = row0 + pp;
+                        tma_load_2d(dst + h * box * DI, &kmap, &sm.full[s], 0, static_cast<int32_t>(row));
+                    }
+                }
+            }
+        } else if (warp == 1) {
+            if (lane == 0) {
+                const uint32_t idesc = make_idesc(0, 0, 0, 0, kTileRows, N);
+                constexpr uint32_t kSbo = 8 * DI;
+                constexpr uint32_t kLayout = (DI == 128) ? kSwizzle128B : kSwizzle64B;
+                const uint32_t qaddr = smem_u32(qtile);
+                for (int t = 0; t < ntiles && !sm.abort; ++t) {
+                    const int s = t % kK1Stages;
+                    const uint32_t ph = (t / kK1Stages) & 1;
+                    const int b = t & 1;
+                    const uint32_t aph = (t >> 1) & 1;
+                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1) || !mbar_wait(&sm.full[s], ph)) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t kaddr = smem_u32(stages + s * kTileBytes);
+#pragma unroll
+                    for (int kk = 0; kk < DI / 32; ++kk) {
+                        const uint64_t ad = make_sdesc(kaddr + kk * 32, 16, kSbo, kLayout);
+                        const uint64_t bd = make_sdesc(qaddr + kk * 32, 16, kSbo, kLayout);
+                        mma_f8_ss(tmem + b * N, ad, bd, idesc, kk > 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sm.empty[s]);
+                    tc_commit(&sm.acc_full[b]);
+                }
+            }
+        } else {
+            // epilogue: warps 2..5; TMEM lane quarter = warp % 4
+            const int quarter = warp & 3;
+            const int r = quarter * 32 + lane;
+            for (int t = 0; t < ntiles; ++t) {
+                const int b = t & 1;
+                const uint32_t aph = (t >> 1) & 1;
+                // every lane waits; the warp proceeds only if all saw the
+                // phase complete (tcgen05.ld below is warp-collective)
+                const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], aph) && !sm.abort);
+                if (!ok) {
+                    if (lane == 0) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                    }
+                    break;
+                }
+                tc_fence_after();
+                const int p = start + t * kTileRows + r;
+                float ks = 1.f;
+                if (a.k_scale && p < nmax) {
+                    int64_t row;
+                    if (a.page_table)
+                        row = static_cast<int64_t>(a.page_table[static_cast<int64_t>(seq) * a.max_pages + p / a.page_size]) * a.page_size + p % a.page_size;
+                    else
+                        row = a.seq_row0[seq] + p;
+                    ks = (row >= 0 && row < a.cache_rows) ? a.k_scale[row] : 0.f;
+                }
+                for (int qi = 0; qi < nqg; ++qi) {
+                    const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                           static_cast<uint32_t>(b * N + qi * HP);
+                    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+                    const float *wq = wts + qi * HP;
+#pragma unroll
+                    for (int c0 = 0; c0 < HP; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld16(taddr + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; j += 4) {
+                            acc0 = fmaf(wq[c0 + j + 0], fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
+                            acc1 = fmaf(wq[c0 + j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+                            acc2 = fmaf(wq[c0 + j + 2], fmaxf(__uint_as_float(v[j + 2]), 0.f), acc2);
+                            acc3 = fmaf(wq[c0 + j + 3], fmaxf(__uint_as_float(v[j + 3]), 0.f), acc3);
+                        }
+                    }
+                    const float score = ((acc0 + acc1) + (acc2 + acc3)) * ks;
+                    if (MODE == kModeScores) {
+                        if (p < end)
+                            a.scores[static_cast<int64_t>(q0 + qi) * a.ld + p] =
+                                p < sm.n_q[qi] ? score : -__int_as_float(0x7f800000);
+                    } else {
+                        if (p < end) keys[qi * a.chunk + (p - start)] = float_to_key(score);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    // ---- selection (fused mode)
+    if (MODE == kModeFused && !sm.abort) {
+        for (int qi = 0; qi < nqg; ++qi) {
+            const int n = sm.n_q[qi];
+            if (n <= a.topk) continue;
+            const int qlen = max(min(end, n) - start, 0);
+            chunk_select(a, sm, q0 + qi, qi, keys + qi * a.chunk, start, qlen, hist);
+            __syncthreads();
+        }
+        if (a.P > 1) {
+            bool any = false;
+            for (int qi = 0; qi < nqg; ++qi) any |= sm.n_q[qi] > a.topk;
+            if (any && arrive_group(a, sm, g)) {
+                // candidate list of the threshold bin lives in the (now free)
+                // streaming area: stages + q tile + keys
+                uint64_t *list = reinterpret_cast<uint64_t *>(base);
+                const int list_cap = static_cast<int>(L.hist / sizeof(uint64_t));
+                for (int qi = 0; qi < nqg; ++qi)
+                    if (sm.n_q[qi] > a.topk) group_merge(a, sm, q0 + qi, hist, list, list_cap);
+            }
+        }
+    }
+
+    // ---- teardown
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, a.tmem_cols);
+}
+
+// ---------------------------------------------------------------------------
+// K2: TopK of scores already in HBM (same chunking and merge as K1).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk);
+    uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
+    K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
+    const int q = blockIdx.x / a.P, c = blockIdx.x % a.P;
+    if (threadIdx.x == 0) {
+        sm.abort = 0;
+        sm.is_last = 0;
+        sm.n_q[0] = a.q_n[q];
+    }
+    __syncthreads();
+    const int n = sm.n_q[0];
+    if (n <= a.topk) {
+        if (c == 0) write_fallback(a, q, n);
+        return;
+    }
+    const int start = c * a.chunk;
+    const int end = min(start + a.chunk, n);
+    const int len = max(end - start, 0);
+    const float *src = a.scores + static_cast<int64_t>(q) * a.ld;
+    for (int i = threadIdx.x; i < len; i += blockDim.x) keys[i] = float_to_key(__ldg(&src[start + i]));
+    __syncthreads();
+    chunk_select(a, sm, q, 0, keys, start, len, hist);
+    __syncthreads();
+    if (a.P > 1 && arrive_group(a, sm, q)) {
+        uint64_t *list = reinterpret_cast<uint64_t *>(base);
+        const int list_cap = static_cast<int>(L.hist / sizeof(uint64_t));
+        group_merge(a, sm, q, hist, list, list_cap);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host-side launchers
+// ---------------------------------------------------------------------------
+template <int MODE, int HP, int DI>
+static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaStream_t st) {
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk);
+    const size_t smem = smem_for_tmem(L.total, a.tmem_cols);
+    auto kern = k1_indexer<MODE, HP, DI>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = a.n_groups * a.P;
+    if (grid == 0) return cudaSuccess;
+    kern<<<grid, kK1Threads, smem, st>>>(kmap, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, const K1Params &a,
+                           cudaStream_t st) {
+#define DSA_K1_CASE(M, H, D) \
+    if (mode == M && hp == H && di == D) return launch_k1_t<M, H, D>(kmap, a, st);
+    DSA_K1_CASE(kModeFused, 64, 128)
+    DSA_K1_CASE(kModeFused, 16, 128)
+    DSA_K1_CASE(kModeFused, 64, 64)
+    DSA_K1_CASE(kModeFused, 16, 64)
+    DSA_K1_CASE(kModeScores, 64, 128)
+    DSA_K1_CASE(kModeScores, 16, 128)
+    DSA_K1_CASE(kModeScores, 64, 64)
+    DSA_K1_CASE(kModeScores, 16, 64)
+#undef DSA_K1_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_topk(const K1Params &a, cudaStream_t st) {
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk);
+    cudaError_t e = cudaFuncSetAttribute(k2_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
+    if (e != cudaSuccess) return e;
+    const int grid = a.nq * a.P;
+    if (grid == 0) return cudaSuccess;
+    k2_topk<<<grid, kK2Threads, L.total, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

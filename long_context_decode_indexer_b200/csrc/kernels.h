@@ -1,0 +1,161 @@
+// kernels.h -- launch parameters and shared-memory layouts of the kernels,
+// shared by the host-side API (dsa_api.cu) and the device code.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace dsa {
+
+// ---------------------------------------------------------------- indexer
+constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
+constexpr int kModeScores = 1;  // scores written to HBM
+constexpr int kModeTopk = 2;    // TopK of scores read from HBM
+
+constexpr int kK1Stages = 5;         // TMA ring depth (128-row k^I tiles)
+constexpr int kK1Threads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kK2Threads = 256;
+constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
+constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
+constexpr int kSelBinsHost = 2048;
+
+struct K1Params {
+    // inputs
+    const uint8_t *q_idx;   // [nq, h_idx, d_idx] e4m3
+    const uint16_t *w;      // [nq, h_idx] bf16
+    const float *k_scale;   // [cache_rows] or null
+    const int32_t *q_seq;
+    const int32_t *q_n;
+    const int64_t *seq_row0;
+    const int32_t *page_table;
+    int32_t max_pages;
+    int32_t page_size;
+    int64_t cache_rows;
+    int32_t nq, h_idx, d_idx, topk;
+    // work split
+    int32_t q_per_seq, qg, groups_per_block, n_groups;
+    int32_t P;      // chunks per group
+    int32_t chunk;  // positions per chunk (multiple of 128)
+    uint32_t tmem_cols;
+    // outputs
+    float *scores;  // kModeScores output / kModeTopk input
+    int64_t ld;
+    int32_t *idx;
+    int32_t *nsel;
+    // workspace
+    uint32_t *ghist;      // [nq, 2048] global top-digit histograms
+    uint64_t *cand;       // [nq, P, topk] candidate composites
+    int32_t *cand_cnt;    // [nq, P]
+    uint32_t *done;       // [n_groups] chunks finished
+    int *status;
+};
+
+struct K1Layout {
+    uint32_t stages, qtile, keys, hist, wts, misc, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// Offsets from a 1024-byte aligned base; `total` includes the alignment slack.
+__host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, int chunk, int P,
+                                              int topk) {
+    K1Layout L;
+    uint32_t off = 0;
+    L.stages = off;
+    if (mode != kModeTopk) off += kK1Stages * 128u * static_cast<uint32_t>(di);
+    L.qtile = off;
+    if (mode != kModeTopk) off += align_up(static_cast<uint32_t>(qg * hp * di), 1024);
+    L.keys = off;
+    if (mode != kModeScores) off += static_cast<uint32_t>(qg) * static_cast<uint32_t>(chunk) * 4u;
+    // the last CTA of a group stages the threshold-bin candidates in the
+    // area below the histogram
+    if (mode != kModeScores && P > 1) {
+        const uint32_t need = static_cast<uint32_t>(P) * static_cast<uint32_t>(topk) * 8u;
+        if (off < need) off = need;
+    }
+    off = align_up(off, 128);
+    L.hist = off;
+    off += (mode != kModeScores) ? kSelBinsHost * 4u : 0u;
+    L.wts = off;
+    off += align_up(static_cast<uint32_t>(qg * hp * 4), 16);
+    off = align_up(off, 128);
+    L.misc = off;
+    off += 1024;
+    L.total = off + 1024;
+    return L;
+}
+
+// Dynamic shared memory to request so that no SM can host more CTAs than
+// its 512 TMEM columns serve at `tmem_cols` each (tcgen05.alloc then never
+// has to wait for another CTA to free columns).
+inline size_t smem_for_tmem(size_t want, uint32_t tmem_cols) {
+    const size_t kSmemPerSm = 233472, kReserved = 1024;
+    const size_t max_ctas = tmem_cols ? 512 / tmem_cols : 32;
+    const size_t floor_bytes = kSmemPerSm / (max_ctas + 1) - kReserved + 1;
+    return want > floor_bytes ? want : floor_bytes;
+}
+
+cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, const K1Params &a,
+                           cudaStream_t st);
+cudaError_t launch_topk(const K1Params &a, cudaStream_t st);
+
+// ------------------------------------------------------ sparse MLA attention
+constexpr int kDqk = 576;           // key width (512 latent + 64 rope)
+constexpr int kDv = 512;            // value width
+constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
+constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
+constexpr int kMlaStages = 3;       // pass-1 ring depth (Q chunk + K chunk)
+constexpr int kMlaVRows = 64;       // rows per pass-2 V tile
+constexpr int kMlaThreads = 192;    // warps 0-3 softmax/epilogue, warp 4 TMA, warp 5 MMA
+
+struct MlaParams {
+    const int32_t *q_seq;
+    const int32_t *q_n;
+    const int64_t *seq_row0;
+    const int32_t *page_table;
+    int32_t max_pages, page_size;
+    int64_t cache_rows;
+    const int32_t *idx;  // [nq, topk]
+    const uint16_t *kv;  // latent cache (bf16 bits)
+    int64_t kv_row_stride;  // elements between cache rows
+    int32_t nq, h, topk;
+    int32_t splits;      // CTAs per query along the index list
+    int32_t rows_per_split;
+    int32_t q0;          // first query of this launch (wave)
+    float scale_log2;    // scale * log2(e)
+    float scale;
+    // outputs
+    uint16_t *out;       // [nq, h, d_v] bf16
+    float *lse;          // [nq, h]
+    float *part_o;       // [wave_q, splits, 128, d_v] normalised partial outputs
+    float *part_lse;     // [wave_q, splits, 128]
+    int *status;
+};
+
+struct MlaLayout {
+    uint32_t ring, p_tile, v_ring, misc, total;
+};
+
+__host__ __device__ inline MlaLayout mla_layout() {
+    MlaLayout L;
+    // pass 1: kMlaStages x (Q chunk 128x64 bf16 = 16 KB + K chunk 256x64 bf16 = 32 KB)
+    const uint32_t stage = 128u * 128u + kMlaMaxRows * 128u;
+    const uint32_t pass1 = kMlaStages * stage;
+    // pass 2: P (128 x 256 bf16 = 64 KB) + 2 V tiles (64 rows x 512 bf16 = 64 KB each)
+    const uint32_t ptile = 128u * kMlaMaxRows * 2u;
+    const uint32_t vtile = kMlaVRows * kDv * 2u;
+    L.ring = 0;
+    L.p_tile = 0;
+    L.v_ring = ptile;
+    uint32_t end = pass1 > ptile + 2 * vtile ? pass1 : ptile + 2 * vtile;
+    L.misc = align_up(end, 128);
+    L.total = L.misc + 4096 + 1024;
+    return L;
+}
+
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap, const MlaParams &a,
+                              int nq_wave, cudaStream_t st);
+cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st);
+
+}  // namespace dsa

@@ -1,0 +1,448 @@
+// sparse_mla.cu -- sparse MQA-mode MLA attention on sm_100a.
+//
+// u_t = Attn(h_t, {c_s : s in I_t}) (DSA blog by marsggbo, section 3) in the
+// MQA form of weight-absorbed MLA: every head attends to the same latent row,
+// softmax(q . [c_kv; k_pe]^T) . c_kv ("DeepSeekV3.2之DSA" by yuyanqi,
+// section 5.1).  Key = the whole 576-wide row, value = its first 512 columns.
+//
+// One CTA owns one query and a slice of at most 256 of its selected rows
+// ("split"); all 128 heads form the MMA's M dimension.
+//   pass 1  S[128 x R] = Q . K^T over 9 chunks of 64 key columns.  Each ring
+//           stage holds a Q chunk (TMA tile, 16 KB) and the R rows' matching
+//           128-byte pieces (TMA gather4, four rows per instruction); the
+//           rows were first prefetched whole into L2.  S accumulates in TMEM.
+//   softmax one thread per head reads its S row from TMEM, takes the exact
+//           max over the split, writes P = exp(S - max) as bf16 into shared
+//           memory (the A operand of pass 2) and keeps the row sum.
+//   pass 2  O[128 x 512] = P . V, V re-gathered (64-row tiles, L2 hits) into
+//           an MN-major swizzled layout; O takes all 512 TMEM columns, which
+//           is why S and O are not live at the same time.
+// A split writes O / l and its log-sum-exp; the combine kernel merges splits
+// by their log-sum-exp.  With one split the CTA writes the final output.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kQChunkBytes = 128 * 128;             // 128 heads x 64 bf16
+constexpr int kStageBytes = kQChunkBytes + kMlaMaxRows * 128;
+constexpr int kNumKChunks = kDqk / 64;              // 9
+constexpr int kVTileBytes = kMlaVRows * kDv * 2;    // 64 KB
+constexpr int kPBlockBytes = 128 * 128;             // 128 heads x 64 rows bf16
+
+struct MlaSmem {
+    uint64_t full[kMlaStages];
+    uint64_t empty[kMlaStages];
+    uint64_t s_full;
+    uint64_t p_full;
+    uint64_t v_full[2];
+    uint64_t v_empty[2];
+    uint64_t o_full;
+    uint32_t tmem_base;
+    volatile int32_t abort;
+    int32_t nvalid;
+    int32_t rows[kMlaMaxRows];
+    uint8_t valid[kMlaMaxRows];
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
+    return a | (b << 16);
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kMlaThreads, 1)
+    k3_sparse_mla(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
+                  const MlaParams a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    const MlaLayout L = mla_layout();
+    MlaSmem &sm = *reinterpret_cast<MlaSmem *>(base + L.misc);
+    uint8_t *ring = base + L.ring;
+    uint8_t *ptile = base + L.p_tile;
+    uint8_t *vring = base + L.v_ring;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int wq = blockIdx.x / a.splits;  // query within this wave
+    const int sp = blockIdx.x % a.splits;
+    const int q = a.q0 + wq;
+    const int e0 = sp * a.rows_per_split;
+    const int R = max(min(a.rows_per_split, a.topk - e0), 0);
+    const int Rp = (R + 15) & ~15;  // MMA N (multiple of 16)
+    const int hbox = a.h < 128 ? a.h : 128;
+
+    if (tid == 0) {
+        sm.abort = 0;
+        sm.nvalid = 0;
+        for (int s = 0; s < kMlaStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.p_full, 4);
+        for (int v = 0; v < 2; ++v) {
+            mbar_init(&sm.v_full[v], 1);
+            mbar_init(&sm.v_empty[v], 1);
+        }
+        mbar_init(&sm.o_full, 1);
+        fence_mbar_init();
+    }
+    // cache rows of this split's entries (invalid entries read row 0 and are
+    // masked; P = 0 there)
+    const int n = a.q_n[q];
+    const int seq = a.q_seq[q];
+    __syncthreads();
+    for (int i = tid; i < kMlaMaxRows; i += blockDim.x) {
+        int32_t row = 0;
+        uint8_t ok = 0;
+        if (i < R) {
+            const int s = a.idx[static_cast<int64_t>(q) * a.topk + e0 + i];
+            if (s >= n) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+            if (s >= 0 && s < n) {
+                int64_t r;
+                if (a.page_table)
+                    r = static_cast<int64_t>(a.page_table[static_cast<int64_t>(seq) * a.max_pages + s / a.page_size]) * a.page_size + s % a.page_size;
+                else
+                    r = a.seq_row0[seq] + s;
+                if (r >= 0 && r < a.cache_rows) {
+                    row = static_cast<int32_t>(r);
+                    ok = 1;
+                } else {
+                    record_status(a.status, DSA_ERR_DEVICE_CHECK);
+                }
+            }
+        }
+        sm.rows[i] = row;
+        sm.valid[i] = ok;
+    }
+    // rows h..127 of every Q chunk are never written by TMA: zero them once
+    if (hbox < 128) {
+        for (int s = 0; s < kMlaStages; ++s)
+            for (int i = tid; i < (128 - hbox) * 8; i += blockDim.x)
+                *reinterpret_cast<uint4 *>(ring + s * kStageBytes + hbox * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+    }
+    if (warp == 5) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (Rp > 0) {
+        if (warp == 4) {
+            // ------------------------------------------------ TMA producer
+            const uint16_t *kvbase = a.kv;
+            for (int i = lane; i < R; i += 32)
+                if (sm.valid[i])
+                    prefetch_l2_bulk(kvbase + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
+            const uint32_t qbytes = static_cast<uint32_t>(hbox) * 128u;
+            const uint32_t kbytes = static_cast<uint32_t>(Rp) * 128u;
+            for (int c = 0; c < kNumKChunks; ++c) {
+                const int s = c % kMlaStages;
+                const uint32_t ph = (c / kMlaStages) & 1;
+                bool ok = true;
+                if (lane == 0) {
+                    ok = !sm.abort && mbar_wait(&sm.empty[s], ph ^ 1);
+                    if (ok) mbar_arrive_expect_tx(&sm.full[s], qbytes + kbytes);
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) {
+                    if (lane == 0) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                    }
+                    break;
+                }
+                uint8_t *st = ring + s * kStageBytes;
+                if (lane == 0) tma_load_2d(st, &qmap, &sm.full[s], c * 64, q * a.h);
+                for (int g = lane; g < Rp / 4; g += 32)
+                    tma_gather4(st + kQChunkBytes + g * 512, &kvmap, &sm.full[s], c * 64,
+                                sm.rows[4 * g], sm.rows[4 * g + 1], sm.rows[4 * g + 2], sm.rows[4 * g + 3]);
+            }
+            // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is done
+            bool ok = true;
+            if (lane == 0) ok = mbar_wait(&sm.s_full, 0) && !sm.abort;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
+            for (int vt = 0; ok && vt < nvt; ++vt) {
+                const int v = vt & 1;
+                const uint32_t ph = (vt >> 1) & 1;
+                bool ok2 = true;
+                if (lane == 0) {
+                    ok2 = !sm.abort && mbar_wait(&sm.v_empty[v], ph ^ 1);
+                    if (ok2) mbar_arrive_expect_tx(&sm.v_full[v], kVTileBytes);
+                }
+                ok2 = __shfl_sync(0xffffffffu, ok2, 0);
+                if (!ok2) {
+                    if (lane == 0) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                    }
+                    break;
+                }
+                uint8_t *vt_base = vring + v * kVTileBytes;
+                // 8 column blocks x 16 groups of 4 rows
+                for (int t = lane; t < 8 * 16; t += 32) {
+                    const int blk = t >> 4, g = t & 15;
+                    const int r0 = vt * kMlaVRows + 4 * g;
+                    int32_t rr[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) rr[u] = (r0 + u < R) ? sm.rows[r0 + u] : 0;
+                    tma_gather4(vt_base + blk * (kMlaVRows * 128) + g * 512, &kvmap, &sm.v_full[v],
+                                blk * 64, rr[0], rr[1], rr[2], rr[3]);
+                }
+            }
+        } else if (warp == 5) {
+            // ------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                bool ok = true;
+                const uint32_t idesc1 = make_idesc(1, 1, 0, 0, 128, static_cast<uint32_t>(Rp));
+                for (int c = 0; c < kNumKChunks; ++c) {
+                    const int s = c % kMlaStages;
+                    const uint32_t ph = (c / kMlaStages) & 1;
+                    if (sm.abort || !mbar_wait(&sm.full[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t qa = smem_u32(ring + s * kStageBytes);
+                    const uint32_t ka = qa + kQChunkBytes;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t ad = make_sdesc(qa + kk * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t bd = make_sdesc(ka + kk * 32, 16, 1024, kSwizzle128B);
+                        mma_bf16_ss(tmem, ad, bd, idesc1, (c > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(&sm.empty[s]);
+                }
+                tc_commit(&sm.s_full);
+                if (ok && mbar_wait(&sm.p_full, 0) && !sm.abort) {
+                    tc_fence_after();
+                    // B = V tile, MN-major: LBO = 8 KB between 64-column blocks,
+                    // SBO = 1 KB between 8-row groups
+                    const uint32_t idesc2 = make_idesc(1, 1, 0, 1, 128, 256);
+                    const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
+                    for (int vt = 0; vt < nvt; ++vt) {
+                        const int v = vt & 1;
+                        const uint32_t ph = (vt >> 1) & 1;
+                        if (sm.abort || !mbar_wait(&sm.v_full[v], ph)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint32_t pa = smem_u32(ptile + vt * kPBlockBytes);
+                        const uint32_t va = smem_u32(vring + v * kVTileBytes);
+                        const int ksteps = min(4, (Rp - vt * kMlaVRows) / 16);
+                        for (int ks = 0; ks < ksteps; ++ks) {
+                            const uint64_t ad = make_sdesc(pa + ks * 32, 16, 1024, kSwizzle128B);
+#pragma unroll
+                            for (int nh = 0; nh < 2; ++nh) {
+                                const uint64_t bd = make_sdesc(va + nh * 4 * (kMlaVRows * 128) + ks * 2048,
+                                                               kMlaVRows * 128, 1024, kSwizzle128B);
+                                mma_bf16_ss(tmem + nh * 256, ad, bd, idesc2, (vt > 0 || ks > 0) ? 1u : 0u);
+                            }
+                        }
+                        tc_commit(&sm.v_empty[v]);
+                    }
+                }
+                tc_commit(&sm.o_full);
+                if (!ok) {
+                    record_status(a.status, DSA_ERR_TIMEOUT);
+                    sm.abort = 1;
+                }
+            }
+        } else if (warp < 4) {
+            // ------------------------------------- softmax, then epilogue
+            const int hrow = warp * 32 + lane;  // head = TMEM lane
+            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+            bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
+            float m = -INFINITY, l = 0.f;
+            if (ok) {
+                tc_fence_after();
+                for (int c0 = 0; c0 < Rp; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        if (c0 + j < R && sm.valid[c0 + j]) m = fmaxf(m, __uint_as_float(v[j]));
+                }
+                const float mlog = (m == -INFINITY) ? 0.f : m * a.scale_log2;
+                for (int c0 = 0; c0 < Rp; c0 += 32) {
+                    uint32_t v[32];
+                    tmem_ld32(lane_addr + c0, v);
+                    tmem_wait_ld();
+                    float p[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const bool vj = (c0 + j < R) && sm.valid[c0 + j];
+                        p[j] = vj ? exp2f(__uint_as_float(v[j]) * a.scale_log2 - mlog) : 0.f;
+                        l += p[j];
+                    }
+                    // P row `hrow`, columns c0..c0+31: K-major 128B-swizzled blocks of 64
+                    uint8_t *blk = ptile + (c0 >> 6) * kPBlockBytes + hrow * 128;
+#pragma unroll
+                    for (int g8 = 0; g8 < 4; ++g8) {
+                        const int ch = ((c0 & 63) >> 3) + g8;  // 16-byte chunk within the 128B row
+                        uint4 u;
+                        u.x = pack_bf16x2(p[g8 * 8 + 0], p[g8 * 8 + 1]);
+                        u.y = pack_bf16x2(p[g8 * 8 + 2], p[g8 * 8 + 3]);
+                        u.z = pack_bf16x2(p[g8 * 8 + 4], p[g8 * 8 + 5]);
+                        u.w = pack_bf16x2(p[g8 * 8 + 6], p[g8 * 8 + 7]);
+                        *reinterpret_cast<uint4 *>(blk + ((ch ^ (hrow & 7)) << 4)) = u;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.p_full);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0) && !sm.abort);
+            if (ok) {
+                tc_fence_after();
+                const bool has = l > 0.f;
+                const float inv_l = has ? 1.f / l : 0.f;
+                const float lse_v = has ? (m * a.scale + logf(l)) : -INFINITY;
+                const bool head_ok = hrow < a.h;
+                if (a.splits == 1) {
+                    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv;
+                    for (int c0 = 0; c0 < kDv; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + c0, v);
+                        tmem_wait_ld();
+                        if (head_ok) {
+#pragma unroll
+                            for (int g8 = 0; g8 < 4; ++g8) {
+                                uint4 u;
+                                u.x = pack_bf16x2(__uint_as_float(v[g8 * 8 + 0]) * inv_l, __uint_as_float(v[g8 * 8 + 1]) * inv_l);
+                                u.y = pack_bf16x2(__uint_as_float(v[g8 * 8 + 2]) * inv_l, __uint_as_float(v[g8 * 8 + 3]) * inv_l);
+                                u.z = pack_bf16x2(__uint_as_float(v[g8 * 8 + 4]) * inv_l, __uint_as_float(v[g8 * 8 + 5]) * inv_l);
+                                u.w = pack_bf16x2(__uint_as_float(v[g8 * 8 + 6]) * inv_l, __uint_as_float(v[g8 * 8 + 7]) * inv_l);
+                                *reinterpret_cast<uint4 *>(o + c0 + g8 * 8) = u;
+                            }
+                        }
+                    }
+                    if (head_ok) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
+                } else {
+                    float *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+                    for (int c0 = 0; c0 < kDv; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(lane_addr + c0, v);
+                        tmem_wait_ld();
+                        if (head_ok) {
+#pragma unroll
+                            for (int g4 = 0; g4 < 8; ++g4) {
+                                float4 f;
+                                f.x = __uint_as_float(v[g4 * 4 + 0]) * inv_l;
+                                f.y = __uint_as_float(v[g4 * 4 + 1]) * inv_l;
+                                f.z = __uint_as_float(v[g4 * 4 + 2]) * inv_l;
+                                f.w = __uint_as_float(v[g4 * 4 + 3]) * inv_l;
+                                *reinterpret_cast<float4 *>(o + c0 + g4 * 4) = f;
+                            }
+                        }
+                    }
+                    if (head_ok) a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
+                }
+            } else if (lane == 0) {
+                record_status(a.status, DSA_ERR_TIMEOUT);
+            }
+        }
+    } else if (warp < 4) {
+        // empty split: no rows at all
+        const int hrow = warp * 32 + lane;
+        if (hrow < a.h) {
+            if (a.splits == 1) {
+                uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv;
+                for (int c0 = 0; c0 < kDv; c0 += 8) *reinterpret_cast<uint4 *>(o + c0) = make_uint4(0, 0, 0, 0);
+                a.lse[static_cast<int64_t>(q) * a.h + hrow] = -INFINITY;
+            } else {
+                float *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+                for (int c0 = 0; c0 < kDv; c0 += 4) *reinterpret_cast<float4 *>(o + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = -INFINITY;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 5) tmem_dealloc(tmem, 512);
+}
+
+// Merge the splits of one (query, head): out = sum_s w_s o_s / sum_s w_s with
+// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.
+__global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a) {
+    const int wq = blockIdx.x / a.h, hh = blockIdx.x % a.h;
+    const int q = a.q0 + wq;
+    float mx = -INFINITY;
+    for (int s = 0; s < a.splits; ++s)
+        mx = fmaxf(mx, a.part_lse[(static_cast<int64_t>(wq) * a.splits + s) * 128 + hh]);
+    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv;
+    if (mx == -INFINITY) {
+        for (int d = threadIdx.x * 4; d < kDv; d += blockDim.x * 4) {
+            *reinterpret_cast<uint2 *>(o + d) = make_uint2(0, 0);
+        }
+        if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
+        return;
+    }
+    float tot = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int d = threadIdx.x * 4;
+    for (int s = 0; s < a.splits; ++s) {
+        const int64_t row = (static_cast<int64_t>(wq) * a.splits + s) * 128 + hh;
+        const float ls = a.part_lse[row];
+        if (ls == -INFINITY) continue;
+        const float wgt = __expf(ls - mx);
+        tot += wgt;
+        const float4 v = *reinterpret_cast<const float4 *>(a.part_o + row * kDv + d);
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    const float inv = 1.f / tot;
+    uint2 u;
+    u.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    u.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(o + d) = u;
+    if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
+}
+
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap, const MlaParams &a,
+                              int nq_wave, cudaStream_t st) {
+    const MlaLayout L = mla_layout();
+    const size_t smem = smem_for_tmem(L.total, 512);
+    cudaError_t e = cudaFuncSetAttribute(k3_sparse_mla, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int grid = nq_wave * a.splits;
+    if (grid == 0) return cudaSuccess;
+    k3_sparse_mla<<<grid, kMlaThreads, smem, st>>>(qmap, kvmap, a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st) {
+    const int grid = nq_wave * a.h;
+    if (grid == 0 || a.splits <= 1) return cudaSuccess;
+    k4_mla_combine<<<grid, 128, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

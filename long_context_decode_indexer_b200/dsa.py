@@ -1,0 +1,182 @@
+"""Python binding of the C ABI in include/dsa.h (argument marshalling only).
+
+Every function here forwards to the same-named entry point of
+``libdsa_b200.so``; tensors are passed as raw device pointers.  Nothing is
+computed in Python and there is no fallback: if the library is missing or a
+call fails, a ``DsaError`` is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa_b200.so")
+
+DSA_OK = 0
+DSA_ERR_INVALID_ARG = -1
+DSA_ERR_UNSUPPORTED = -2
+DSA_ERR_CUDA = -3
+DSA_ERR_WORKSPACE = -4
+DSA_ERR_TIMEOUT = -5
+DSA_ERR_DEVICE_CHECK = -6
+
+OP_INDEXER_SCORES = 0
+OP_TOPK = 1
+OP_INDEXER_TOPK = 2
+OP_SPARSE_MLA_DECODE = 3
+OP_SPARSE_MLA_PREFILL = 4
+OP_FORWARD = 5
+
+# Entry points declared in include/dsa.h.
+ENTRY_POINTS = (
+    "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk",
+    "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill", "dsa_forward", "dsa_forward_paged",
+    "dsa_check_status", "dsa_last_error",
+)
+
+
+class DsaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__("%s (status %d)" % (msg, code))
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    _fields_ = [("nq", ctypes.c_int32), ("h_idx", ctypes.c_int32), ("d_idx", ctypes.c_int32),
+                ("h", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("max_n", ctypes.c_int32),
+                ("q_per_seq", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class KV(ctypes.Structure):
+    _fields_ = [("q_seq", ctypes.c_void_p), ("q_n", ctypes.c_void_p),
+                ("seq_row0", ctypes.c_void_p), ("page_table", ctypes.c_void_p),
+                ("max_pages", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("cache_rows", ctypes.c_int64)]
+
+
+_lock = threading.Lock()
+_lib: Optional[ctypes.CDLL] = None
+_P = ctypes.c_void_p
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa_b200.so (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise DsaError(DSA_ERR_CUDA, "libdsa_b200.so not built (run "
+                               "python -m long_context_decode_indexer_b200.build)")
+            L = ctypes.CDLL(LIB_PATH)
+            pp, kp = ctypes.POINTER(Params), ctypes.POINTER(KV)
+            L.dsa_workspace_size.argtypes = [pp, kp, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]
+            L.dsa_indexer_scores.argtypes = [pp, kp, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
+                                             ctypes.c_size_t, _P]
+            L.dsa_topk.argtypes = [pp, _P, ctypes.c_int64, _P, _P, _P, _P, ctypes.c_size_t, _P]
+            L.dsa_indexer_topk.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+            for name in ("dsa_sparse_mla_decode", "dsa_sparse_mla_prefill"):
+                getattr(L, name).argtypes = [pp, kp, _P, _P, ctypes.c_int64, _P, _P, _P, _P,
+                                             ctypes.c_size_t, _P]
+            for name in ("dsa_forward", "dsa_forward_paged"):
+                getattr(L, name).argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
+                                             _P, _P, _P, ctypes.c_size_t, _P]
+            L.dsa_check_status.argtypes = [_P, _P]
+            L.dsa_last_error.restype = ctypes.c_char_p
+            for name in ENTRY_POINTS[:-1]:
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def last_error() -> str:
+    return lib().dsa_last_error().decode()
+
+
+def _check(rc: int, what: str):
+    if rc != DSA_OK:
+        raise DsaError(rc, "%s: %s" % (what, last_error()))
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def make_params(*, nq, h_idx, d_idx, h, topk, max_n, q_per_seq=1, scale, d_qk=576, d_v=512) -> Params:
+    return Params(int(nq), int(h_idx), int(d_idx), int(h), int(d_qk), int(d_v), int(topk),
+                  int(max_n), int(q_per_seq), float(scale))
+
+
+def make_kv(*, q_seq, q_n, seq_row0=None, page_table=None, page_size=0, cache_rows) -> KV:
+    max_pages = int(page_table.shape[1]) if page_table is not None else 0
+    return KV(_ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+              int(page_size) if page_table is not None else 0, int(cache_rows))
+
+
+def workspace_size(p: Params, kv: Optional[KV], op: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().dsa_workspace_size(ctypes.byref(p), ctypes.byref(kv) if kv is not None else None,
+                                    int(op), ctypes.byref(out)), "dsa_workspace_size")
+    return int(out.value)
+
+
+def indexer_scores(p, kv, q_idx, w, kidx_cache, k_scale, scores, ld_scores, ws, stream=None):
+    _check(lib().dsa_indexer_scores(ctypes.byref(p), ctypes.byref(kv), _ptr(q_idx), _ptr(w),
+                                    _ptr(kidx_cache), _ptr(k_scale), _ptr(scores), int(ld_scores),
+                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_indexer_scores")
+
+
+def topk(p, scores, ld_scores, q_n, idx, nsel, ws, stream=None):
+    _check(lib().dsa_topk(ctypes.byref(p), _ptr(scores), int(ld_scores), _ptr(q_n), _ptr(idx),
+                          _ptr(nsel), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_topk")
+
+
+def indexer_topk(p, kv, q_idx, w, kidx_cache, k_scale, idx, nsel, ws, stream=None):
+    _check(lib().dsa_indexer_topk(ctypes.byref(p), ctypes.byref(kv), _ptr(q_idx), _ptr(w),
+                                  _ptr(kidx_cache), _ptr(k_scale), _ptr(idx), _ptr(nsel), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_indexer_topk")
+
+
+def sparse_mla_decode(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, stream=None):
+    _check(lib().dsa_sparse_mla_decode(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(kv_cache),
+                                       int(kv_row_stride), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_sparse_mla_decode")
+
+
+def sparse_mla_prefill(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, stream=None):
+    _check(lib().dsa_sparse_mla_prefill(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(kv_cache),
+                                        int(kv_row_stride), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_sparse_mla_prefill")
+
+
+def forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, out, lse, idx_out,
+            ws, stream=None, paged=False):
+    fn = lib().dsa_forward_paged if paged else lib().dsa_forward
+    _check(fn(ctypes.byref(p), ctypes.byref(kv), _ptr(q_idx), _ptr(w), _ptr(kidx_cache),
+              _ptr(k_scale), _ptr(q), _ptr(kv_cache), int(kv_row_stride), _ptr(out), _ptr(lse),
+              _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_forward_paged" if paged else "dsa_forward")
+
+
+def check_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (then clear) the device status word."""
+    return int(lib().dsa_check_status(_ptr(ws), _stream(stream)))
