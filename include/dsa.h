@@ -11,7 +11,9 @@
  * Conventions shared by every call
  *   - Pointers.  Every tensor argument is a DEVICE pointer owned by the caller.
  *     The library allocates no device memory; scratch comes from the caller's
- *     `ws` buffer of at least dsa_workspace_size() bytes, 256-byte aligned.
+ *     `ws` buffer of at least dsa_workspace_size() bytes, 256-byte aligned and
+ *     zero-filled before its first use (its first word is the status word;
+ *     every call leaves the rest of ws ready for the next call).
  *     `dsa_params` and `dsa_kv` themselves are host structs (their pointer
  *     members are device pointers).
  *   - Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy
@@ -147,7 +149,7 @@ int dsa_indexer_scores(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  *   scores  [nq, ld_scores] fp32 (entries s >= q_n[i] are not read)
  *   q_n     [nq] int32 device
  *   idx     [nq, topk] int32 output: the min(topk, n) selected positions in
- *           unspecified order, then -1
+ *           ascending order, then -1 (the same output every run)
  *   nsel    [nq] int32 output min(topk, n), or NULL
  * The result is exact: identical scores give identical sets. */
 int dsa_topk(const dsa_params *p, const float *scores, int64_t ld_scores,

@@ -69,9 +69,10 @@ def upload(inp: Inputs, device="cuda") -> DeviceBatch:
 
 
 def workspace(nbytes: int, device="cuda") -> torch.Tensor:
-    """A 256-byte aligned device buffer of at least nbytes (torch's caching
+    """A zero-filled, 256-byte aligned device buffer of at least nbytes (the
+    C ABI wants the workspace zeroed before its first use; torch's caching
     allocator returns 512-byte aligned blocks)."""
-    t = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+    t = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
     assert t.data_ptr() % 256 == 0
     return t
 

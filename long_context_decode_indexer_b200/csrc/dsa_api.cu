@@ -115,7 +115,7 @@ int check_kv(const dsa_params *p, const dsa_kv *kv) {
 
 // ----------------------------------------------------------------- planning
 struct IndexerPlan {
-    int hp, qg, gpb, n_groups, P, chunk;
+    int hp, qg, gpb, n_groups, P, chunk, stages;
     uint32_t tmem_cols;
     size_t smem;
 };
@@ -163,7 +163,18 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(2 * pl.qg * pl.hp)) cols <<= 1;
     pl.tmem_cols = cols;
-    const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk);
+    // TMA ring: as many 128-row tiles as the shared memory left by the keys holds
+    // (the merge area reuses the ring once streaming is over)
+    pl.stages = 0;
+    if (mode != dsa::kModeTopk) {
+        int st = dsa::kK1MaxStages;
+        while (st >= 2 &&
+               dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st).total > 232448)
+            --st;
+        if (st < 2) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
+        pl.stages = st;
+    }
+    const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, pl.stages);
     pl.smem = L.total;
     if (pl.smem > 232448) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
     return DSA_OK;
@@ -311,6 +322,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.n_groups = pl.n_groups;
     a.P = pl.P;
     a.chunk = pl.chunk;
+    a.stages = pl.stages;
     a.tmem_cols = pl.tmem_cols;
     a.scores = scores;
     a.ld = ld;

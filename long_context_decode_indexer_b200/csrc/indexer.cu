@@ -42,8 +42,8 @@ namespace {
 constexpr int kTileRows = 128;
 
 struct K1Smem {
-    uint64_t full[kK1Stages];
-    uint64_t empty[kK1Stages];
+    uint64_t full[kK1MaxStages];
+    uint64_t empty[kK1MaxStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
@@ -101,64 +101,65 @@ __device__ void local_top_hist(const uint32_t *keys, int len, uint32_t *hist) {
 
 // Everything one query of a chunk does after its keys are in shared memory:
 // direct selection (one chunk), or publishing candidates (several chunks).
-// `keys` holds the chunk's keys for positions [start, start + len).
-__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, const uint32_t *keys,
-                             int start, int len, uint32_t *hist) {
+// `keys` holds the chunk's keys for positions [start, start + len).  Every
+// emission is an ordered compaction, so results come out in ascending
+// position order and are identical from run to run.
+__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, const uint32_t *keys, int start,
+                             int len, uint32_t *hist) {
     const int K = a.topk;
-    const int n = sm.n_q[qi];
     LocalSrc src{keys, start};
     if (a.P == 1) {
-        // the whole history is here: n == len > K
+        // the whole history is here: len == n > K
         local_top_hist(keys, len, hist);
         find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
         const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
         __syncthreads();
         const uint32_t need = static_cast<uint32_t>(K) - above;
-        uint64_t thr = (static_cast<uint64_t>(d) << 53);
+        uint64_t thr = static_cast<uint64_t>(d) << 53;
         if (bucket != need) thr = radix_refine(src, len, d, 1, need, hist, sm.sel);
-        if (threadIdx.x == 0) sm.sel.counter[0] = 0;
-        __syncthreads();
         int32_t *out = a.idx + static_cast<int64_t>(q) * K;
-        emit_selected(src, len, [thr](uint64_t v) { return v >= thr; },
-                      [out, K](uint32_t slot, uint64_t v) {
-                          if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
-                      },
-                      sm.sel, 0);
-        __syncthreads();
+        const uint32_t cnt = emit_ordered(
+            src, len, [thr](uint64_t v) { return v >= thr; },
+            [out, K](uint32_t slot, uint64_t v) {
+                if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
+            },
+            0u, sm.sel.wsum);
         if (threadIdx.x == 0) {
-            if (sm.sel.counter[0] != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+            if (cnt != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
             if (a.nsel) a.nsel[q] = K;
         }
-        (void)n;
+        __syncthreads();
         return;
     }
 
     // ---- several chunks: publish this chunk's candidates
     uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
-    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + blockIdx.x % a.P) * K;
+    const int c = blockIdx.x % a.P;
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * K;
     local_top_hist(keys, len, hist);
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
         if (hist[b]) atomicAdd(&G[b], hist[b]);
     __threadfence();
     __syncthreads();
-    // snapshot of G (a lower bound of the final histogram, bin by bin)
+    // a snapshot of G is a bin-wise lower bound of the final histogram
     uint32_t *snap = hist;
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) snap[b] = __ldcg(&G[b]);
     __syncthreads();
     find_digit(snap, kSelBins, static_cast<uint32_t>(K), sm.sel);
     const uint32_t dlow = sm.sel.res[0];
     __syncthreads();
-    // how many local keys sit at or above dlow
+    // local keys at or above dlow
     if (threadIdx.x == 0) sm.sel.counter[1] = 0;
     __syncthreads();
     {
-        uint32_t c = 0;
-        for (int i = threadIdx.x; i < len; i += blockDim.x) c += (top_digit(keys[i]) >= dlow);
-        c = warp_sum(c);
-        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], c);
+        uint32_t n_at = 0;
+        for (int i = threadIdx.x; i < len; i += blockDim.x) n_at += (top_digit(keys[i]) >= dlow);
+        n_at = warp_sum(n_at);
+        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], n_at);
     }
     __syncthreads();
     const uint32_t at_or_above = sm.sel.counter[1];
+    __syncthreads();
     uint64_t thr = static_cast<uint64_t>(dlow) << 53;
     if (at_or_above > static_cast<uint32_t>(K)) {
         // cap at the exact local TopK: a key beaten by k keys of its own
@@ -172,26 +173,26 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, const
         if (bucket != need) lthr = radix_refine(src, len, d, 1, need, hist, sm.sel);
         thr = lthr > thr ? lthr : thr;
     }
-    if (threadIdx.x == 0) sm.sel.counter[0] = 0;
-    __syncthreads();
-    emit_selected(src, len, [thr](uint64_t v) { return v >= thr; },
-                  [cand, K](uint32_t slot, uint64_t v) {
-                      if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
-                  },
-                  sm.sel, 0);
-    __syncthreads();
+    uint32_t m = emit_ordered(
+        src, len, [thr](uint64_t v) { return v >= thr; },
+        [cand, K](uint32_t slot, uint64_t v) {
+            if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
+        },
+        0u, sm.sel.wsum);
     if (threadIdx.x == 0) {
-        uint32_t m = sm.sel.counter[0];
         if (m > static_cast<uint32_t>(K)) {
             record_status(a.status, DSA_ERR_DEVICE_CHECK);
             m = K;
         }
-        a.cand_cnt[static_cast<int64_t>(q) * a.P + blockIdx.x % a.P] = static_cast<int32_t>(m);
+        a.cand_cnt[static_cast<int64_t>(q) * a.P + c] = static_cast<int32_t>(m);
     }
-    (void)n;
+    __syncthreads();
 }
 
 // The last CTA of a group: final selection of query q from all candidates.
+// Chunks publish their candidates in ascending position order and chunk c
+// covers positions below chunk c + 1, so staging the lists chunk by chunk
+// keeps the whole candidate list in ascending position order.
 __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, uint32_t *hist, uint64_t *list,
                             int list_cap) {
     const int K = a.topk;
@@ -201,66 +202,65 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, uint32_t *hist
     find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
     const uint32_t dstar = sm.sel.res[0], above = sm.sel.res[1];
     __syncthreads();
-    int32_t *out = a.idx + static_cast<int64_t>(q) * K;
-    if (threadIdx.x == 0) {
-        sm.sel.counter[0] = 0;  // slots in out
-        sm.sel.counter[1] = 0;  // bucket list length
-    }
-    __syncthreads();
-    // pass over all candidates: digit > d* -> selected; digit == d* -> list
+    // stage all candidates (ordered) in shared memory
     const uint64_t *cand = a.cand + static_cast<int64_t>(q) * a.P * K;
     const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * a.P;
-    const int lane = threadIdx.x & 31;
+    int total = 0;
     for (int c = 0; c < a.P; ++c) {
-        const int m = __ldcg(&cnt[c]);
-        for (int i0 = 0; i0 < m; i0 += blockDim.x) {
-            const int i = i0 + threadIdx.x;
-            uint64_t v = 0;
-            if (i < m) v = __ldcg(&cand[static_cast<int64_t>(c) * K + i]);
-            const uint32_t dg = static_cast<uint32_t>(v >> 53);
-            const bool take = (i < m) && dg > dstar;
-            const bool keep = (i < m) && dg == dstar;
-            unsigned mt = __ballot_sync(0xffffffffu, take);
-            unsigned mk = __ballot_sync(0xffffffffu, keep);
-            uint32_t bt = 0, bk = 0;
-            if (lane == 0) {
-                if (mt) bt = atomicAdd(&sm.sel.counter[0], static_cast<uint32_t>(__popc(mt)));
-                if (mk) bk = atomicAdd(&sm.sel.counter[1], static_cast<uint32_t>(__popc(mk)));
+        const int m = min(__ldcg(&cnt[c]), K);
+        const uint64_t *src = cand + static_cast<int64_t>(c) * K;
+        if (total + m > list_cap) {
+            if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+            __syncthreads();
+            return;
+        }
+        for (int j0 = 0; j0 < m; j0 += 4 * blockDim.x) {
+            uint64_t v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * blockDim.x + threadIdx.x;
+                v[u] = j < m ? __ldcg(&src[j]) : 0ull;
             }
-            bt = __shfl_sync(0xffffffffu, bt, 0);
-            bk = __shfl_sync(0xffffffffu, bk, 0);
-            const unsigned lt = (1u << lane) - 1u;
-            if (take) {
-                const uint32_t s = bt + __popc(mt & lt);
-                if (s < static_cast<uint32_t>(K)) out[s] = static_cast<int32_t>(composite_pos(v));
-            }
-            if (keep) {
-                const uint32_t s = bk + __popc(mk & lt);
-                if (s < static_cast<uint32_t>(list_cap)) list[s] = v;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * blockDim.x + threadIdx.x;
+                if (j < m) list[total + j] = v[u];
             }
         }
+        total += m;
     }
     __syncthreads();
-    const uint32_t taken = sm.sel.counter[0];
-    const uint32_t nlist = sm.sel.counter[1];
+    // bucket d* count among the candidates must cover what is needed
+    if (threadIdx.x == 0) sm.sel.counter[1] = 0;
     __syncthreads();
-    if (taken != above || nlist > static_cast<uint32_t>(list_cap) ||
-        nlist < static_cast<uint32_t>(K) - above) {
+    {
+        uint32_t n_b = 0;
+        for (int i = threadIdx.x; i < total; i += blockDim.x)
+            n_b += static_cast<uint32_t>(list[i] >> 53) == dstar;
+        n_b = warp_sum(n_b);
+        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], n_b);
+    }
+    __syncthreads();
+    const uint32_t nbucket = sm.sel.counter[1];
+    __syncthreads();
+    const uint32_t need = static_cast<uint32_t>(K) - above;
+    int32_t *out = a.idx + static_cast<int64_t>(q) * K;
+    if (nbucket < need) {
         if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        __syncthreads();
         return;
     }
-    const uint32_t need = static_cast<uint32_t>(K) - above;
     ListSrc src{list};
     uint64_t thr = static_cast<uint64_t>(dstar) << 53;
-    if (nlist != need) thr = radix_refine(src, static_cast<int>(nlist), dstar, 1, need, hist, sm.sel);
-    emit_selected(src, static_cast<int>(nlist), [thr](uint64_t v) { return v >= thr; },
-                  [out, K](uint32_t slot, uint64_t v) {
-                      if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
-                  },
-                  sm.sel, 0);
-    __syncthreads();
+    if (nbucket != need) thr = radix_refine(src, total, dstar, 1, need, hist, sm.sel);
+    const uint32_t got = emit_ordered(
+        src, total, [thr](uint64_t v) { return v >= thr; },
+        [out, K](uint32_t slot, uint64_t v) {
+            if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
+        },
+        0u, sm.sel.wsum);
     if (threadIdx.x == 0) {
-        if (sm.sel.counter[0] != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        if (got != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
         if (a.nsel) a.nsel[q] = K;
     }
     __syncthreads();
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     k1_indexer(const __grid_constant__ CUtensorMap kmap, const K1Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk);
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages);
     uint8_t *stages = base + L.stages;
     uint8_t *qtile = base + L.qtile;
     uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (tid == 0) {
         sm.abort = 0;
         sm.is_last = 0;
-        for (int s = 0; s < kK1Stages; ++s) {
+        for (int s = 0; s < a.stages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -380,8 +380,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 const int64_t row0 = paged ? 0 : a.seq_row0[seq];
                 const int box = paged ? a.page_size : kTileRows;
                 for (int t = 0; t < ntiles && !sm.abort; ++t) {
-                    const int s = t % kK1Stages;
-                    const uint32_t ph = (t / kK1Stages) & 1;
+                    const int s = t % a.stages;
+                    const uint32_t ph = (t / a.stages) & 1;
                     if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
@@ -412,8 +412,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 constexpr uint32_t kLayout = (DI == 128) ? kSwizzle128B : kSwizzle64B;
                 const uint32_t qaddr = smem_u32(qtile);
                 for (int t = 0; t < ntiles && !sm.abort; ++t) {
-                    const int s = t % kK1Stages;
-                    const uint32_t ph = (t / kK1Stages) & 1;
+                    const int s = t % a.stages;
+                    const uint32_t ph = (t / a.stages) & 1;
                     const int b = t & 1;
                     const uint32_t aph = (t >> 1) & 1;
                     if (!mbar_wait(&sm.acc_empty[b], aph ^ 1) || !mbar_wait(&sm.full[s], ph)) {
@@ -466,18 +466,18 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                                            static_cast<uint32_t>(b * N + qi * HP);
                     float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
                     const float *wq = wts + qi * HP;
+                    uint32_t v[HP];
+                    // issue every load of the row, then wait once
 #pragma unroll
-                    for (int c0 = 0; c0 < HP; c0 += 16) {
-                        uint32_t v[16];
-                        tmem_ld16(taddr + c0, v);
-                        tmem_wait_ld();
+                    for (int c0 = 0; c0 < HP; c0 += 16)
+                        tmem_ld16(taddr + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[c0]));
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int j = 0; j < 16; j += 4) {
-                            acc0 = fmaf(wq[c0 + j + 0], fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
-                            acc1 = fmaf(wq[c0 + j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
-                            acc2 = fmaf(wq[c0 + j + 2], fmaxf(__uint_as_float(v[j + 2]), 0.f), acc2);
-                            acc3 = fmaf(wq[c0 + j + 3], fmaxf(__uint_as_float(v[j + 3]), 0.f), acc3);
-                        }
+                    for (int j = 0; j < HP; j += 4) {
+                        acc0 = fmaf(wq[j + 0], fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
+                        acc1 = fmaf(wq[j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
+                        acc2 = fmaf(wq[j + 2], fmaxf(__uint_as_float(v[j + 2]), 0.f), acc2);
+                        acc3 = fmaf(wq[j + 3], fmaxf(__uint_as_float(v[j + 3]), 0.f), acc3);
                     }
                     const float score = ((acc0 + acc1) + (acc2 + acc3)) * ks;
                     if (MODE == kModeScores) {
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             const int n = sm.n_q[qi];
             if (n <= a.topk) continue;
             const int qlen = max(min(end, n) - start, 0);
-            chunk_select(a, sm, q0 + qi, qi, keys + qi * a.chunk, start, qlen, hist);
+            chunk_select(a, sm, q0 + qi, keys + qi * a.chunk, start, qlen, hist);
             __syncthreads();
         }
         if (a.P > 1) {
@@ -534,7 +534,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk);
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0);
     uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
     uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
     K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
@@ -556,7 +556,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     const float *src = a.scores + static_cast<int64_t>(q) * a.ld;
     for (int i = threadIdx.x; i < len; i += blockDim.x) keys[i] = float_to_key(__ldg(&src[start + i]));
     __syncthreads();
-    chunk_select(a, sm, q, 0, keys, start, len, hist);
+    chunk_select(a, sm, q, keys, start, len, hist);
     __syncthreads();
     if (a.P > 1 && arrive_group(a, sm, q)) {
         uint64_t *list = reinterpret_cast<uint64_t *>(base);
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
 // ---------------------------------------------------------------------------
 template <int MODE, int HP, int DI>
 static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaStream_t st) {
-    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk);
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages);
     const size_t smem = smem_for_tmem(L.total, a.tmem_cols);
     auto kern = k1_indexer<MODE, HP, DI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -598,7 +598,7 @@ cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, co
 }
 
 cudaError_t launch_topk(const K1Params &a, cudaStream_t st) {
-    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk);
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0);
     cudaError_t e = cudaFuncSetAttribute(k2_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
     if (e != cudaSuccess) return e;
     const int grid = a.nq * a.P;

@@ -13,7 +13,7 @@ constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
 constexpr int kModeScores = 1;  // scores written to HBM
 constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 
-constexpr int kK1Stages = 5;         // TMA ring depth (128-row k^I tiles)
+constexpr int kK1MaxStages = 12;     // TMA ring depth limit (128-row k^I tiles)
 constexpr int kK1Threads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr int kK2Threads = 256;
 constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
@@ -37,6 +37,7 @@ struct K1Params {
     int32_t q_per_seq, qg, groups_per_block, n_groups;
     int32_t P;      // chunks per group
     int32_t chunk;  // positions per chunk (multiple of 128)
+    int32_t stages; // TMA ring depth
     uint32_t tmem_cols;
     // outputs
     float *scores;  // kModeScores output / kModeTopk input
@@ -59,11 +60,11 @@ __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x
 
 // Offsets from a 1024-byte aligned base; `total` includes the alignment slack.
 __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, int chunk, int P,
-                                              int topk) {
+                                              int topk, int stages) {
     K1Layout L;
     uint32_t off = 0;
     L.stages = off;
-    if (mode != kModeTopk) off += kK1Stages * 128u * static_cast<uint32_t>(di);
+    if (mode != kModeTopk) off += static_cast<uint32_t>(stages) * 128u * static_cast<uint32_t>(di);
     L.qtile = off;
     if (mode != kModeTopk) off += align_up(static_cast<uint32_t>(qg * hp * di), 1024);
     L.keys = off;
@@ -106,7 +107,7 @@ constexpr int kDv = 512;            // value width
 constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
 constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
 constexpr int kMlaStages = 3;       // pass-1 ring depth (Q chunk + K chunk)
-constexpr int kMlaVRows = 64;       // rows per pass-2 V tile
+constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
 constexpr int kMlaThreads = 192;    // warps 0-3 softmax/epilogue, warp 4 TMA, warp 5 MMA
 
 struct MlaParams {
@@ -134,7 +135,7 @@ struct MlaParams {
 };
 
 struct MlaLayout {
-    uint32_t ring, p_tile, v_ring, misc, total;
+    uint32_t ring, p_tile, p_lo, v_ring, misc, total;
 };
 
 __host__ __device__ inline MlaLayout mla_layout() {
@@ -142,13 +143,15 @@ __host__ __device__ inline MlaLayout mla_layout() {
     // pass 1: kMlaStages x (Q chunk 128x64 bf16 = 16 KB + K chunk 256x64 bf16 = 32 KB)
     const uint32_t stage = 128u * 128u + kMlaMaxRows * 128u;
     const uint32_t pass1 = kMlaStages * stage;
-    // pass 2: P (128 x 256 bf16 = 64 KB) + 2 V tiles (64 rows x 512 bf16 = 64 KB each)
+    // pass 2: P as a hi + lo pair of bf16 tiles (128 x 256 each, 64 KB each)
+    // + 2 V tiles (32 rows x 512 bf16 = 32 KB each)
     const uint32_t ptile = 128u * kMlaMaxRows * 2u;
     const uint32_t vtile = kMlaVRows * kDv * 2u;
     L.ring = 0;
     L.p_tile = 0;
-    L.v_ring = ptile;
-    uint32_t end = pass1 > ptile + 2 * vtile ? pass1 : ptile + 2 * vtile;
+    L.p_lo = ptile;
+    L.v_ring = 2 * ptile;
+    uint32_t end = pass1 > 2 * ptile + 2 * vtile ? pass1 : 2 * ptile + 2 * vtile;
     L.misc = align_up(end, 128);
     L.total = L.misc + 4096 + 1024;
     return L;

@@ -25,6 +25,7 @@ struct SelectScratch {
     uint32_t csum[64];     // per-32-bin chunk sums
     uint32_t res[4];       // digit, count above the digit's bucket, bucket size
     uint32_t counter[4];   // emission slots
+    uint32_t wsum[32];     // per-warp counts of an ordered compaction
 };
 
 __device__ __forceinline__ uint64_t make_composite(uint32_t key, uint32_t pos) {
@@ -149,6 +150,47 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
         if (bucket == need) return prefix << shift;
     }
     return prefix;
+}
+
+// Ordered block-wide compaction: the elements i in [0, n) with pred(v) true
+// are handed to out(slot, v) with consecutive slots base, base + 1, ... in
+// increasing i.  Each thread owns 8 consecutive elements per round; a block
+// scan of the per-thread counts gives every thread its first slot.  Returns
+// the next free slot.  `wsum` is shared scratch of 32 words.
+template <class Src, class Pred, class Out>
+__device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
+                                 uint32_t base, uint32_t *wsum) {
+    constexpr int kPer = 8;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    const int round = blockDim.x * kPer;
+    for (int r0 = 0; r0 < n; r0 += round) {
+        uint64_t vals[kPer];
+        uint32_t mask = 0;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int i = r0 + tid * kPer + e;
+            uint64_t v = 0;
+            if (i < n && src(i, v) && pred(v)) mask |= 1u << e;
+            vals[e] = v;
+        }
+        const uint32_t cnt = static_cast<uint32_t>(__popc(mask));
+        const uint32_t incl = warp_incl_scan(cnt);
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        uint32_t before = 0, total = 0;
+        for (int w = 0; w < nw; ++w) {
+            const uint32_t c = wsum[w];
+            before += (w < warp) ? c : 0u;
+            total += c;
+        }
+        uint32_t slot = base + before + incl - cnt;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e)
+            if ((mask >> e) & 1u) out(slot++, vals[e]);
+        base += total;
+        __syncthreads();
+    }
+    return base;
 }
 
 // Block-wide compaction: every element with pred(i, v) true is handed to

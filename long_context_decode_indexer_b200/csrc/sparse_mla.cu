@@ -12,11 +12,14 @@
 //           128-byte pieces (TMA gather4, four rows per instruction); the
 //           rows were first prefetched whole into L2.  S accumulates in TMEM.
 //   softmax one thread per head reads its S row from TMEM, takes the exact
-//           max over the split, writes P = exp(S - max) as bf16 into shared
-//           memory (the A operand of pass 2) and keeps the row sum.
-//   pass 2  O[128 x 512] = P . V, V re-gathered (64-row tiles, L2 hits) into
-//           an MN-major swizzled layout; O takes all 512 TMEM columns, which
-//           is why S and O are not live at the same time.
+//           max over the split, writes P = exp(S - max) into shared memory
+//           as a pair of bf16 tiles P_hi = bf16(P), P_lo = bf16(P - P_hi)
+//           (the A operands of pass 2) and keeps the row sum.  A single bf16
+//           P would add ~1e-3 relative error on top of the ~1.7e-3 that the
+//           bf16 output itself carries; the pair makes P exact to ~2^-16.
+//   pass 2  O[128 x 512] = P_hi . V + P_lo . V, V re-gathered (32-row tiles,
+//           L2 hits) into an MN-major swizzled layout; O takes all 512 TMEM
+//           columns, which is why S and O are not live at the same time.
 // A split writes O / l and its log-sum-exp; the combine kernel merges splits
 // by their log-sum-exp.  With one split the CTA writes the final output.
 #include <cuda.h>
@@ -35,7 +38,8 @@ namespace {
 constexpr int kQChunkBytes = 128 * 128;             // 128 heads x 64 bf16
 constexpr int kStageBytes = kQChunkBytes + kMlaMaxRows * 128;
 constexpr int kNumKChunks = kDqk / 64;              // 9
-constexpr int kVTileBytes = kMlaVRows * kDv * 2;    // 64 KB
+constexpr int kVTileBytes = kMlaVRows * kDv * 2;    // 32 KB
+constexpr int kVBlockBytes = kMlaVRows * 128;       // one 64-column block of a V tile
 constexpr int kPBlockBytes = 128 * 128;             // 128 heads x 64 rows bf16
 
 struct MlaSmem {
@@ -74,6 +78,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     MlaSmem &sm = *reinterpret_cast<MlaSmem *>(base + L.misc);
     uint8_t *ring = base + L.ring;
     uint8_t *ptile = base + L.p_tile;
+    uint8_t *plo = base + L.p_lo;
     uint8_t *vring = base + L.v_ring;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -198,14 +203,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     break;
                 }
                 uint8_t *vt_base = vring + v * kVTileBytes;
-                // 8 column blocks x 16 groups of 4 rows
-                for (int t = lane; t < 8 * 16; t += 32) {
-                    const int blk = t >> 4, g = t & 15;
+                // 8 column blocks x (kMlaVRows / 4) groups of 4 rows
+                constexpr int kGroups = kMlaVRows / 4;
+                for (int t = lane; t < 8 * kGroups; t += 32) {
+                    const int blk = t / kGroups, g = t % kGroups;
                     const int r0 = vt * kMlaVRows + 4 * g;
                     int32_t rr[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) rr[u] = (r0 + u < R) ? sm.rows[r0 + u] : 0;
-                    tma_gather4(vt_base + blk * (kMlaVRows * 128) + g * 512, &kvmap, &sm.v_full[v],
+                    tma_gather4(vt_base + blk * kVBlockBytes + g * 512, &kvmap, &sm.v_full[v],
                                 blk * 64, rr[0], rr[1], rr[2], rr[3]);
                 }
             }
@@ -235,8 +241,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 tc_commit(&sm.s_full);
                 if (ok && mbar_wait(&sm.p_full, 0) && !sm.abort) {
                     tc_fence_after();
-                    // B = V tile, MN-major: LBO = 8 KB between 64-column blocks,
-                    // SBO = 1 KB between 8-row groups
+                    // B = V tile, MN-major: LBO = distance between 64-column
+                    // blocks, SBO = 1 KB between 8-row groups.  A = P_hi, P_lo:
+                    // K-major, 64-row blocks of 16 KB, 16-row k-steps 32 B apart.
                     const uint32_t idesc2 = make_idesc(1, 1, 0, 1, 128, 256);
                     const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
                     for (int vt = 0; vt < nvt; ++vt) {
@@ -247,16 +254,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                             break;
                         }
                         tc_fence_after();
-                        const uint32_t pa = smem_u32(ptile + vt * kPBlockBytes);
+                        const int row0 = vt * kMlaVRows;
+                        const uint32_t poff = (row0 >> 6) * kPBlockBytes + ((row0 & 63) >> 4) * 32;
+                        const uint32_t pa_hi = smem_u32(ptile) + poff;
+                        const uint32_t pa_lo = smem_u32(plo) + poff;
                         const uint32_t va = smem_u32(vring + v * kVTileBytes);
-                        const int ksteps = min(4, (Rp - vt * kMlaVRows) / 16);
+                        const int ksteps = min(kMlaVRows / 16, (Rp - row0) / 16);
                         for (int ks = 0; ks < ksteps; ++ks) {
-                            const uint64_t ad = make_sdesc(pa + ks * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t ad_hi = make_sdesc(pa_hi + ks * 32, 16, 1024, kSwizzle128B);
+                            const uint64_t ad_lo = make_sdesc(pa_lo + ks * 32, 16, 1024, kSwizzle128B);
 #pragma unroll
                             for (int nh = 0; nh < 2; ++nh) {
-                                const uint64_t bd = make_sdesc(va + nh * 4 * (kMlaVRows * 128) + ks * 2048,
-                                                               kMlaVRows * 128, 1024, kSwizzle128B);
-                                mma_bf16_ss(tmem + nh * 256, ad, bd, idesc2, (vt > 0 || ks > 0) ? 1u : 0u);
+                                const uint64_t bd = make_sdesc(va + nh * 4 * kVBlockBytes + ks * 2048,
+                                                               kVBlockBytes, 1024, kSwizzle128B);
+                                mma_bf16_ss(tmem + nh * 256, ad_hi, bd, idesc2, (vt > 0 || ks > 0) ? 1u : 0u);
+                                mma_bf16_ss(tmem + nh * 256, ad_lo, bd, idesc2, 1u);
                             }
                         }
                         tc_commit(&sm.v_empty[v]);
@@ -297,16 +309,22 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                         l += p[j];
                     }
                     // P row `hrow`, columns c0..c0+31: K-major 128B-swizzled blocks of 64
-                    uint8_t *blk = ptile + (c0 >> 6) * kPBlockBytes + hrow * 128;
+                    const uint32_t rowoff = (c0 >> 6) * kPBlockBytes + hrow * 128;
 #pragma unroll
                     for (int g8 = 0; g8 < 4; ++g8) {
                         const int ch = ((c0 & 63) >> 3) + g8;  // 16-byte chunk within the 128B row
-                        uint4 u;
-                        u.x = pack_bf16x2(p[g8 * 8 + 0], p[g8 * 8 + 1]);
-                        u.y = pack_bf16x2(p[g8 * 8 + 2], p[g8 * 8 + 3]);
-                        u.z = pack_bf16x2(p[g8 * 8 + 4], p[g8 * 8 + 5]);
-                        u.w = pack_bf16x2(p[g8 * 8 + 6], p[g8 * 8 + 7]);
-                        *reinterpret_cast<uint4 *>(blk + ((ch ^ (hrow & 7)) << 4)) = u;
+                        uint32_t hi[4], lo[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a0 = p[g8 * 8 + 2 * e], a1 = p[g8 * 8 + 2 * e + 1];
+                            const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
+                            hi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+                            lo[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+                        }
+                        const uint32_t off = rowoff + ((ch ^ (hrow & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(ptile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        *reinterpret_cast<uint4 *>(plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     }
                 }
             }

@@ -113,6 +113,7 @@ def check_scores(gpu: np.ndarray, ref: np.ndarray, absref: np.ndarray, q_n: np.n
 
 def check_index_set_exact(gpu_idx: np.ndarray, ref_idx: np.ndarray, n: int, k: int):
     m = min(n, k)
+    assert np.all(np.diff(gpu_idx[:m]) > 0), "selected positions are not in ascending order"
     g = np.sort(gpu_idx[:m])
     r = np.sort(ref_idx[:m])
     assert np.all(gpu_idx[m:] == -1), "padding is not -1"
@@ -128,6 +129,7 @@ def check_recall(gpu_idx: np.ndarray, ref_scores: np.ndarray, q_n: np.ndarray, k
         m = min(n, k)
         gi = gpu_idx[qi, :m]
         assert np.all(gi >= 0) and np.all(gi < n), "query %d: index out of range" % qi
+        assert np.all(np.diff(gi) > 0), "query %d: positions not in ascending order" % qi
         assert len(np.unique(gi)) == m, "query %d: duplicate indices" % qi
         assert np.all(gpu_idx[qi, m:] == -1), "query %d: padding is not -1" % qi
         ref_idx, _ = oracle.topk(ref_scores[qi, :n], k)
