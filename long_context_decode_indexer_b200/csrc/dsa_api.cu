@@ -213,7 +213,7 @@ MlaPlan plan_mla(const dsa_params *p) {
 
 // -------------------------------------------------------------- workspace
 struct WsLayout {
-    size_t status, ghist, cand, cand_cnt, done, idx, part_o, part_lse, total;
+    size_t status, ghist, gtot, cand, cand_cnt, done, idx, part_o, part_lse, total;
     size_t zero_begin, zero_end;  // cleared at the start of every call
 };
 
@@ -223,6 +223,8 @@ size_t indexer_ws(const dsa_params *p, const IndexerPlan &pl, int mode, size_t o
     w.zero_begin = off;
     w.ghist = off;
     off = up(off + static_cast<size_t>(p->nq) * 2048 * 4, 256);
+    w.gtot = off;
+    off = up(off + static_cast<size_t>(p->nq) * 4, 256);
     w.done = off;
     off = up(off + static_cast<size_t>(pl.n_groups) * 4, 256);
     w.zero_end = off;
@@ -331,7 +333,10 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.status = at<int>(ws, wl.status);
     if (mode != dsa::kModeScores && pl.P > 1) {
         a.ghist = at<uint32_t>(ws, wl.ghist);
+        a.gtot = at<uint32_t>(ws, wl.gtot);
         a.done = at<uint32_t>(ws, wl.done);
+        // every CTA of the launch is resident at once (one CTA per SM)
+        a.wait_hist = (static_cast<int64_t>(pl.n_groups) * pl.P <= num_sms()) ? 1 : 0;
         a.cand = at<uint64_t>(ws, wl.cand);
         a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
         cudaError_t e = cudaMemsetAsync(static_cast<uint8_t *>(ws) + wl.zero_begin, 0,

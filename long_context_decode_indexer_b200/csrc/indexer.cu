@@ -10,9 +10,10 @@
 // sequence; a group's history [0, span) is cut into P chunks, one CTA each.
 // A CTA streams its chunk of the FP8 index-K cache through a TMA ring, and
 // the tensor cores compute D[128 positions x qg*hp heads] = K_tile . Q^T
-// (tcgen05 kind::f8f6f4, M = 128, N = qg*hp, K = d_I) into TMEM.  Four
-// epilogue warps read D back (one TMEM lane = one position per thread) and
-// apply ReLU, * w, the head sum and * k_s.
+// (tcgen05 kind::f8f6f4, M = 128, N = qg*hp, K = d_I) into a double-buffered
+// TMEM accumulator.  Two groups of four epilogue warps, one per accumulator
+// buffer (even and odd tiles), read D back (one TMEM lane = one position per
+// thread) and apply ReLU, * w, the head sum and * k_s.
 //
 // Fused mode keeps the chunk's scores in shared memory as order-preserving
 // keys.  Exact selection across chunks without a grid barrier:
@@ -77,6 +78,15 @@ struct LocalSrc {
         v = make_composite(keys[i], static_cast<uint32_t>(base + i));
         return true;
     }
+    // eight consecutive elements from i0 (a multiple of 8; the buffer is
+    // padded to a multiple of 128 entries)
+    __device__ void get8(int i0, uint64_t (&v)[8]) const {
+        const uint4 a = *reinterpret_cast<const uint4 *>(keys + i0);
+        const uint4 b = *reinterpret_cast<const uint4 *>(keys + i0 + 4);
+        const uint32_t k[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = make_composite(k[e], static_cast<uint32_t>(base + i0 + e));
+    }
 };
 // Candidates staged in shared memory (already composites).
 struct ListSrc {
@@ -85,38 +95,48 @@ struct ListSrc {
         v = list[i];
         return true;
     }
+    __device__ void get8(int i0, uint64_t (&v)[8]) const {
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(list + i0 + e);
+            v[e] = (static_cast<uint64_t>(u.y) << 32) | u.x;
+            v[e + 1] = (static_cast<uint64_t>(u.w) << 32) | u.z;
+        }
+    }
 };
 
-// Local histogram of the top digit of every key of this chunk.
-__device__ void local_top_hist(const uint32_t *keys, int len, uint32_t *hist) {
-    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = 0;
+// Sum of hist[b] for b >= lo (block-wide; every thread gets the result).
+__device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScratch &sc) {
+    if (threadIdx.x == 0) sc.counter[2] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < len; i0 += blockDim.x) {
-        const int i = i0 + threadIdx.x;
-        const bool act = i < len;
-        hist_add(hist, act, act ? top_digit(keys[i]) : 0u);
-    }
+    uint32_t c = 0;
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) c += (static_cast<uint32_t>(b) >= lo) ? hist[b] : 0u;
+    c = warp_sum(c);
+    if ((threadIdx.x & 31) == 0) atomicAdd(&sc.counter[2], c);
     __syncthreads();
+    const uint32_t r = sc.counter[2];
+    __syncthreads();
+    return r;
 }
 
 // Everything one query of a chunk does after its keys are in shared memory:
 // direct selection (one chunk), or publishing candidates (several chunks).
-// `keys` holds the chunk's keys for positions [start, start + len).  Every
-// emission is an ordered compaction, so results come out in ascending
-// position order and are identical from run to run.
-__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, const uint32_t *keys, int start,
-                             int len, uint32_t *hist) {
+// `keys` holds the chunk's keys for positions [start, start + len) and
+// `lhist` the histogram of their top digits.  Every emission is an ordered
+// compaction, so results come out in ascending position order and are the
+// same from run to run.
+__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int n, const uint32_t *keys,
+                             int start, int len, const uint32_t *lhist, uint32_t *scratch) {
     const int K = a.topk;
     LocalSrc src{keys, start};
     if (a.P == 1) {
         // the whole history is here: len == n > K
-        local_top_hist(keys, len, hist);
-        find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+        find_digit(lhist, kSelBins, static_cast<uint32_t>(K), sm.sel);
         const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
         __syncthreads();
         const uint32_t need = static_cast<uint32_t>(K) - above;
         uint64_t thr = static_cast<uint64_t>(d) << 53;
-        if (bucket != need) thr = radix_refine(src, len, d, 1, need, hist, sm.sel);
+        if (bucket != need) thr = radix_refine(src, len, d, 1, need, scratch, sm.sel);
         int32_t *out = a.idx + static_cast<int64_t>(q) * K;
         const uint32_t cnt = emit_ordered(
             src, len, [thr](uint64_t v) { return v >= thr; },
@@ -132,45 +152,45 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, const uint32_
         return;
     }
 
-    // ---- several chunks: publish this chunk's candidates
+    // ---- several chunks: publish this chunk's histogram, then its candidates
     uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
     const int c = blockIdx.x % a.P;
     uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * K;
-    local_top_hist(keys, len, hist);
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
-        if (hist[b]) atomicAdd(&G[b], hist[b]);
+        if (lhist[b]) atomicAdd(&G[b], lhist[b]);
     __threadfence();
     __syncthreads();
-    // a snapshot of G is a bin-wise lower bound of the final histogram
-    uint32_t *snap = hist;
-    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) snap[b] = __ldcg(&G[b]);
-    __syncthreads();
-    find_digit(snap, kSelBins, static_cast<uint32_t>(K), sm.sel);
-    const uint32_t dlow = sm.sel.res[0];
-    __syncthreads();
-    // local keys at or above dlow
-    if (threadIdx.x == 0) sm.sel.counter[1] = 0;
-    __syncthreads();
-    {
-        uint32_t n_at = 0;
-        for (int i = threadIdx.x; i < len; i += blockDim.x) n_at += (top_digit(keys[i]) >= dlow);
-        n_at = warp_sum(n_at);
-        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], n_at);
+    if (threadIdx.x == 0) {
+        atomicAdd(&a.gtot[q], static_cast<uint32_t>(len));
+        // When every chunk of the query runs at the same time, wait (bounded)
+        // until all of them have added their histograms: the bound below is
+        // then the final threshold bin.  Any earlier snapshot is still a valid
+        // (weaker) bound, so running out of time only costs candidates.
+        if (a.wait_hist) {
+            const long long t0 = clock64();
+            while (ld_acquire_u32(&a.gtot[q]) < static_cast<uint32_t>(n)) {
+                if (clock64() - t0 > kHistWaitCycles) break;
+                __nanosleep(64);
+            }
+        }
     }
     __syncthreads();
-    const uint32_t at_or_above = sm.sel.counter[1];
+    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) scratch[b] = __ldcg(&G[b]);
     __syncthreads();
+    find_digit(scratch, kSelBins, static_cast<uint32_t>(K), sm.sel);
+    const uint32_t dlow = sm.sel.res[0];
+    __syncthreads();
+    const uint32_t at_or_above = hist_sum_from(lhist, dlow, sm.sel);
     uint64_t thr = static_cast<uint64_t>(dlow) << 53;
     if (at_or_above > static_cast<uint32_t>(K)) {
         // cap at the exact local TopK: a key beaten by k keys of its own
         // chunk can never be selected; keep the intersection of both sets
-        local_top_hist(keys, len, hist);
-        find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+        find_digit(lhist, kSelBins, static_cast<uint32_t>(K), sm.sel);
         const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
         __syncthreads();
         const uint32_t need = static_cast<uint32_t>(K) - above;
         uint64_t lthr = static_cast<uint64_t>(d) << 53;
-        if (bucket != need) lthr = radix_refine(src, len, d, 1, need, hist, sm.sel);
+        if (bucket != need) lthr = radix_refine(src, len, d, 1, need, scratch, sm.sel);
         thr = lthr > thr ? lthr : thr;
     }
     uint32_t m = emit_ordered(
@@ -214,15 +234,15 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, uint32_t *hist
             __syncthreads();
             return;
         }
-        for (int j0 = 0; j0 < m; j0 += 4 * blockDim.x) {
-            uint64_t v[4];
+        for (int j0 = 0; j0 < m; j0 += 8 * blockDim.x) {
+            uint64_t v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int j = j0 + u * blockDim.x + threadIdx.x;
                 v[u] = j < m ? __ldcg(&src[j]) : 0ull;
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 const int j = j0 + u * blockDim.x + threadIdx.x;
                 if (j < m) list[total + j] = v[u];
             }
@@ -302,7 +322,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     uint8_t *stages = base + L.stages;
     uint8_t *qtile = base + L.qtile;
     uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
-    uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
+    uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);  // radix scratch
+    uint32_t *lhist = hist + kSelBins;                                  // [qg][2048]
     float *wts = reinterpret_cast<float *>(base + L.wts);
     K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
 
@@ -323,7 +344,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], 4);
+            mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b
         }
         fence_mbar_init();
     }
@@ -343,6 +364,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         const int qi = i / HP, j = i % HP;
         wts[i] = (qi < nqg && j < a.h_idx) ? bf16_bits_to_float(a.w[static_cast<int64_t>(q0 + qi) * a.h_idx + j]) : 0.f;
     }
+    if (MODE == kModeFused)
+        for (int i = tid; i < a.qg * kSelBins; i += blockDim.x) lhist[i] = 0;
     if (warp == 1) {
         tmem_alloc(&sm.tmem_base, a.tmem_cols);
         tmem_relinquish();
@@ -434,10 +457,12 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 }
             }
         } else {
-            // epilogue: warps 2..5; TMEM lane quarter = warp % 4
+            // epilogue: group 0 = warps 2..5 takes even tiles (buffer 0),
+            // group 1 = warps 6..9 odd tiles (buffer 1); TMEM lane quarter = warp % 4
             const int quarter = warp & 3;
+            const int grp = (warp - 2) >> 2;
             const int r = quarter * 32 + lane;
-            for (int t = 0; t < ntiles; ++t) {
+            for (int t = grp; t < ntiles; t += 2) {
                 const int b = t & 1;
                 const uint32_t aph = (t >> 1) & 1;
                 // every lane waits; the warp proceeds only if all saw the
@@ -485,7 +510,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                             a.scores[static_cast<int64_t>(q0 + qi) * a.ld + p] =
                                 p < sm.n_q[qi] ? score : -__int_as_float(0x7f800000);
                     } else {
-                        if (p < end) keys[qi * a.chunk + (p - start)] = float_to_key(score);
+                        const uint32_t key = float_to_key(score);
+                        if (p < end) keys[qi * a.chunk + (p - start)] = key;
+                        if (p < end && p < sm.n_q[qi]) atomicAdd(&lhist[qi * kSelBins + top_digit(key)], 1u);
                     }
                 }
                 tc_fence_before();
@@ -504,7 +531,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             const int n = sm.n_q[qi];
             if (n <= a.topk) continue;
             const int qlen = max(min(end, n) - start, 0);
-            chunk_select(a, sm, q0 + qi, keys + qi * a.chunk, start, qlen, hist);
+            chunk_select(a, sm, q0 + qi, n, keys + qi * a.chunk, start, qlen, lhist + qi * kSelBins,
+                         hist);
             __syncthreads();
         }
         if (a.P > 1) {
@@ -554,9 +582,17 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     const int end = min(start + a.chunk, n);
     const int len = max(end - start, 0);
     const float *src = a.scores + static_cast<int64_t>(q) * a.ld;
-    for (int i = threadIdx.x; i < len; i += blockDim.x) keys[i] = float_to_key(__ldg(&src[start + i]));
+    uint32_t *lhist = hist + kSelBins;
+    for (int i = threadIdx.x; i < kSelBins; i += blockDim.x) lhist[i] = 0;
     __syncthreads();
-    chunk_select(a, sm, q, keys, start, len, hist);
+    for (int i0 = 0; i0 < len; i0 += blockDim.x) {
+        const int i = i0 + threadIdx.x;
+        const uint32_t key = i < len ? float_to_key(__ldg(&src[start + i])) : 0u;
+        if (i < len) keys[i] = key;
+        hist_add(lhist, i < len, top_digit(key));
+    }
+    __syncthreads();
+    chunk_select(a, sm, q, n, keys, start, len, lhist, hist);
     __syncthreads();
     if (a.P > 1 && arrive_group(a, sm, q)) {
         uint64_t *list = reinterpret_cast<uint64_t *>(base);

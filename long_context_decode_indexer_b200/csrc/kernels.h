@@ -14,11 +14,12 @@ constexpr int kModeScores = 1;  // scores written to HBM
 constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 
 constexpr int kK1MaxStages = 12;     // TMA ring depth limit (128-row k^I tiles)
-constexpr int kK1Threads = 192;      // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
 constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
 constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
 constexpr int kSelBinsHost = 2048;
+constexpr long long kHistWaitCycles = 100000;  // ~50 us: bounded wait for a query's full histogram
 
 struct K1Params {
     // inputs
@@ -46,6 +47,8 @@ struct K1Params {
     int32_t *nsel;
     // workspace
     uint32_t *ghist;      // [nq, 2048] global top-digit histograms
+    uint32_t *gtot;       // [nq] positions counted into ghist so far
+    int32_t wait_hist;    // all CTAs are co-resident: wait (bounded) for the full histogram
     uint64_t *cand;       // [nq, P, topk] candidate composites
     int32_t *cand_cnt;    // [nq, P]
     uint32_t *done;       // [n_groups] chunks finished
@@ -76,8 +79,8 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
         if (off < need) off = need;
     }
     off = align_up(off, 128);
-    L.hist = off;
-    off += (mode != kModeScores) ? kSelBinsHost * 4u : 0u;
+    L.hist = off;  // radix scratch histogram, then one local histogram per query
+    off += (mode != kModeScores) ? static_cast<uint32_t>(qg + 1) * kSelBinsHost * 4u : 0u;
     L.wts = off;
     off += align_up(static_cast<uint32_t>(qg * hp * 4), 16);
     off = align_up(off, 128);
@@ -106,9 +109,9 @@ constexpr int kDqk = 576;           // key width (512 latent + 64 rope)
 constexpr int kDv = 512;            // value width
 constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
 constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
-constexpr int kMlaStages = 3;       // pass-1 ring depth (Q chunk + K chunk)
+constexpr int kMlaStages = 4;       // pass-1 ring depth (Q chunk + K chunk)
 constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
-constexpr int kMlaThreads = 192;    // warps 0-3 softmax/epilogue, warp 4 TMA, warp 5 MMA
+constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers
 
 struct MlaParams {
     const int32_t *q_seq;

@@ -154,9 +154,10 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
 
 // Ordered block-wide compaction: the elements i in [0, n) with pred(v) true
 // are handed to out(slot, v) with consecutive slots base, base + 1, ... in
-// increasing i.  Each thread owns 8 consecutive elements per round; a block
-// scan of the per-thread counts gives every thread its first slot.  Returns
-// the next free slot.  `wsum` is shared scratch of 32 words.
+// increasing i.  Each thread owns 8 consecutive elements per round (fetched
+// with src.get8(i0, v[8]), i0 a multiple of 8; entries past n are ignored);
+// a block scan of the per-thread counts gives every thread its first slot.
+// Returns the next free slot.  `wsum` is shared scratch of 32 words.
 template <class Src, class Pred, class Out>
 __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
                                  uint32_t base, uint32_t *wsum) {
@@ -166,13 +167,11 @@ __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const 
     for (int r0 = 0; r0 < n; r0 += round) {
         uint64_t vals[kPer];
         uint32_t mask = 0;
+        const int i0 = r0 + tid * kPer;
+        if (i0 < n) src.get8(i0, vals);
 #pragma unroll
-        for (int e = 0; e < kPer; ++e) {
-            const int i = r0 + tid * kPer + e;
-            uint64_t v = 0;
-            if (i < n && src(i, v) && pred(v)) mask |= 1u << e;
-            vals[e] = v;
-        }
+        for (int e = 0; e < kPer; ++e)
+            if (i0 + e < n && pred(vals[e])) mask |= 1u << e;
         const uint32_t cnt = static_cast<uint32_t>(__popc(mask));
         const uint32_t incl = warp_incl_scan(cnt);
         if (lane == 31) wsum[warp] = incl;

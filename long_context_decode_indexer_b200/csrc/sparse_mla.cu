@@ -9,17 +9,19 @@
 // ("split"); all 128 heads form the MMA's M dimension.
 //   pass 1  S[128 x R] = Q . K^T over 9 chunks of 64 key columns.  Each ring
 //           stage holds a Q chunk (TMA tile, 16 KB) and the R rows' matching
-//           128-byte pieces (TMA gather4, four rows per instruction); the
-//           rows were first prefetched whole into L2.  S accumulates in TMEM.
+//           128-byte pieces, gathered by four warps with 16-byte cp.async
+//           into the 128B-swizzled layout (the rows were first prefetched
+//           whole into L2).  S accumulates in TMEM.
 //   softmax one thread per head reads its S row from TMEM, takes the exact
 //           max over the split, writes P = exp(S - max) into shared memory
 //           as a pair of bf16 tiles P_hi = bf16(P), P_lo = bf16(P - P_hi)
 //           (the A operands of pass 2) and keeps the row sum.  A single bf16
 //           P would add ~1e-3 relative error on top of the ~1.7e-3 that the
 //           bf16 output itself carries; the pair makes P exact to ~2^-16.
-//   pass 2  O[128 x 512] = P_hi . V + P_lo . V, V re-gathered (32-row tiles,
-//           L2 hits) into an MN-major swizzled layout; O takes all 512 TMEM
-//           columns, which is why S and O are not live at the same time.
+//   pass 2  O[128 x 512] = P_hi . V + P_lo . V, V re-gathered by the same
+//           warps (32-row tiles, L2 hits) into an MN-major swizzled layout; O
+//           takes all 512 TMEM columns, which is why S and O are not live at
+//           the same time.
 // A split writes O / l and its log-sum-exp; the combine kernel merges splits
 // by their log-sum-exp.  With one split the CTA writes the final output.
 #include <cuda.h>
@@ -41,6 +43,9 @@ constexpr int kNumKChunks = kDqk / 64;              // 9
 constexpr int kVTileBytes = kMlaVRows * kDv * 2;    // 32 KB
 constexpr int kVBlockBytes = kMlaVRows * 128;       // one 64-column block of a V tile
 constexpr int kPBlockBytes = 128 * 128;             // 128 heads x 64 rows bf16
+constexpr int kGatherWarp0 = 6;                     // warps 6..9 gather rows
+constexpr int kGatherThreads = 128;
+constexpr int kGatherLag = 2;                       // pass-1 chunks in flight per gather thread
 
 struct MlaSmem {
     uint64_t full[kMlaStages];
@@ -55,6 +60,7 @@ struct MlaSmem {
     int32_t nvalid;
     int32_t rows[kMlaMaxRows];
     uint8_t valid[kMlaMaxRows];
+    uint32_t vmask[kMlaMaxRows / 32];  // bit j of word w: entry 32w + j is valid
 };
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -94,13 +100,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         sm.abort = 0;
         sm.nvalid = 0;
         for (int s = 0; s < kMlaStages; ++s) {
-            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.full[s], 1 + 4);  // Q TMA (with its bytes) + four gather warps
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.p_full, 4);
         for (int v = 0; v < 2; ++v) {
-            mbar_init(&sm.v_full[v], 1);
+            mbar_init(&sm.v_full[v], 4);     // four gather warps
             mbar_init(&sm.v_empty[v], 1);
         }
         mbar_init(&sm.o_full, 1);
@@ -133,6 +139,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
         sm.rows[i] = row;
         sm.valid[i] = ok;
+        const unsigned bits = __ballot_sync(0xffffffffu, ok != 0);
+        if ((i & 31) == 0) sm.vmask[i >> 5] = bits;
     }
     // rows h..127 of every Q chunk are never written by TMA: zero them once
     if (hbox < 128) {
@@ -152,68 +160,84 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 
     if (Rp > 0) {
         if (warp == 4) {
-            // ------------------------------------------------ TMA producer
-            const uint16_t *kvbase = a.kv;
-            for (int i = lane; i < R; i += 32)
-                if (sm.valid[i])
-                    prefetch_l2_bulk(kvbase + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
+            // ------------------------------------------ Q chunks by TMA
             const uint32_t qbytes = static_cast<uint32_t>(hbox) * 128u;
-            const uint32_t kbytes = static_cast<uint32_t>(Rp) * 128u;
-            for (int c = 0; c < kNumKChunks; ++c) {
-                const int s = c % kMlaStages;
-                const uint32_t ph = (c / kMlaStages) & 1;
-                bool ok = true;
-                if (lane == 0) {
-                    ok = !sm.abort && mbar_wait(&sm.empty[s], ph ^ 1);
-                    if (ok) mbar_arrive_expect_tx(&sm.full[s], qbytes + kbytes);
-                }
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) {
-                    if (lane == 0) {
+            if (lane == 0) {
+                for (int c = 0; c < kNumKChunks; ++c) {
+                    const int s = c % kMlaStages;
+                    const uint32_t ph = (c / kMlaStages) & 1;
+                    if (sm.abort || !mbar_wait(&sm.empty[s], ph ^ 1)) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
+                        break;
                     }
-                    break;
+                    mbar_arrive_expect_tx(&sm.full[s], qbytes);
+                    tma_load_2d(ring + s * kStageBytes, &qmap, &sm.full[s], c * 64, q * a.h);
                 }
-                uint8_t *st = ring + s * kStageBytes;
-                if (lane == 0) tma_load_2d(st, &qmap, &sm.full[s], c * 64, q * a.h);
-                for (int g = lane; g < Rp / 4; g += 32)
-                    tma_gather4(st + kQChunkBytes + g * 512, &kvmap, &sm.full[s], c * 64,
-                                sm.rows[4 * g], sm.rows[4 * g + 1], sm.rows[4 * g + 2], sm.rows[4 * g + 3]);
+            }
+        } else if (warp >= kGatherWarp0) {
+            // ------------------------------------------ row gathers (cp.async)
+            const int gt = tid - kGatherWarp0 * 32;  // 0..127
+            for (int i = gt; i < R; i += kGatherThreads)
+                if (sm.valid[i])
+                    prefetch_l2_bulk(a.kv + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
+            bool ok = true;
+            // pass 1: chunk c of every row -> K area of ring stage c % kMlaStages
+            for (int c = 0; c < kNumKChunks + kGatherLag; ++c) {
+                if (c < kNumKChunks) {
+                    const int s = c % kMlaStages;
+                    const uint32_t ph = (c / kMlaStages) & 1;
+                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1) && !sm.abort);
+                    if (ok) {
+                        uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
+                        for (int i = gt; i < Rp * 8; i += kGatherThreads) {
+                            const int r = i >> 3, j = i & 7;
+                            const uint16_t *src = a.kv + static_cast<int64_t>(sm.rows[r]) * a.kv_row_stride + c * 64 + j * 8;
+                            cp_async16(kst + r * 128 + ((j ^ (r & 7)) << 4), src);
+                        }
+                    }
+                    cp_async_commit();
+                }
+                if (c >= kGatherLag) {
+                    // chunk c - lag is complete for this thread: publish it
+                    if (c < kNumKChunks) cp_async_wait<kGatherLag>();
+                    else cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.full[(c - kGatherLag) % kMlaStages]);
+                }
             }
             // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is done
-            bool ok = true;
-            if (lane == 0) ok = mbar_wait(&sm.s_full, 0) && !sm.abort;
-            ok = __shfl_sync(0xffffffffu, ok, 0);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
             const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
-            for (int vt = 0; ok && vt < nvt; ++vt) {
-                const int v = vt & 1;
-                const uint32_t ph = (vt >> 1) & 1;
-                bool ok2 = true;
-                if (lane == 0) {
-                    ok2 = !sm.abort && mbar_wait(&sm.v_empty[v], ph ^ 1);
-                    if (ok2) mbar_arrive_expect_tx(&sm.v_full[v], kVTileBytes);
-                }
-                ok2 = __shfl_sync(0xffffffffu, ok2, 0);
-                if (!ok2) {
-                    if (lane == 0) {
-                        record_status(a.status, DSA_ERR_TIMEOUT);
-                        sm.abort = 1;
+            for (int vt = 0; vt < nvt + 1; ++vt) {
+                if (vt < nvt) {
+                    const int v = vt & 1;
+                    const uint32_t ph = (vt >> 1) & 1;
+                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1) && !sm.abort);
+                    if (ok) {
+                        uint8_t *vt_base = vring + v * kVTileBytes;
+                        // 32 rows x 8 column blocks x 8 pieces of 16 bytes
+                        for (int i = gt; i < kMlaVRows * 64; i += kGatherThreads) {
+                            const int r = i >> 6, blk = (i >> 3) & 7, j = i & 7;
+                            const int e = vt * kMlaVRows + r;
+                            const uint16_t *src = a.kv + static_cast<int64_t>(sm.rows[e]) * a.kv_row_stride + blk * 64 + j * 8;
+                            cp_async16(vt_base + blk * kVBlockBytes + r * 128 + ((j ^ (r & 7)) << 4), src);
+                        }
                     }
-                    break;
+                    cp_async_commit();
                 }
-                uint8_t *vt_base = vring + v * kVTileBytes;
-                // 8 column blocks x (kMlaVRows / 4) groups of 4 rows
-                constexpr int kGroups = kMlaVRows / 4;
-                for (int t = lane; t < 8 * kGroups; t += 32) {
-                    const int blk = t / kGroups, g = t % kGroups;
-                    const int r0 = vt * kMlaVRows + 4 * g;
-                    int32_t rr[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) rr[u] = (r0 + u < R) ? sm.rows[r0 + u] : 0;
-                    tma_gather4(vt_base + blk * kVBlockBytes + g * 512, &kvmap, &sm.v_full[v],
-                                blk * 64, rr[0], rr[1], rr[2], rr[3]);
+                if (vt >= 1) {
+                    if (vt < nvt) cp_async_wait<1>();
+                    else cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sm.v_full[(vt - 1) & 1]);
                 }
+            }
+            if (!ok && lane == 0) {
+                record_status(a.status, DSA_ERR_TIMEOUT);
+                sm.abort = 1;
             }
         } else if (warp == 5) {
             // ------------------------------------------------ MMA issuer
@@ -288,25 +312,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             float m = -INFINITY, l = 0.f;
             if (ok) {
                 tc_fence_after();
+                // row max: four independent partial maxima, 32 columns per TMEM load
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 for (int c0 = 0; c0 < Rp; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld32(lane_addr + c0, v);
+                    const uint32_t vm = sm.vmask[c0 >> 5];
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 32; ++j)
-                        if (c0 + j < R && sm.valid[c0 + j]) m = fmaxf(m, __uint_as_float(v[j]));
+                        m4[j & 3] = fmaxf(m4[j & 3], ((vm >> j) & 1u) ? __uint_as_float(v[j]) : -INFINITY);
                 }
+                m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
                 const float mlog = (m == -INFINITY) ? 0.f : m * a.scale_log2;
+                float l4[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int c0 = 0; c0 < Rp; c0 += 32) {
                     uint32_t v[32];
                     tmem_ld32(lane_addr + c0, v);
+                    const uint32_t vm = sm.vmask[c0 >> 5];
                     tmem_wait_ld();
                     float p[32];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
-                        const bool vj = (c0 + j < R) && sm.valid[c0 + j];
-                        p[j] = vj ? exp2f(__uint_as_float(v[j]) * a.scale_log2 - mlog) : 0.f;
-                        l += p[j];
+                        p[j] = ((vm >> j) & 1u) ? fast_exp2(fmaf(__uint_as_float(v[j]), a.scale_log2, -mlog)) : 0.f;
+                        l4[j & 3] += p[j];
                     }
                     // P row `hrow`, columns c0..c0+31: K-major 128B-swizzled blocks of 64
                     const uint32_t rowoff = (c0 >> 6) * kPBlockBytes + hrow * 128;
@@ -327,6 +356,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                         *reinterpret_cast<uint4 *>(plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     }
                 }
+                l = (l4[0] + l4[1]) + (l4[2] + l4[3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -341,10 +371,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 const bool head_ok = hrow < a.h;
                 if (a.splits == 1) {
                     uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv;
-                    for (int c0 = 0; c0 < kDv; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(lane_addr + c0, v);
+                    for (int c1 = 0; c1 < kDv; c1 += 64) {
+                        uint32_t v2[2][32];
+                        tmem_ld32(lane_addr + c1, v2[0]);
+                        tmem_ld32(lane_addr + c1 + 32, v2[1]);
                         tmem_wait_ld();
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t (&v)[32] = v2[hh];
+                        const int c0 = c1 + hh * 32;
                         if (head_ok) {
 #pragma unroll
                             for (int g8 = 0; g8 < 4; ++g8) {
@@ -356,14 +391,20 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                                 *reinterpret_cast<uint4 *>(o + c0 + g8 * 8) = u;
                             }
                         }
+                        }
                     }
                     if (head_ok) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
                 } else {
                     float *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
-                    for (int c0 = 0; c0 < kDv; c0 += 32) {
-                        uint32_t v[32];
-                        tmem_ld32(lane_addr + c0, v);
+                    for (int c1 = 0; c1 < kDv; c1 += 64) {
+                        uint32_t v2[2][32];
+                        tmem_ld32(lane_addr + c1, v2[0]);
+                        tmem_ld32(lane_addr + c1 + 32, v2[1]);
                         tmem_wait_ld();
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t (&v)[32] = v2[hh];
+                        const int c0 = c1 + hh * 32;
                         if (head_ok) {
 #pragma unroll
                             for (int g4 = 0; g4 < 8; ++g4) {
@@ -374,6 +415,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                                 f.w = __uint_as_float(v[g4 * 4 + 3]) * inv_l;
                                 *reinterpret_cast<float4 *>(o + c0 + g4 * 4) = f;
                             }
+                        }
                         }
                     }
                     if (head_ok) a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
