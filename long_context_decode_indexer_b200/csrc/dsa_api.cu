@@ -148,7 +148,8 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     if (P < 1) P = 1;
     if (mode != dsa::kModeScores) {
         // the merge list (P * topk composites) must fit on chip
-        const int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
+        int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
+        if (p_cap > dsa::kMaxChunks) p_cap = dsa::kMaxChunks;
         if (P > p_cap) {
             if (p_min > p_cap) return fail(DSA_ERR_UNSUPPORTED, "history too long for topk=%d (max_n=%d)", p->topk, p->max_n);
             P = p_cap;
@@ -229,7 +230,7 @@ size_t indexer_ws(const dsa_params *p, const IndexerPlan &pl, int mode, size_t o
     off = up(off + static_cast<size_t>(pl.n_groups) * 4, 256);
     w.zero_end = off;
     w.cand = off;
-    off = up(off + static_cast<size_t>(p->nq) * pl.P * p->topk * 8, 256);
+    off = up(off + static_cast<size_t>(p->nq) * pl.P * ((p->topk + 1) & ~1) * 8, 256);
     w.cand_cnt = off;
     off = up(off + static_cast<size_t>(p->nq) * pl.P * 4, 256);
     return off;
@@ -338,6 +339,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
         // every CTA of the launch is resident at once (one CTA per SM)
         a.wait_hist = (static_cast<int64_t>(pl.n_groups) * pl.P <= num_sms()) ? 1 : 0;
         a.cand = at<uint64_t>(ws, wl.cand);
+        a.cand_stride = (p->topk + 1) & ~1;
         a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
         cudaError_t e = cudaMemsetAsync(static_cast<uint8_t *>(ws) + wl.zero_begin, 0,
                                         wl.zero_end - wl.zero_begin, st);

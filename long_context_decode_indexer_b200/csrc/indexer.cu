@@ -51,8 +51,13 @@ struct K1Smem {
     volatile int32_t abort;
     int32_t is_last;
     int32_t n_q[kMaxGroupQueries];
-    uint32_t g_digit[kMaxGroupQueries];  // threshold bin seen in G
-    uint32_t cand_count[kMaxGroupQueries];
+    uint32_t g_digit[kMaxGroupQueries];  // final threshold bin (when the snapshot was complete)
+    uint32_t g_above[kMaxGroupQueries];  // positions in higher bins
+    int32_t g_complete[kMaxGroupQueries];
+    int32_t cand_off[kMaxChunks + 1];    // merge: prefix of the chunks' (padded) candidate counts
+    int32_t cand_n[kMaxChunks];
+    uint64_t merge_bar;                  // merge: bulk copies of the candidate lists
+    uint32_t merge_phase;
     SelectScratch sel;
 };
 
@@ -71,37 +76,30 @@ __device__ __forceinline__ void group_queries(const K1Params &a, int g, int &q0,
 }
 
 // Key of position p's score in the local chunk buffer -> composite.
+// (the key buffer is padded to a multiple of 128 entries)
 struct LocalSrc {
     const uint32_t *keys;
     int base;
-    __device__ bool operator()(int i, uint64_t &v) const {
-        v = make_composite(keys[i], static_cast<uint32_t>(base + i));
-        return true;
-    }
-    // eight consecutive elements from i0 (a multiple of 8; the buffer is
-    // padded to a multiple of 128 entries)
-    __device__ void get8(int i0, uint64_t (&v)[8]) const {
-        const uint4 a = *reinterpret_cast<const uint4 *>(keys + i0);
-        const uint4 b = *reinterpret_cast<const uint4 *>(keys + i0 + 4);
-        const uint32_t k[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = make_composite(k[e], static_cast<uint32_t>(base + i0 + e));
+    __device__ void load4(int i, uint64_t (&v)[4]) const {
+        const uint4 k = *reinterpret_cast<const uint4 *>(keys + i);
+        const uint32_t p = static_cast<uint32_t>(base + i);
+        v[0] = make_composite(k.x, p);
+        v[1] = make_composite(k.y, p + 1);
+        v[2] = make_composite(k.z, p + 2);
+        v[3] = make_composite(k.w, p + 3);
     }
 };
-// Candidates staged in shared memory (already composites).
+// Candidates staged in shared memory (already composites; the staging area
+// has room past the last entry).
 struct ListSrc {
     const uint64_t *list;
-    __device__ bool operator()(int i, uint64_t &v) const {
-        v = list[i];
-        return true;
-    }
-    __device__ void get8(int i0, uint64_t (&v)[8]) const {
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(list + i0 + e);
-            v[e] = (static_cast<uint64_t>(u.y) << 32) | u.x;
-            v[e + 1] = (static_cast<uint64_t>(u.w) << 32) | u.z;
-        }
+    __device__ void load4(int i, uint64_t (&v)[4]) const {
+        const uint4 a = *reinterpret_cast<const uint4 *>(list + i);
+        const uint4 b = *reinterpret_cast<const uint4 *>(list + i + 2);
+        v[0] = (static_cast<uint64_t>(a.y) << 32) | a.x;
+        v[1] = (static_cast<uint64_t>(a.w) << 32) | a.z;
+        v[2] = (static_cast<uint64_t>(b.y) << 32) | b.x;
+        v[3] = (static_cast<uint64_t>(b.w) << 32) | b.z;
     }
 };
 
@@ -125,8 +123,9 @@ __device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScrat
 // `lhist` the histogram of their top digits.  Every emission is an ordered
 // compaction, so results come out in ascending position order and are the
 // same from run to run.
-__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int n, const uint32_t *keys,
-                             int start, int len, const uint32_t *lhist, uint32_t *scratch) {
+__device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n,
+                             const uint32_t *keys, int start, int len, const uint32_t *lhist,
+                             uint32_t *scratch) {
     const int K = a.topk;
     LocalSrc src{keys, start};
     if (a.P == 1) {
@@ -155,7 +154,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int n, const 
     // ---- several chunks: publish this chunk's histogram, then its candidates
     uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
     const int c = blockIdx.x % a.P;
-    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * K;
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * a.cand_stride;
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
         if (lhist[b]) atomicAdd(&G[b], lhist[b]);
     __threadfence();
@@ -179,6 +178,13 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int n, const 
     __syncthreads();
     find_digit(scratch, kSelBins, static_cast<uint32_t>(K), sm.sel);
     const uint32_t dlow = sm.sel.res[0];
+    if (threadIdx.x == 0) {
+        // complete if every position of the query was counted before the snapshot
+        sm.g_complete[qi] = ld_acquire_u32(&a.gtot[q]) >= static_cast<uint32_t>(n) &&
+                            sm.sel.res[1] + sm.sel.res[2] >= static_cast<uint32_t>(K);
+        sm.g_digit[qi] = dlow;
+        sm.g_above[qi] = sm.sel.res[1];
+    }
     __syncthreads();
     const uint32_t at_or_above = hist_sum_from(lhist, dlow, sm.sel);
     uint64_t thr = static_cast<uint64_t>(dlow) << 53;
@@ -213,43 +219,61 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int n, const 
 // Chunks publish their candidates in ascending position order and chunk c
 // covers positions below chunk c + 1, so staging the lists chunk by chunk
 // keeps the whole candidate list in ascending position order.
-__device__ void group_merge(const K1Params &a, K1Smem &sm, int q, uint32_t *hist, uint64_t *list,
-                            int list_cap) {
+__device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32_t *hist,
+                            uint64_t *list, int list_cap) {
     const int K = a.topk;
-    const uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
-    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = __ldcg(&G[b]);
-    __syncthreads();
-    find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
-    const uint32_t dstar = sm.sel.res[0], above = sm.sel.res[1];
-    __syncthreads();
-    // stage all candidates (ordered) in shared memory
-    const uint64_t *cand = a.cand + static_cast<int64_t>(q) * a.P * K;
+    uint32_t dstar, above;
+    if (sm.g_complete[qi]) {
+        // this CTA's snapshot already held every chunk's histogram
+        dstar = sm.g_digit[qi];
+        above = sm.g_above[qi];
+    } else {
+        const uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
+        for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = __ldcg(&G[b]);
+        __syncthreads();
+        find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
+        dstar = sm.sel.res[0];
+        above = sm.sel.res[1];
+        __syncthreads();
+    }
+    // stage all candidates (ordered) in shared memory: one bulk copy per
+    // chunk list, each padded to an even length (16-byte units); the pad
+    // entries are set to 0, a composite no valid score reaches
+    const uint64_t *cand = a.cand + static_cast<int64_t>(q) * a.P * a.cand_stride;
     const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * a.P;
-    int total = 0;
-    for (int c = 0; c < a.P; ++c) {
-        const int m = min(__ldcg(&cnt[c]), K);
-        const uint64_t *src = cand + static_cast<int64_t>(c) * K;
-        if (total + m > list_cap) {
-            if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
-            __syncthreads();
-            return;
+    if (threadIdx.x == 0) {
+        int off = 0;
+        for (int c = 0; c < a.P; ++c) {
+            const int m = min(__ldcg(&cnt[c]), K);
+            sm.cand_off[c] = off;
+            sm.cand_n[c] = m;
+            off += (m + 1) & ~1;
         }
-        for (int j0 = 0; j0 < m; j0 += 8 * blockDim.x) {
-            uint64_t v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int j = j0 + u * blockDim.x + threadIdx.x;
-                v[u] = j < m ? __ldcg(&src[j]) : 0ull;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int j = j0 + u * blockDim.x + threadIdx.x;
-                if (j < m) list[total + j] = v[u];
-            }
-        }
-        total += m;
+        sm.cand_off[a.P] = off;
+        if (off <= list_cap) mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(off) * 8u);
     }
     __syncthreads();
+    const int total = sm.cand_off[a.P];
+    if (total > list_cap) {
+        if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        __syncthreads();
+        return;
+    }
+    if (threadIdx.x < a.P) {
+        const int c = threadIdx.x, m = sm.cand_n[c];
+        if (m > 0)
+            bulk_load(list + sm.cand_off[c], cand + static_cast<int64_t>(c) * a.cand_stride,
+                      static_cast<uint32_t>((m + 1) & ~1) * 8u, &sm.merge_bar);
+    }
+    const bool staged = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase));
+    if (threadIdx.x < a.P && (sm.cand_n[threadIdx.x] & 1)) list[sm.cand_off[threadIdx.x] + sm.cand_n[threadIdx.x]] = 0ull;
+    if (threadIdx.x == 0) sm.merge_phase ^= 1u;
+    __syncthreads();
+    if (!staged) {
+        if (threadIdx.x == 0) record_status(a.status, DSA_ERR_TIMEOUT);
+        __syncthreads();
+        return;
+    }
     // bucket d* count among the candidates must cover what is needed
     if (threadIdx.x == 0) sm.sel.counter[1] = 0;
     __syncthreads();
@@ -338,6 +362,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (tid == 0) {
         sm.abort = 0;
         sm.is_last = 0;
+        for (int i = 0; i < kMaxGroupQueries; ++i) sm.g_complete[i] = 0;
+        mbar_init(&sm.merge_bar, 1);
+        sm.merge_phase = 0;
         for (int s = 0; s < a.stages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
@@ -531,8 +558,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             const int n = sm.n_q[qi];
             if (n <= a.topk) continue;
             const int qlen = max(min(end, n) - start, 0);
-            chunk_select(a, sm, q0 + qi, n, keys + qi * a.chunk, start, qlen, lhist + qi * kSelBins,
-                         hist);
+            chunk_select(a, sm, q0 + qi, qi, n, keys + qi * a.chunk, start, qlen,
+                         lhist + qi * kSelBins, hist);
             __syncthreads();
         }
         if (a.P > 1) {
@@ -544,7 +571,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 uint64_t *list = reinterpret_cast<uint64_t *>(base);
                 const int list_cap = static_cast<int>(L.hist / sizeof(uint64_t));
                 for (int qi = 0; qi < nqg; ++qi)
-                    if (sm.n_q[qi] > a.topk) group_merge(a, sm, q0 + qi, hist, list, list_cap);
+                    if (sm.n_q[qi] > a.topk) group_merge(a, sm, q0 + qi, qi, hist, list, list_cap);
             }
         }
     }
@@ -571,6 +598,10 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
         sm.abort = 0;
         sm.is_last = 0;
         sm.n_q[0] = a.q_n[q];
+        sm.g_complete[0] = 0;
+        mbar_init(&sm.merge_bar, 1);
+        sm.merge_phase = 0;
+        fence_mbar_init();
     }
     __syncthreads();
     const int n = sm.n_q[0];
@@ -588,16 +619,18 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     for (int i0 = 0; i0 < len; i0 += blockDim.x) {
         const int i = i0 + threadIdx.x;
         const uint32_t key = i < len ? float_to_key(__ldg(&src[start + i])) : 0u;
-        if (i < len) keys[i] = key;
-        hist_add(lhist, i < len, top_digit(key));
+        if (i < len) {
+            keys[i] = key;
+            atomicAdd(&lhist[top_digit(key)], 1u);
+        }
     }
     __syncthreads();
-    chunk_select(a, sm, q, n, keys, start, len, lhist, hist);
+    chunk_select(a, sm, q, 0, n, keys, start, len, lhist, hist);
     __syncthreads();
     if (a.P > 1 && arrive_group(a, sm, q)) {
         uint64_t *list = reinterpret_cast<uint64_t *>(base);
         const int list_cap = static_cast<int>(L.hist / sizeof(uint64_t));
-        group_merge(a, sm, q, hist, list, list_cap);
+        group_merge(a, sm, q, 0, hist, list, list_cap);
     }
 }
 

@@ -17,6 +17,7 @@ constexpr int kK1MaxStages = 12;     // TMA ring depth limit (128-row k^I tiles)
 constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
 constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
+constexpr int kMaxChunks = 32;       // chunks per query group (merge bookkeeping)
 constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
 constexpr int kSelBinsHost = 2048;
 constexpr long long kHistWaitCycles = 100000;  // ~50 us: bounded wait for a query's full histogram
@@ -49,7 +50,8 @@ struct K1Params {
     uint32_t *ghist;      // [nq, 2048] global top-digit histograms
     uint32_t *gtot;       // [nq] positions counted into ghist so far
     int32_t wait_hist;    // all CTAs are co-resident: wait (bounded) for the full histogram
-    uint64_t *cand;       // [nq, P, topk] candidate composites
+    uint64_t *cand;       // [nq, P, cand_stride] candidate composites
+    int32_t cand_stride;  // topk rounded up to even (16-byte aligned chunk lists)
     int32_t *cand_cnt;    // [nq, P]
     uint32_t *done;       // [n_groups] chunks finished
     int *status;
@@ -75,7 +77,7 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
     // the last CTA of a group stages the threshold-bin candidates in the
     // area below the histogram
     if (mode != kModeScores && P > 1) {
-        const uint32_t need = static_cast<uint32_t>(P) * static_cast<uint32_t>(topk) * 8u;
+        const uint32_t need = static_cast<uint32_t>(P) * static_cast<uint32_t>(topk + 1) * 8u;
         if (off < need) off = need;
     }
     off = align_up(off, 128);
@@ -111,6 +113,7 @@ constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
 constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
 constexpr int kMlaStages = 4;       // pass-1 ring depth (Q chunk + K chunk)
 constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
+constexpr int kMlaVStages = 3;      // pass-2 ring depth
 constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers
 
 struct MlaParams {
@@ -147,16 +150,17 @@ __host__ __device__ inline MlaLayout mla_layout() {
     const uint32_t stage = 128u * 128u + kMlaMaxRows * 128u;
     const uint32_t pass1 = kMlaStages * stage;
     // pass 2: P as a hi + lo pair of bf16 tiles (128 x 256 each, 64 KB each)
-    // + 2 V tiles (32 rows x 512 bf16 = 32 KB each)
+    // + kMlaVStages V tiles (32 rows x 512 bf16 = 32 KB each)
     const uint32_t ptile = 128u * kMlaMaxRows * 2u;
     const uint32_t vtile = kMlaVRows * kDv * 2u;
     L.ring = 0;
     L.p_tile = 0;
     L.p_lo = ptile;
     L.v_ring = 2 * ptile;
-    uint32_t end = pass1 > 2 * ptile + 2 * vtile ? pass1 : 2 * ptile + 2 * vtile;
+    const uint32_t pass2 = 2 * ptile + kMlaVStages * vtile;
+    uint32_t end = pass1 > pass2 ? pass1 : pass2;
     L.misc = align_up(end, 128);
-    L.total = L.misc + 4096 + 1024;
+    L.total = L.misc + 2048 + 1024;  // barriers and row table, alignment slack
     return L;
 }
 

@@ -98,6 +98,15 @@ __device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, u
         "r"(smem_u32(bar))
         : "memory");
 }
+// Contiguous global -> shared copy by the TMA engine (both addresses 16-byte
+// aligned, bytes a multiple of 16); completion is counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
 // Ask L2 to fetch [ptr, ptr + bytes) (bytes a multiple of 16, ptr 16-aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void *ptr, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");

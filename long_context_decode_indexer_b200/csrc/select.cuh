@@ -51,16 +51,6 @@ __device__ __forceinline__ uint32_t warp_sum(uint32_t x) {
     return x;
 }
 
-// Warp-aggregated histogram increment (lanes with the same bin add once).
-__device__ __forceinline__ void hist_add(uint32_t *hist, bool active, uint32_t bin) {
-    const unsigned m = __ballot_sync(0xffffffffu, active);
-    if (active) {
-        const unsigned peers = __match_any_sync(m, bin);
-        if ((threadIdx.x & 31) == static_cast<unsigned>(__ffs(peers) - 1))
-            atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
-    }
-}
-
 // Scanning `hist` (nbins bins) from the highest bin down, find the bin where
 // the running count first reaches `need` (1 <= need <= total).  Writes
 // res[0] = bin, res[1] = count in higher bins, res[2] = count in the bin.
@@ -68,10 +58,16 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, bool active, uint32_t b
 __device__ void find_digit(const uint32_t *hist, int nbins, uint32_t need, SelectScratch &sc) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int nch = nbins >> 5;
-    for (int c = warp; c < nch; c += nwarps) {
-        uint32_t x = warp_sum(hist[c * 32 + lane]);
-        if (lane == 0) sc.csum[c] = x;
+    // chunk sums: eight threads per 32-bin chunk, four bins per 16-byte load
+    for (int t = tid; t < nbins / 4; t += blockDim.x) {
+        const uint4 h4 = reinterpret_cast<const uint4 *>(hist)[t];
+        uint32_t x = (h4.x + h4.y) + (h4.z + h4.w);
+        x += __shfl_xor_sync(0xffffffffu, x, 1);
+        x += __shfl_xor_sync(0xffffffffu, x, 2);
+        x += __shfl_xor_sync(0xffffffffu, x, 4);
+        if ((t & 7) == 0) sc.csum[t >> 3] = x;
     }
+    (void)nwarps;
     __syncthreads();
     if (warp == 0) {
         // chunks in descending order: lane l holds chunk nch-1-l and nch-33-l
@@ -115,7 +111,8 @@ __device__ void find_digit(const uint32_t *hist, int nbins, uint32_t need, Selec
 // Refine the K-th largest composite among elements of `src` whose digits
 // above pass `pass0` equal `prefix` (prefix holds the top digits, already
 // decided), needing the `need`-th largest of them (1 <= need <= their count).
-// `src(i, v)` returns true and sets v for a present element i in [0, n).
+// `src.load4(i, v)` fills v with elements i..i+3 (i a multiple of 4; the
+// source is readable up to the next multiple of 4 past n).
 // Returns the threshold T: the wanted set is {V >= T} among the elements
 // with that prefix (plus everything with a larger prefix, decided earlier).
 template <class Src>
@@ -128,18 +125,15 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
         const int hi = shift + width;
         for (int b = tid; b < nbins; b += nt) hist[b] = 0;
         __syncthreads();
-        for (int i0 = 0; i0 < n; i0 += nt) {
-            const int i = i0 + tid;
-            bool act = false;
-            uint32_t d = 0;
-            uint64_t v;
-            if (i < n && src(i, v)) {
-                if (pass == 0 || (v >> hi) == prefix) {
-                    act = true;
-                    d = static_cast<uint32_t>(v >> shift) & static_cast<uint32_t>(nbins - 1);
-                }
+        for (int i0 = 4 * tid; i0 < n; i0 += 4 * nt) {
+            uint64_t v[4];
+            src.load4(i0, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                // refinement passes see few, spread-out elements: plain atomics
+                if (i0 + e < n && (pass == 0 || (v[e] >> hi) == prefix))
+                    atomicAdd(&hist[static_cast<uint32_t>(v[e] >> shift) & static_cast<uint32_t>(nbins - 1)], 1u);
             }
-            hist_add(hist, act, d);
         }
         __syncthreads();
         find_digit(hist, nbins, need, sc);
@@ -154,62 +148,54 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
 
 // Ordered block-wide compaction: the elements i in [0, n) with pred(v) true
 // are handed to out(slot, v) with consecutive slots base, base + 1, ... in
-// increasing i.  Each thread owns 8 consecutive elements per round (fetched
-// with src.get8(i0, v[8]), i0 a multiple of 8; entries past n are ignored);
-// a block scan of the per-thread counts gives every thread its first slot.
-// Returns the next free slot.  `wsum` is shared scratch of 32 words.
+// increasing i.  Warp w owns a contiguous slice (a multiple of 128
+// elements); each lane takes four consecutive elements per step (one
+// src.load4).  Pass 1 counts, one block-wide scan of the warp counts gives
+// every warp its first slot, pass 2 emits in order with a warp scan of the
+// lanes' counts.  Returns the next free slot.  `wsum`: 32 shared words.
 template <class Src, class Pred, class Out>
 __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
                                  uint32_t base, uint32_t *wsum) {
-    constexpr int kPer = 8;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    const int round = blockDim.x * kPer;
-    for (int r0 = 0; r0 < n; r0 += round) {
-        uint64_t vals[kPer];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int per = ((n + nw - 1) / nw + 127) & ~127;
+    const int lo = min(warp * per, n), hi = min(lo + per, n);
+    uint32_t cnt = 0;
+    for (int i0 = lo + 4 * lane; i0 < hi; i0 += 128) {
+        uint64_t v[4];
+        src.load4(i0, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cnt += (i0 + e < hi && pred(v[e])) ? 1u : 0u;
+    }
+    cnt = warp_sum(cnt);
+    if (lane == 0) wsum[warp] = cnt;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+        const uint32_t c = wsum[w];
+        before += (w < warp) ? c : 0u;
+        total += c;
+    }
+    uint32_t slot = base + before;
+    for (int b0 = lo; b0 < hi; b0 += 128) {
+        const int i0 = b0 + 4 * lane;
+        uint64_t v[4] = {0, 0, 0, 0};
         uint32_t mask = 0;
-        const int i0 = r0 + tid * kPer;
-        if (i0 < n) src.get8(i0, vals);
+        if (i0 < hi) {
+            src.load4(i0, v);
 #pragma unroll
-        for (int e = 0; e < kPer; ++e)
-            if (i0 + e < n && pred(vals[e])) mask |= 1u << e;
-        const uint32_t cnt = static_cast<uint32_t>(__popc(mask));
-        const uint32_t incl = warp_incl_scan(cnt);
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        uint32_t before = 0, total = 0;
-        for (int w = 0; w < nw; ++w) {
-            const uint32_t c = wsum[w];
-            before += (w < warp) ? c : 0u;
-            total += c;
+            for (int e = 0; e < 4; ++e)
+                if (i0 + e < hi && pred(v[e])) mask |= 1u << e;
         }
-        uint32_t slot = base + before + incl - cnt;
+        const uint32_t c = static_cast<uint32_t>(__popc(mask));
+        const uint32_t incl = warp_incl_scan(c);
+        uint32_t s0 = slot + incl - c;
 #pragma unroll
-        for (int e = 0; e < kPer; ++e)
-            if ((mask >> e) & 1u) out(slot++, vals[e]);
-        base += total;
-        __syncthreads();
+        for (int e = 0; e < 4; ++e)
+            if ((mask >> e) & 1u) out(s0++, v[e]);
+        slot += __shfl_sync(0xffffffffu, incl, 31);
     }
-    return base;
-}
-
-// Block-wide compaction: every element with pred(i, v) true is handed to
-// out(slot, v) with a unique slot from counter[which] (order unspecified).
-template <class Src, class Pred, class Out>
-__device__ void emit_selected(const Src &src, int n, const Pred &pred, const Out &out,
-                              SelectScratch &sc, int which) {
-    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31;
-    for (int i0 = 0; i0 < n; i0 += nt) {
-        const int i = i0 + tid;
-        uint64_t v = 0;
-        bool sel = (i < n) && src(i, v) && pred(v);
-        const unsigned m = __ballot_sync(0xffffffffu, sel);
-        if (m) {
-            uint32_t base = 0;
-            if (lane == 0) base = atomicAdd(&sc.counter[which], static_cast<uint32_t>(__popc(m)));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (sel) out(base + __popc(m & ((1u << lane) - 1u)), v);
-        }
-    }
+    __syncthreads();
+    return base + total;
 }
 
 }  // namespace dsa

@@ -45,15 +45,17 @@ constexpr int kVBlockBytes = kMlaVRows * 128;       // one 64-column block of a 
 constexpr int kPBlockBytes = 128 * 128;             // 128 heads x 64 rows bf16
 constexpr int kGatherWarp0 = 6;                     // warps 6..9 gather rows
 constexpr int kGatherThreads = 128;
-constexpr int kGatherLag = 2;                       // pass-1 chunks in flight per gather thread
+constexpr int kGatherLag = 3;                       // pass-1 chunks in flight per gather thread
+constexpr int kVLag = 2;                            // pass-2 tiles in flight per gather thread
+constexpr int kStageRowFloats = 68;                 // epilogue staging row (64 + 4 pad)
 
 struct MlaSmem {
     uint64_t full[kMlaStages];
     uint64_t empty[kMlaStages];
     uint64_t s_full;
     uint64_t p_full;
-    uint64_t v_full[2];
-    uint64_t v_empty[2];
+    uint64_t v_full[kMlaVStages];
+    uint64_t v_empty[kMlaVStages];
     uint64_t o_full;
     uint32_t tmem_base;
     volatile int32_t abort;
@@ -62,6 +64,8 @@ struct MlaSmem {
     uint8_t valid[kMlaMaxRows];
     uint32_t vmask[kMlaMaxRows / 32];  // bit j of word w: entry 32w + j is valid
 };
+
+static_assert(sizeof(MlaSmem) <= 2048, "MlaSmem must fit the reserve in mla_layout()");
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -105,7 +109,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
         mbar_init(&sm.s_full, 1);
         mbar_init(&sm.p_full, 4);
-        for (int v = 0; v < 2; ++v) {
+        for (int v = 0; v < kMlaVStages; ++v) {
             mbar_init(&sm.v_full[v], 4);     // four gather warps
             mbar_init(&sm.v_empty[v], 1);
         }
@@ -210,10 +214,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is done
             ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
             const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
-            for (int vt = 0; vt < nvt + 1; ++vt) {
+            for (int vt = 0; vt < nvt + kVLag; ++vt) {
                 if (vt < nvt) {
-                    const int v = vt & 1;
-                    const uint32_t ph = (vt >> 1) & 1;
+                    const int v = vt % kMlaVStages;
+                    const uint32_t ph = (vt / kMlaVStages) & 1;
                     ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1) && !sm.abort);
                     if (ok) {
                         uint8_t *vt_base = vring + v * kVTileBytes;
@@ -227,12 +231,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     }
                     cp_async_commit();
                 }
-                if (vt >= 1) {
-                    if (vt < nvt) cp_async_wait<1>();
+                if (vt >= kVLag && vt - kVLag < nvt) {
+                    if (vt < nvt) cp_async_wait<kVLag>();
                     else cp_async_wait<0>();
                     fence_proxy_async_smem();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.v_full[(vt - 1) & 1]);
+                    if (lane == 0) mbar_arrive(&sm.v_full[(vt - kVLag) % kMlaVStages]);
                 }
             }
             if (!ok && lane == 0) {
@@ -271,8 +275,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     const uint32_t idesc2 = make_idesc(1, 1, 0, 1, 128, 256);
                     const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
                     for (int vt = 0; vt < nvt; ++vt) {
-                        const int v = vt & 1;
-                        const uint32_t ph = (vt >> 1) & 1;
+                        const int v = vt % kMlaVStages;
+                        const uint32_t ph = (vt / kMlaVStages) & 1;
                         if (sm.abort || !mbar_wait(&sm.v_full[v], ph)) {
                             ok = false;
                             break;
@@ -368,57 +372,39 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 const bool has = l > 0.f;
                 const float inv_l = has ? 1.f / l : 0.f;
                 const float lse_v = has ? (m * a.scale + logf(l)) : -INFINITY;
-                const bool head_ok = hrow < a.h;
-                if (a.splits == 1) {
-                    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv;
-                    for (int c1 = 0; c1 < kDv; c1 += 64) {
-                        uint32_t v2[2][32];
-                        tmem_ld32(lane_addr + c1, v2[0]);
-                        tmem_ld32(lane_addr + c1 + 32, v2[1]);
-                        tmem_wait_ld();
+                if (hrow < a.h) {
+                    if (a.splits == 1) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
+                    else a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
+                }
+                // O / l, 64 columns at a time: TMEM -> padded staging rows ->
+                // coalesced row stores (a warp writes one output row per step)
+                float *stage = reinterpret_cast<float *>(ptile);  // pass-2 area is free now
+                const int64_t prow0 = (static_cast<int64_t>(wq) * a.splits + sp) * 128;
+                for (int c1 = 0, blk = 0; c1 < kDv; c1 += 64, ++blk) {
+                    float *buf = stage + (blk & 1) * (128 * kStageRowFloats);
+                    uint32_t v2[2][32];
+                    tmem_ld32(lane_addr + c1, v2[0]);
+                    tmem_ld32(lane_addr + c1 + 32, v2[1]);
+                    tmem_wait_ld();
+                    float *row = buf + hrow * kStageRowFloats;
 #pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t (&v)[32] = v2[hh];
-                        const int c0 = c1 + hh * 32;
-                        if (head_ok) {
-#pragma unroll
-                            for (int g8 = 0; g8 < 4; ++g8) {
-                                uint4 u;
-                                u.x = pack_bf16x2(__uint_as_float(v[g8 * 8 + 0]) * inv_l, __uint_as_float(v[g8 * 8 + 1]) * inv_l);
-                                u.y = pack_bf16x2(__uint_as_float(v[g8 * 8 + 2]) * inv_l, __uint_as_float(v[g8 * 8 + 3]) * inv_l);
-                                u.z = pack_bf16x2(__uint_as_float(v[g8 * 8 + 4]) * inv_l, __uint_as_float(v[g8 * 8 + 5]) * inv_l);
-                                u.w = pack_bf16x2(__uint_as_float(v[g8 * 8 + 6]) * inv_l, __uint_as_float(v[g8 * 8 + 7]) * inv_l);
-                                *reinterpret_cast<uint4 *>(o + c0 + g8 * 8) = u;
-                            }
-                        }
-                        }
+                    for (int g4 = 0; g4 < 16; ++g4) {
+                        const uint32_t *u = &v2[g4 >> 3][(g4 & 7) * 4];
+                        *reinterpret_cast<float4 *>(row + g4 * 4) =
+                            make_float4(__uint_as_float(u[0]) * inv_l, __uint_as_float(u[1]) * inv_l,
+                                        __uint_as_float(u[2]) * inv_l, __uint_as_float(u[3]) * inv_l);
                     }
-                    if (head_ok) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
-                } else {
-                    float *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
-                    for (int c1 = 0; c1 < kDv; c1 += 64) {
-                        uint32_t v2[2][32];
-                        tmem_ld32(lane_addr + c1, v2[0]);
-                        tmem_ld32(lane_addr + c1 + 32, v2[1]);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t (&v)[32] = v2[hh];
-                        const int c0 = c1 + hh * 32;
-                        if (head_ok) {
-#pragma unroll
-                            for (int g4 = 0; g4 < 8; ++g4) {
-                                float4 f;
-                                f.x = __uint_as_float(v[g4 * 4 + 0]) * inv_l;
-                                f.y = __uint_as_float(v[g4 * 4 + 1]) * inv_l;
-                                f.z = __uint_as_float(v[g4 * 4 + 2]) * inv_l;
-                                f.w = __uint_as_float(v[g4 * 4 + 3]) * inv_l;
-                                *reinterpret_cast<float4 *>(o + c0 + g4 * 4) = f;
-                            }
-                        }
-                        }
+                    asm volatile("bar.sync 1, 128;" ::: "memory");
+                    for (int rr = 0; rr < 32; ++rr) {
+                        const int r = warp * 32 + rr;
+                        if (r >= a.h) break;
+                        const float2 f = *reinterpret_cast<const float2 *>(buf + r * kStageRowFloats + 2 * lane);
+                        if (a.splits == 1)
+                            *reinterpret_cast<uint32_t *>(a.out + (static_cast<int64_t>(q) * a.h + r) * kDv + c1 + 2 * lane) =
+                                pack_bf16x2(f.x, f.y);
+                        else
+                            *reinterpret_cast<float2 *>(a.part_o + (prow0 + r) * kDv + c1 + 2 * lane) = f;
                     }
-                    if (head_ok) a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
                 }
             } else if (lane == 0) {
                 record_status(a.status, DSA_ERR_TIMEOUT);
