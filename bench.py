@@ -44,6 +44,28 @@ DEFAULT_WORKLOAD = CONFIGS[3]["name"]
 L2_BYTES = 126 * 1024 * 1024
 
 
+# DRAM traffic of the fused indexer from one ncu capture (see
+# profiles/k1_indexer_long_decode_16x96k.md): read + write bytes per scored
+# position, valid only while the kernel sources hash to the captured build.
+K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
+              "long_context_decode_indexer_b200/csrc/select.cuh",
+              "long_context_decode_indexer_b200/csrc/ptx.cuh",
+              "long_context_decode_indexer_b200/csrc/kernels.h")
+K1_PROFILED = {"sha256_16": "eb56cc5ce509249b", "bytes_per_position": 130.80875651041666}
+
+
+def k1_traffic(inp):
+    import hashlib
+    h = hashlib.sha256()
+    for f in K1_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != K1_PROFILED["sha256_16"]:
+        return None
+    n = inp.q_n.astype(np.int64)
+    return float(K1_PROFILED["bytes_per_position"] * n[n > inp.topk].sum())
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -293,7 +315,7 @@ def run_ours(args, world, rank):
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "flushed (256 MiB write) before every timed step"},
         "roofline": {"bound": "hbm", "achieved": idx_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": idx_gbs / hbm, "traffic": None,
+                     "frac": idx_gbs / hbm, "traffic": k1_traffic(inp),
                      "kernel": "k1_indexer (fused indexer + TopK)",
                      "peak_source": peak_kind},
         "stages": {
