@@ -212,6 +212,30 @@ int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
                       void *out, float *lse, int32_t *idx_out, void *ws,
                       size_t ws_bytes, void *stream);
 
+/* dsa_indexer_topk without a workspace, for callers that cannot allocate
+ * device memory (their allocator owns the device, they run under a fixed
+ * memory budget, or they must not enter the driver's allocator on this
+ * path).  The pages have no counterpart: this is a deployment variant of
+ * steps 1 + 2, same arguments and same results as dsa_indexer_topk.
+ *   - Scratch lives in one fixed 8 MiB device array inside the library;
+ *     every GPU that loads the library holds it until the process exits.
+ *     A shape needing more scratch is rejected with DSA_ERR_UNSUPPORTED
+ *     before anything is launched (decode batches of up to about 48
+ *     queries at 128K context fit).
+ *   - The call allocates nothing (no cudaMalloc, no allocating library
+ *     call).  The first call on each device resolves the array's device
+ *     address (cudaGetSymbolAddress); make that first call outside any
+ *     stream capture.
+ *   - All calls share the array and it keeps the last call's contents: the
+ *     call clears what must start at zero itself, but calls whose work
+ *     overlaps on the GPU (other streams, other threads) race; serialise them.
+ *   - status (device int32, nullable) receives the device status word of
+ *     this call (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK) in stream
+ *     order; dsa_check_status does not apply (there is no ws). */
+int dsa_indexer_topk_static(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
+                            const void *w, const void *kidx_cache, const float *k_scale,
+                            int32_t *idx, int32_t *nsel, int32_t *status, void *stream);
+
 /* Synchronise `stream`, return the device status word stored in `ws`
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE_CHECK) and clear it. */
 int dsa_check_status(void *ws, void *stream);

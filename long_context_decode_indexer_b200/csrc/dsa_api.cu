@@ -595,3 +595,82 @@ int dsa_check_status(void *ws, void *stream) {
 const char *dsa_last_error(void) { return g_err; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Fused indexer + TopK with scratch in a fixed device array.
+//
+// For callers that cannot call cudaMalloc -- code running where allocation is
+// off limits (inside a framework whose allocator owns all device memory, a
+// runtime with a fixed memory budget, a real-time path that must not enter
+// the driver's allocator) -- the scratch this operation needs lives in one
+// file-scope device array instead of a caller-provided workspace.  Every GPU
+// that loads this library holds the array until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+// Device address of the array for the current device, resolved once per
+// device (cudaGetSymbolAddress, with that device current).  In host code the
+// array's name is only a host-side stand-in, never a device address.
+int static_scratch(void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+        g_static_ptr[dev] = ptr;
+    }
+    *out = g_static_ptr[dev];
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_indexer_topk_static(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,
+                            const void *kidx_cache, const float *k_scale, int32_t *idx,
+                            int32_t *nsel, int32_t *status, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (!rc) rc = check_indexer_inputs(p, q_idx, w, kidx_cache);
+    if (rc) return rc;
+    if (p->nq > 0 && !idx) return fail(DSA_ERR_INVALID_ARG, "idx is NULL");
+    WsLayout wl;
+    IndexerPlan pl;
+    rc = layout_for(p, DSA_OP_INDEXER_TOPK, wl, &pl, nullptr, p->max_n);
+    if (rc) return rc;
+    if (wl.total > kStaticScratchBytes)
+        return fail(DSA_ERR_UNSUPPORTED,
+                    "dsa_indexer_topk_static: this shape needs %zu bytes of scratch, the fixed "
+                    "array holds %zu (use dsa_indexer_topk with a workspace)",
+                    wl.total, kStaticScratchBytes);
+    void *ws = nullptr;
+    rc = static_scratch(&ws);
+    if (rc) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the array keeps the previous call's contents: start from a clear status
+    // word (the per-call counters and histograms are cleared by run_indexer)
+    cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+    rc = run_indexer(p, kv, dsa::kModeFused, q_idx, w, kidx_cache, k_scale, nullptr, 0, idx, nsel,
+                     ws, wl, pl, st);
+    if (rc) return rc;
+    if (status) {
+        e = cudaMemcpyAsync(status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync(status)");
+    }
+    return DSA_OK;
+}
+
+}  // extern "C"

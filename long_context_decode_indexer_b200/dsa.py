@@ -34,7 +34,7 @@ OP_FORWARD = 5
 ENTRY_POINTS = (
     "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk",
     "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill", "dsa_forward", "dsa_forward_paged",
-    "dsa_check_status", "dsa_last_error",
+    "dsa_indexer_topk_static", "dsa_check_status", "dsa_last_error",
 )
 
 
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
             for name in ("dsa_forward", "dsa_forward_paged"):
                 getattr(L, name).argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
                                              _P, _P, _P, ctypes.c_size_t, _P]
+            L.dsa_indexer_topk_static.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, _P]
             L.dsa_check_status.argtypes = [_P, _P]
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ENTRY_POINTS[:-1]:
@@ -152,6 +153,14 @@ def indexer_topk(p, kv, q_idx, w, kidx_cache, k_scale, idx, nsel, ws, stream=Non
                                   _ptr(kidx_cache), _ptr(k_scale), _ptr(idx), _ptr(nsel), _ptr(ws),
                                   ws.numel() * ws.element_size(), _stream(stream)),
            "dsa_indexer_topk")
+
+
+def indexer_topk_static(p, kv, q_idx, w, kidx_cache, k_scale, idx, nsel, status, stream=None):
+    """dsa_indexer_topk with the library's fixed scratch array (no workspace)."""
+    _check(lib().dsa_indexer_topk_static(ctypes.byref(p), ctypes.byref(kv), _ptr(q_idx), _ptr(w),
+                                         _ptr(kidx_cache), _ptr(k_scale), _ptr(idx), _ptr(nsel),
+                                         _ptr(status), _stream(stream)),
+           "dsa_indexer_topk_static")
 
 
 def sparse_mla_decode(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, stream=None):
