@@ -220,8 +220,9 @@ int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  *   - Scratch lives in one fixed 8 MiB device array inside the library;
  *     every GPU that loads the library holds it until the process exits.
  *     A shape needing more scratch is rejected with DSA_ERR_UNSUPPORTED
- *     before anything is launched (decode batches of up to about 48
- *     queries at 128K context fit).
+ *     before anything is launched.  On a 148-SM B200 a decode batch of
+ *     up to 78 queries at 128K context (204 at 32K) fits;
+ *     dsa_workspace_size(DSA_OP_INDEXER_TOPK) gives a shape's need.
  *   - The call allocates nothing (no cudaMalloc, no allocating library
  *     call).  The first call on each device resolves the array's device
  *     address (cudaGetSymbolAddress); make that first call outside any
