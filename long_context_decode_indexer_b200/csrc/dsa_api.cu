@@ -115,7 +115,7 @@ int check_kv(const dsa_params *p, const dsa_kv *kv) {
 
 // ----------------------------------------------------------------- planning
 struct IndexerPlan {
-    int hp, qg, gpb, n_groups, P, chunk, stages;
+    int hp, qg, gpb, n_groups, P, chunk, stages, acc_bufs;
     uint32_t tmem_cols;
     size_t smem;
 };
@@ -161,8 +161,9 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     P = (sp + chunk - 1) / chunk;
     pl.P = static_cast<int>(P);
     pl.chunk = static_cast<int>(chunk);
+    pl.acc_bufs = (dsa::kK1MaxAcc * pl.qg * pl.hp <= 512) ? dsa::kK1MaxAcc : 2;
     uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(2 * pl.qg * pl.hp)) cols <<= 1;
+    while (cols < static_cast<uint32_t>(pl.acc_bufs * pl.qg * pl.hp)) cols <<= 1;
     pl.tmem_cols = cols;
     // TMA ring: as many 128-row tiles as the shared memory left by the keys holds
     // (the merge area reuses the ring once streaming is over)
@@ -326,6 +327,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.P = pl.P;
     a.chunk = pl.chunk;
     a.stages = pl.stages;
+    a.acc_bufs = pl.acc_bufs;
     a.tmem_cols = pl.tmem_cols;
     a.scores = scores;
     a.ld = ld;

@@ -10,10 +10,12 @@
 // sequence; a group's history [0, span) is cut into P chunks, one CTA each.
 // A CTA streams its chunk of the FP8 index-K cache through a TMA ring, and
 // the tensor cores compute D[128 positions x qg*hp heads] = K_tile . Q^T
-// (tcgen05 kind::f8f6f4, M = 128, N = qg*hp, K = d_I) into a double-buffered
-// TMEM accumulator.  Two groups of four epilogue warps, one per accumulator
-// buffer (even and odd tiles), read D back (one TMEM lane = one position per
-// thread) and apply ReLU, * w, the head sum and * k_s.
+// (tcgen05 kind::f8f6f4, M = 128, N = qg*hp, K = d_I) into a ring of two or
+// four TMEM accumulators.  Two groups of four epilogue warps (even and odd
+// tiles) read D back (one TMEM lane = one position per thread) and apply
+// ReLU, * w, the head sum and * k_s.  With four accumulators the tensor cores
+// run two tiles ahead of each group, so the round trip epilogue -> MMA issue
+// -> MMA completion no longer paces the stream.
 //
 // Fused mode keeps the chunk's scores in shared memory as order-preserving
 // keys.  Exact selection across chunks without a grid barrier:
@@ -45,8 +47,8 @@ constexpr int kTileRows = 128;
 struct K1Smem {
     uint64_t full[kK1MaxStages];
     uint64_t empty[kK1MaxStages];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
+    uint64_t acc_full[kK1MaxAcc];
+    uint64_t acc_empty[kK1MaxAcc];
     uint32_t tmem_base;
     volatile int32_t abort;
     int32_t is_last;
@@ -54,12 +56,15 @@ struct K1Smem {
     uint32_t g_digit[kMaxGroupQueries];  // final threshold bin (when the snapshot was complete)
     uint32_t g_above[kMaxGroupQueries];  // positions in higher bins
     int32_t g_complete[kMaxGroupQueries];
+    uint32_t g_seen;                     // positions counted into G before the snapshot
     int32_t cand_off[kMaxChunks + 1];    // merge: prefix of the chunks' (padded) candidate counts
     int32_t cand_n[kMaxChunks];
     uint64_t merge_bar;                  // merge: bulk copies of the candidate lists
     uint32_t merge_phase;
     SelectScratch sel;
 };
+
+static_assert(sizeof(K1Smem) <= 1024, "K1Smem must fit the 1 KB misc area of k1_layout");
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -172,6 +177,11 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
                 __nanosleep(64);
             }
         }
+        // Read the count BEFORE the snapshot: every chunk adds its histogram
+        // to G before its count to gtot, so if the count already covers all n
+        // positions here, the snapshot below holds every chunk's histogram.
+        // (Read after the snapshot, it could cover chunks the snapshot missed.)
+        sm.g_seen = ld_acquire_u32(&a.gtot[q]);
     }
     __syncthreads();
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) scratch[b] = __ldcg(&G[b]);
@@ -180,7 +190,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
     const uint32_t dlow = sm.sel.res[0];
     if (threadIdx.x == 0) {
         // complete if every position of the query was counted before the snapshot
-        sm.g_complete[qi] = ld_acquire_u32(&a.gtot[q]) >= static_cast<uint32_t>(n) &&
+        sm.g_complete[qi] = sm.g_seen >= static_cast<uint32_t>(n) &&
                             sm.sel.res[1] + sm.sel.res[2] >= static_cast<uint32_t>(K);
         sm.g_digit[qi] = dlow;
         sm.g_above[qi] = sm.sel.res[1];
@@ -369,9 +379,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < a.acc_bufs; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b
+            mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b % 2
         }
         fence_mbar_init();
     }
@@ -426,32 +436,42 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (ntiles > 0) {
         if (warp == 0) {
             if (lane == 0) {
-                const bool paged = a.page_table != nullptr;
-                const int64_t row0 = paged ? 0 : a.seq_row0[seq];
-                const int box = paged ? a.page_size : kTileRows;
-                for (int t = 0; t < ntiles && !sm.abort; ++t) {
-                    const int s = t % a.stages;
-                    const uint32_t ph = (t / a.stages) & 1;
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1)) {
-                        record_status(a.status, DSA_ERR_TIMEOUT);
-                        sm.abort = 1;
-                        break;
+                // ring position (s, ph) advances by one per tile: no divisions
+                // in this single-thread loop, which paces the whole stream
+                int s = 0;
+                uint32_t ph = 0;
+                if (a.page_table == nullptr) {
+                    int32_t row = static_cast<int32_t>(a.seq_row0[seq] + start);
+                    for (int t = 0; t < ntiles; ++t, row += kTileRows) {
+                        if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
+                            record_status(a.status, DSA_ERR_TIMEOUT);
+                            sm.abort = 1;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+                        tma_load_2d(stages + s * kTileBytes, &kmap, &sm.full[s], 0, row);
+                        if (++s == a.stages) { s = 0; ph ^= 1; }
                     }
-                    const int p0 = start + t * kTileRows;
-                    uint32_t bytes = 0;
-                    for (int h = 0; h < kTileRows / box; ++h)
-                        if (p0 + h * box < nmax) bytes += box * DI;
-                    mbar_arrive_expect_tx(&sm.full[s], bytes);
-                    uint8_t *dst = stages + s * kTileBytes;
-                    for (int h = 0; h < kTileRows / box; ++h) {
-                        const int pp = p0 + h * box;
-                        if (pp >= nmax) break;
-                        int64_t row;
-                        if (paged)
-                            row = static_cast<int64_t>(a.page_table[static_cast<int64_t>(seq) * a.max_pages + pp / box]) * box;
-                        else
-                            row = row0 + pp;
-                        tma_load_2d(dst + h * box * DI, &kmap, &sm.full[s], 0, static_cast<int32_t>(row));
+                } else {
+                    const int box = a.page_size;
+                    const int per_tile = kTileRows / box;
+                    const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages;
+                    int page = start / box;
+                    for (int t = 0; t < ntiles; ++t) {
+                        if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
+                            record_status(a.status, DSA_ERR_TIMEOUT);
+                            sm.abort = 1;
+                            break;
+                        }
+                        const int p0 = start + t * kTileRows;
+                        int n_box = 0;
+                        for (int h = 0; h < per_tile; ++h) n_box += (p0 + h * box < nmax);
+                        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
+                        uint8_t *dst = stages + s * kTileBytes;
+                        for (int h = 0; h < n_box; ++h, dst += box * DI)
+                            tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[page + h] * box);
+                        page += per_tile;
+                        if (++s == a.stages) { s = 0; ph ^= 1; }
                     }
                 }
             }
@@ -460,27 +480,27 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 const uint32_t idesc = make_idesc(0, 0, 0, 0, kTileRows, N);
                 constexpr uint32_t kSbo = 8 * DI;
                 constexpr uint32_t kLayout = (DI == 128) ? kSwizzle128B : kSwizzle64B;
-                const uint32_t qaddr = smem_u32(qtile);
-                for (int t = 0; t < ntiles && !sm.abort; ++t) {
-                    const int s = t % a.stages;
-                    const uint32_t ph = (t / a.stages) & 1;
-                    const int b = t & 1;
-                    const uint32_t aph = (t >> 1) & 1;
-                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1) || !mbar_wait(&sm.full[s], ph)) {
+                // descriptors of stage 0 and of the q tile; a stage (or a 32-byte
+                // K step) is a fixed offset in the 16-byte address field
+                const uint64_t ad0 = make_sdesc(smem_u32(stages), 16, kSbo, kLayout);
+                const uint64_t bd0 = make_sdesc(smem_u32(qtile), 16, kSbo, kLayout);
+                int s = 0, b = 0;
+                uint32_t ph = 0, aph = 0;
+                for (int t = 0; t < ntiles; ++t) {
+                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1) || !mbar_wait(&sm.full[s], ph) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t kaddr = smem_u32(stages + s * kTileBytes);
+                    const uint64_t ad = ad0 + static_cast<uint64_t>(s * (kTileBytes >> 4));
 #pragma unroll
-                    for (int kk = 0; kk < DI / 32; ++kk) {
-                        const uint64_t ad = make_sdesc(kaddr + kk * 32, 16, kSbo, kLayout);
-                        const uint64_t bd = make_sdesc(qaddr + kk * 32, 16, kSbo, kLayout);
-                        mma_f8_ss(tmem + b * N, ad, bd, idesc, kk > 0 ? 1u : 0u);
-                    }
+                    for (int kk = 0; kk < DI / 32; ++kk)
+                        mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                     tc_commit(&sm.empty[s]);
                     tc_commit(&sm.acc_full[b]);
+                    if (++s == a.stages) { s = 0; ph ^= 1; }
+                    if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
                 }
             }
         } else {
@@ -489,9 +509,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             const int quarter = warp & 3;
             const int grp = (warp - 2) >> 2;
             const int r = quarter * 32 + lane;
+            // this group's tiles t = grp, grp + 2, ... use buffers grp, grp + 2, ...
+            int b = grp;
+            uint32_t aph = 0;
             for (int t = grp; t < ntiles; t += 2) {
-                const int b = t & 1;
-                const uint32_t aph = (t >> 1) & 1;
                 // every lane waits; the warp proceeds only if all saw the
                 // phase complete (tcgen05.ld below is warp-collective)
                 const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], aph) && !sm.abort);
@@ -516,8 +537,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 for (int qi = 0; qi < nqg; ++qi) {
                     const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) +
                                            static_cast<uint32_t>(b * N + qi * HP);
-                    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-                    const float *wq = wts + qi * HP;
+                    // four running sums (heads j mod 4), kept as two pairs
+                    float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
+                    const float4 *wq = reinterpret_cast<const float4 *>(wts + qi * HP);
                     uint32_t v[HP];
                     // issue every load of the row, then wait once
 #pragma unroll
@@ -526,12 +548,17 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < HP; j += 4) {
-                        acc0 = fmaf(wq[j + 0], fmaxf(__uint_as_float(v[j + 0]), 0.f), acc0);
-                        acc1 = fmaf(wq[j + 1], fmaxf(__uint_as_float(v[j + 1]), 0.f), acc1);
-                        acc2 = fmaf(wq[j + 2], fmaxf(__uint_as_float(v[j + 2]), 0.f), acc2);
-                        acc3 = fmaf(wq[j + 3], fmaxf(__uint_as_float(v[j + 3]), 0.f), acc3);
+                        const float4 w4 = wq[j / 4];
+                        acc01 = fma2(make_float2(w4.x, w4.y),
+                                     make_float2(fmaxf(__uint_as_float(v[j + 0]), 0.f),
+                                                 fmaxf(__uint_as_float(v[j + 1]), 0.f)),
+                                     acc01);
+                        acc23 = fma2(make_float2(w4.z, w4.w),
+                                     make_float2(fmaxf(__uint_as_float(v[j + 2]), 0.f),
+                                                 fmaxf(__uint_as_float(v[j + 3]), 0.f)),
+                                     acc23);
                     }
-                    const float score = ((acc0 + acc1) + (acc2 + acc3)) * ks;
+                    const float score = ((acc01.x + acc01.y) + (acc23.x + acc23.y)) * ks;
                     if (MODE == kModeScores) {
                         if (p < end)
                             a.scores[static_cast<int64_t>(q0 + qi) * a.ld + p] =
@@ -545,6 +572,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
+                b += 2;
+                if (b >= a.acc_bufs) { b -= a.acc_bufs; aph ^= 1; }
             }
         }
     }

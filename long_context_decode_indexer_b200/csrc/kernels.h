@@ -14,6 +14,7 @@ constexpr int kModeScores = 1;  // scores written to HBM
 constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 
 constexpr int kK1MaxStages = 12;     // TMA ring depth limit (128-row k^I tiles)
+constexpr int kK1MaxAcc = 4;         // TMEM accumulator buffers (even: one parity per epilogue group)
 constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
 constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
@@ -40,6 +41,7 @@ struct K1Params {
     int32_t P;      // chunks per group
     int32_t chunk;  // positions per chunk (multiple of 128)
     int32_t stages; // TMA ring depth
+    int32_t acc_bufs;  // TMEM accumulator buffers of qg*hp columns (2 or 4)
     uint32_t tmem_cols;
     // outputs
     float *scores;  // kModeScores output / kModeTopk input
