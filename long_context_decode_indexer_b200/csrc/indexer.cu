@@ -108,6 +108,20 @@ struct ListSrc {
     }
 };
 
+// Copy a query's global histogram (2048 words, L2) to shared memory.  All
+// of a thread's loads are issued before any store, so the copy costs one L2
+// round trip instead of one per loop iteration.  Needs blockDim >= 256.
+__device__ __forceinline__ void load_global_hist(uint32_t *dst, const uint32_t *G) {
+    constexpr int kVec = kSelBins / 4;  // 512 uint4
+    const uint4 *src = reinterpret_cast<const uint4 *>(G);
+    const int i0 = threadIdx.x, i1 = threadIdx.x + blockDim.x;
+    const uint4 zero = make_uint4(0, 0, 0, 0);
+    const uint4 v0 = i0 < kVec ? __ldcg(src + i0) : zero;
+    const uint4 v1 = i1 < kVec ? __ldcg(src + i1) : zero;
+    if (i0 < kVec) reinterpret_cast<uint4 *>(dst)[i0] = v0;
+    if (i1 < kVec) reinterpret_cast<uint4 *>(dst)[i1] = v1;
+}
+
 // Sum of hist[b] for b >= lo (block-wide; every thread gets the result).
 __device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScratch &sc) {
     if (threadIdx.x == 0) sc.counter[2] = 0;
@@ -184,7 +198,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
         sm.g_seen = ld_acquire_u32(&a.gtot[q]);
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) scratch[b] = __ldcg(&G[b]);
+    load_global_hist(scratch, G);
     __syncthreads();
     find_digit(scratch, kSelBins, static_cast<uint32_t>(K), sm.sel);
     const uint32_t dlow = sm.sel.res[0];
@@ -239,7 +253,7 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
         above = sm.g_above[qi];
     } else {
         const uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
-        for (int b = threadIdx.x; b < kSelBins; b += blockDim.x) hist[b] = __ldcg(&G[b]);
+        load_global_hist(hist, G);
         __syncthreads();
         find_digit(hist, kSelBins, static_cast<uint32_t>(K), sm.sel);
         dstar = sm.sel.res[0];
@@ -251,16 +265,22 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
     // entries are set to 0, a composite no valid score reaches
     const uint64_t *cand = a.cand + static_cast<int64_t>(q) * a.P * a.cand_stride;
     const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * a.P;
-    if (threadIdx.x == 0) {
-        int off = 0;
-        for (int c = 0; c < a.P; ++c) {
-            const int m = min(__ldcg(&cnt[c]), K);
-            sm.cand_off[c] = off;
+    if (threadIdx.x < 32) {
+        // one lane per chunk (P <= 32): the counts are loaded in parallel,
+        // the offsets are a warp scan of the padded counts
+        const int c = threadIdx.x;
+        const int m = c < a.P ? min(__ldcg(&cnt[c]), K) : 0;
+        const int padded = (m + 1) & ~1;
+        const int incl = static_cast<int>(warp_incl_scan(static_cast<uint32_t>(padded)));
+        if (c < a.P) {
+            sm.cand_off[c] = incl - padded;
             sm.cand_n[c] = m;
-            off += (m + 1) & ~1;
         }
-        sm.cand_off[a.P] = off;
-        if (off <= list_cap) mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(off) * 8u);
+        const int off = __shfl_sync(0xffffffffu, incl, 31);
+        if (c == 0) {
+            sm.cand_off[a.P] = off;
+            if (off <= list_cap) mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(off) * 8u);
+        }
     }
     __syncthreads();
     const int total = sm.cand_off[a.P];
@@ -284,29 +304,13 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
         __syncthreads();
         return;
     }
-    // bucket d* count among the candidates must cover what is needed
-    if (threadIdx.x == 0) sm.sel.counter[1] = 0;
-    __syncthreads();
-    {
-        uint32_t n_b = 0;
-        for (int i = threadIdx.x; i < total; i += blockDim.x)
-            n_b += static_cast<uint32_t>(list[i] >> 53) == dstar;
-        n_b = warp_sum(n_b);
-        if ((threadIdx.x & 31) == 0) atomicAdd(&sm.sel.counter[1], n_b);
-    }
-    __syncthreads();
-    const uint32_t nbucket = sm.sel.counter[1];
-    __syncthreads();
+    // the need-th largest candidate of bucket d* is the threshold (if the
+    // candidates held fewer than `need` of the bucket, the emission count
+    // below comes out short and flags it)
     const uint32_t need = static_cast<uint32_t>(K) - above;
     int32_t *out = a.idx + static_cast<int64_t>(q) * K;
-    if (nbucket < need) {
-        if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
-        __syncthreads();
-        return;
-    }
     ListSrc src{list};
-    uint64_t thr = static_cast<uint64_t>(dstar) << 53;
-    if (nbucket != need) thr = radix_refine(src, total, dstar, 1, need, hist, sm.sel);
+    const uint64_t thr = radix_refine(src, total, dstar, 1, need, hist, sm.sel);
     const uint32_t got = emit_ordered(
         src, total, [thr](uint64_t v) { return v >= thr; },
         [out, K](uint32_t slot, uint64_t v) {
@@ -369,6 +373,40 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     const int N = a.qg * HP;  // MMA N (columns per accumulator buffer)
 
     // ---- set-up
+    // ---- span of positions this CTA covers (every thread, from global q_n)
+    int nmax = 0, nscored = 0;
+    for (int i = 0; i < nqg; ++i) {
+        const int n_i = a.q_n[q0 + i];
+        nmax = max(nmax, n_i);
+        if (MODE == kModeScores || n_i > a.topk) nscored = max(nscored, n_i);
+    }
+    const int seq = nqg > 0 ? a.q_seq[q0] : 0;
+    const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
+    const int start = c * a.chunk;
+    const int end = min(start + a.chunk, span);
+    const int len = max(end - start, 0);
+    const int ntiles = (len + kTileRows - 1) / kTileRows;
+
+    // The producer (thread 0) fills the TMA ring as soon as its barriers
+    // exist, so the first tiles are in flight during the rest of the set-up.
+    const int64_t row0 = (a.page_table == nullptr && nqg > 0) ? a.seq_row0[seq] : 0;
+    auto issue_tile = [&](int t, int s) {
+        const int p0 = start + t * kTileRows;
+        uint8_t *dst = stages + s * kTileBytes;
+        if (a.page_table == nullptr) {
+            mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+            tma_load_2d(dst, &kmap, &sm.full[s], 0, static_cast<int32_t>(row0 + p0));
+        } else {
+            const int box = a.page_size;
+            const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages + p0 / box;
+            int n_box = 0;
+            for (int h = 0; h < kTileRows / box; ++h) n_box += (p0 + h * box < nmax);
+            mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
+            for (int h = 0; h < n_box; ++h, dst += box * DI) tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[h] * box);
+        }
+    };
+    const int n_pro = min(ntiles, a.stages);  // tiles issued before the set-up barrier
+
     if (tid == 0) {
         sm.abort = 0;
         sm.is_last = 0;
@@ -384,9 +422,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b % 2
         }
         fence_mbar_init();
+        for (int t = 0; t < n_pro; ++t) issue_tile(t, t);
     }
     if (tid < kMaxGroupQueries) sm.n_q[tid] = tid < nqg ? a.q_n[q0 + tid] : 0;
-    const int seq = nqg > 0 ? a.q_seq[q0] : 0;
     // q^I tile (B operand, K-major, swizzled like the TMA tiles) and weights
     for (int i = tid; i < N * (DI / 16); i += blockDim.x) {
         const int r = i / (DI / 16), ch = i % (DI / 16);
@@ -416,18 +454,6 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     // a query group must read one sequence
     if (tid < nqg && a.q_seq[q0 + tid] != seq) record_status(a.status, DSA_ERR_DEVICE_CHECK);
 
-    // ---- span of positions this CTA covers
-    int nmax = 0, nscored = 0;
-    for (int i = 0; i < nqg; ++i) {
-        nmax = max(nmax, sm.n_q[i]);
-        if (MODE == kModeScores || sm.n_q[i] > a.topk) nscored = max(nscored, sm.n_q[i]);
-    }
-    const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
-    const int start = c * a.chunk;
-    const int end = min(start + a.chunk, span);
-    const int len = max(end - start, 0);
-    const int ntiles = (len + kTileRows - 1) / kTileRows;
-
     if (MODE == kModeFused && c == 0)
         for (int i = 0; i < nqg; ++i)
             if (sm.n_q[i] <= a.topk) write_fallback(a, q0 + i, sm.n_q[i]);
@@ -438,41 +464,16 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             if (lane == 0) {
                 // ring position (s, ph) advances by one per tile: no divisions
                 // in this single-thread loop, which paces the whole stream
-                int s = 0;
-                uint32_t ph = 0;
-                if (a.page_table == nullptr) {
-                    int32_t row = static_cast<int32_t>(a.seq_row0[seq] + start);
-                    for (int t = 0; t < ntiles; ++t, row += kTileRows) {
-                        if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
-                            record_status(a.status, DSA_ERR_TIMEOUT);
-                            sm.abort = 1;
-                            break;
-                        }
-                        mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-                        tma_load_2d(stages + s * kTileBytes, &kmap, &sm.full[s], 0, row);
-                        if (++s == a.stages) { s = 0; ph ^= 1; }
+                int s = n_pro == a.stages ? 0 : n_pro;
+                uint32_t ph = n_pro == a.stages ? 1u : 0u;
+                for (int t = n_pro; t < ntiles; ++t) {
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                        break;
                     }
-                } else {
-                    const int box = a.page_size;
-                    const int per_tile = kTileRows / box;
-                    const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages;
-                    int page = start / box;
-                    for (int t = 0; t < ntiles; ++t) {
-                        if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
-                            record_status(a.status, DSA_ERR_TIMEOUT);
-                            sm.abort = 1;
-                            break;
-                        }
-                        const int p0 = start + t * kTileRows;
-                        int n_box = 0;
-                        for (int h = 0; h < per_tile; ++h) n_box += (p0 + h * box < nmax);
-                        mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
-                        uint8_t *dst = stages + s * kTileBytes;
-                        for (int h = 0; h < n_box; ++h, dst += box * DI)
-                            tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[page + h] * box);
-                        page += per_tile;
-                        if (++s == a.stages) { s = 0; ph ^= 1; }
-                    }
+                    issue_tile(t, s);
+                    if (++s == a.stages) { s = 0; ph ^= 1; }
                 }
             }
         } else if (warp == 1) {

@@ -149,22 +149,36 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
 // Ordered block-wide compaction: the elements i in [0, n) with pred(v) true
 // are handed to out(slot, v) with consecutive slots base, base + 1, ... in
 // increasing i.  Warp w owns a contiguous slice (a multiple of 128
-// elements); each lane takes four consecutive elements per step (one
-// src.load4).  Pass 1 counts, one block-wide scan of the warp counts gives
-// every warp its first slot, pass 2 emits in order with a warp scan of the
-// lanes' counts.  Returns the next free slot.  `wsum`: 32 shared words.
+// elements); each lane takes four consecutive elements per 128-element step
+// (one src.load4), and a warp works on kEmitUnroll steps at once so that
+// their loads and predicate chains overlap.  Pass 1 counts, one block-wide
+// scan of the warp counts gives every warp its first slot, pass 2 emits in
+// order: four ballots per step (one per element of the lanes' quads) give
+// each lane the number of matches in lower lanes without a shuffle chain.
+// Returns the next free slot.  `wsum`: 32 shared words.
+constexpr int kEmitUnroll = 4;
+
 template <class Src, class Pred, class Out>
 __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
                                  uint32_t base, uint32_t *wsum) {
+    constexpr int U = kEmitUnroll;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int per = ((n + nw - 1) / nw + 127) & ~127;
     const int lo = min(warp * per, n), hi = min(lo + per, n);
     uint32_t cnt = 0;
-    for (int i0 = lo + 4 * lane; i0 < hi; i0 += 128) {
-        uint64_t v[4];
-        src.load4(i0, v);
+    for (int b0 = lo; b0 < hi; b0 += 128 * U) {
+        uint64_t v[U][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) cnt += (i0 + e < hi && pred(v[e])) ? 1u : 0u;
+        for (int u = 0; u < U; ++u) {
+            const int i0 = b0 + 128 * u + 4 * lane;
+            if (i0 < hi) src.load4(i0, v[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i0 = b0 + 128 * u + 4 * lane;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) cnt += (i0 + e < hi && pred(v[u][e])) ? 1u : 0u;
+        }
     }
     cnt = warp_sum(cnt);
     if (lane == 0) wsum[warp] = cnt;
@@ -176,23 +190,33 @@ __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const 
         total += c;
     }
     uint32_t slot = base + before;
-    for (int b0 = lo; b0 < hi; b0 += 128) {
-        const int i0 = b0 + 4 * lane;
-        uint64_t v[4] = {0, 0, 0, 0};
-        uint32_t mask = 0;
-        if (i0 < hi) {
-            src.load4(i0, v);
+    const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
+    for (int b0 = lo; b0 < hi; b0 += 128 * U) {
+        uint64_t v[U][4];
+        uint32_t mask[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i0 = b0 + 128 * u + 4 * lane;
+            mask[u] = 0;
+            if (i0 < hi) {
+                src.load4(i0, v[u]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (i0 + e < hi && pred(v[u][e])) mask[u] |= 1u << e;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const uint32_t q0 = __ballot_sync(0xffffffffu, mask[u] & 1u);
+            const uint32_t q1 = __ballot_sync(0xffffffffu, mask[u] & 2u);
+            const uint32_t q2 = __ballot_sync(0xffffffffu, mask[u] & 4u);
+            const uint32_t q3 = __ballot_sync(0xffffffffu, mask[u] & 8u);
+            uint32_t s0 = slot + __popc(q0 & lt) + __popc(q1 & lt) + __popc(q2 & lt) + __popc(q3 & lt);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-                if (i0 + e < hi && pred(v[e])) mask |= 1u << e;
+                if ((mask[u] >> e) & 1u) out(s0++, v[u][e]);
+            slot += __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
         }
-        const uint32_t c = static_cast<uint32_t>(__popc(mask));
-        const uint32_t incl = warp_incl_scan(c);
-        uint32_t s0 = slot + incl - c;
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-            if ((mask >> e) & 1u) out(s0++, v[e]);
-        slot += __shfl_sync(0xffffffffu, incl, 31);
     }
     __syncthreads();
     return base + total;
