@@ -285,10 +285,11 @@ def run_ours(args, world, rank):
     d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
 
     def e2e_step():
+        # the current stream (the capture stream while a graph is recorded)
         for d, h in ((d_qidx, h_qidx), (d_w, h_w), (d_q, h_q), (d_qn, h_qn), (d_qseq, h_qseq)):
             d.copy_(h, non_blocking=True)
         dsa.forward(p, kv_e, d_qidx, d_w, db.kidx, db.k_scale, d_q, db.kv, db.kv_row_stride,
-                    out, lse, idx, ws, stream=st, paged=paged)
+                    out, lse, idx, ws, paged=paged)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
         h_idx.copy_(idx, non_blocking=True)
@@ -297,7 +298,31 @@ def run_ours(args, world, rank):
         e2e_step()
     torch.cuda.synchronize()
     barrier(world)
-    t_e2e = max_over_ranks(timed(e2e_step, args.steps), world)
+    t_e2e_eager = max_over_ranks(timed(e2e_step, args.steps), world)
+    # The same step recorded once as a CUDA graph (copies from the pinned
+    # buffers, the dsa_forward launches, copies back) and replayed: one host
+    # launch per step, as a decode loop would run it.
+    e2e_launch = "cuda_graph"
+    try:
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(st)
+        with torch.cuda.stream(side):
+            e2e_step()
+        st.wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph):
+            e2e_step()
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        t_e2e = max_over_ranks(timed(graph.replay, args.steps), world)
+        del graph
+    except RuntimeError as exc:  # capture refused: report the eager loop
+        print("e2e graph capture failed (%s); reporting the eager loop" % exc, file=sys.stderr)
+        e2e_launch, t_e2e = "eager", t_e2e_eager
+    assert dsa.check_status(ws) == dsa.DSA_OK, dsa.last_error()
 
     alg = algorithmic_bytes(inp)
     hbm, bf16, peak_kind = peaks()
@@ -346,7 +371,8 @@ def run_ours(args, world, rank):
             "algorithmic_bytes_per_step": alg["indexer"] + alg["attention"],
         },
         "e2e": {"value": total_q / t_e2e, "unit": "queries/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h, "launch": e2e_launch,
+                "eager_value": total_q / t_e2e_eager},
         "gpu_launches": 3 * args.steps,
         "device_status": status,
         "input_gen_s": gen_s,

@@ -161,6 +161,15 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     P = (sp + chunk - 1) / chunk;
     pl.P = static_cast<int>(P);
     pl.chunk = static_cast<int>(chunk);
+    if (mode != dsa::kModeScores) {
+        // the ordered emissions record their ballots in the 2048-word radix
+        // scratch (chunk lists) and in the whole histogram area (the merge)
+        const int nw = (mode == dsa::kModeTopk ? dsa::kK2Threads : dsa::kK1Threads) / 32;
+        const int merge_n = pl.P * (p->topk + 2);
+        if (dsa::emit_ballot_words(pl.chunk, nw) > dsa::kSelBinsHost ||
+            dsa::emit_ballot_words(merge_n, nw) > (pl.qg + 1) * dsa::kSelBinsHost)
+            return fail(DSA_ERR_UNSUPPORTED, "selection scratch too small for this plan");
+    }
     pl.acc_bufs = (dsa::kK1MaxAcc * pl.qg * pl.hp <= 512) ? dsa::kK1MaxAcc : 2;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(pl.acc_bufs * pl.qg * pl.hp)) cols <<= 1;
@@ -201,11 +210,11 @@ MlaPlan plan_mla(const dsa_params *p) {
     rps = (rps + 15) / 16 * 16;
     if (rps > dsa::kMlaMaxRows) rps = dsa::kMlaMaxRows;
     m.rows_per_split = rps;
-    m.splits = (k + rps - 1) / rps;
+    m.splits = (k + rps - 1) / rps;  // <= ceil(2048 / 64) = kMlaMaxSplits: rps >= 64 unless s_min binds
     if (m.splits == 1) {
         m.wave = p->nq;
     } else {
-        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv + 1) * 4;
+        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv * 2 + 4);
         size_t w = kPartialBudget / per_q;
         if (w < 1) w = 1;
         m.wave = p->nq < static_cast<int>(w) ? p->nq : static_cast<int>(w);
@@ -241,7 +250,7 @@ size_t mla_ws(const dsa_params *p, const MlaPlan &m, size_t off, WsLayout &w) {
     w.part_o = w.part_lse = off;
     if (m.splits <= 1) return off;
     w.part_o = off;
-    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * dsa::kDv * 4, 256);
+    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * dsa::kDv * 2, 256);  // fp16
     w.part_lse = off;
     off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 4, 256);
     return off;
@@ -288,6 +297,7 @@ int layout_for(const dsa_params *p, int op, WsLayout &w, IndexerPlan *ipl, MlaPl
     default:
         return fail(DSA_ERR_INVALID_ARG, "unknown op %d", op);
     }
+    if (m.splits > dsa::kMlaMaxSplits) return fail(DSA_ERR_UNSUPPORTED, "too many attention splits (%d)", m.splits);
     w.total = off;
     if (ipl) *ipl = pl;
     if (mpl) *mpl = m;
@@ -407,7 +417,7 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.scale_log2 = p->scale * 1.4426950408889634f;
     a.out = static_cast<uint16_t *>(out);
     a.lse = lse;
-    a.part_o = m.splits > 1 ? at<float>(ws, wl.part_o) : nullptr;
+    a.part_o = m.splits > 1 ? at<uint16_t>(ws, wl.part_o) : nullptr;
     a.part_lse = m.splits > 1 ? at<float>(ws, wl.part_lse) : nullptr;
     a.status = at<int>(ws, wl.status);
     for (int q0 = 0; q0 < p->nq; q0 += m.wave) {

@@ -161,7 +161,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
             [out, K](uint32_t slot, uint64_t v) {
                 if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
             },
-            0u, sm.sel.wsum);
+            0u, sm.sel.wsum, reinterpret_cast<uint4 *>(scratch));
         if (threadIdx.x == 0) {
             if (cnt != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
             if (a.nsel) a.nsel[q] = K;
@@ -228,7 +228,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
         [cand, K](uint32_t slot, uint64_t v) {
             if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
         },
-        0u, sm.sel.wsum);
+        0u, sm.sel.wsum, reinterpret_cast<uint4 *>(scratch));
     if (threadIdx.x == 0) {
         if (m > static_cast<uint32_t>(K)) {
             record_status(a.status, DSA_ERR_DEVICE_CHECK);
@@ -316,7 +316,7 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
         [out, K](uint32_t slot, uint64_t v) {
             if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
         },
-        0u, sm.sel.wsum);
+        0u, sm.sel.wsum, reinterpret_cast<uint4 *>(hist));
     if (threadIdx.x == 0) {
         if (got != static_cast<uint32_t>(K)) record_status(a.status, DSA_ERR_DEVICE_CHECK);
         if (a.nsel) a.nsel[q] = K;
@@ -581,6 +581,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the attention kernel may start launching on SMs this grid frees up
+    // (it waits for this grid's completion before reading the indices)
+    if (tid == 0) grid_launch_dependents();
 
     // ---- selection (fused mode)
     if (MODE == kModeFused && !sm.abort) {

@@ -23,6 +23,13 @@ constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
 constexpr int kSelBinsHost = 2048;
 constexpr long long kHistWaitCycles = 100000;  // ~50 us: bounded wait for a query's full histogram
 
+// Shared words an ordered emission over n elements by `nwarps` warps needs
+// for its recorded ballots (one uint4 per 128-element step of each warp's
+// slice; see emit_ordered).
+__host__ __device__ constexpr int emit_ballot_words(int n, int nwarps) {
+    return 4 * nwarps * ((((n + nwarps - 1) / nwarps + 127) & ~127) / 128);
+}
+
 struct K1Params {
     // inputs
     const uint8_t *q_idx;   // [nq, h_idx, d_idx] e4m3
@@ -116,7 +123,8 @@ constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
 constexpr int kMlaStages = 4;       // pass-1 ring depth (Q chunk + K chunk)
 constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
 constexpr int kMlaVStages = 3;      // pass-2 ring depth
-constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers
+constexpr int kMlaMaxSplits = 32;   // splits per query (the combine kernel's warp reads one LSE per lane)
+constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers (0-3 help in pass 1)
 
 struct MlaParams {
     const int32_t *q_seq;
@@ -137,7 +145,7 @@ struct MlaParams {
     // outputs
     uint16_t *out;       // [nq, h, d_v] bf16
     float *lse;          // [nq, h]
-    float *part_o;       // [wave_q, splits, 128, d_v] normalised partial outputs
+    uint16_t *part_o;    // [wave_q, splits, 128, d_v] normalised partial outputs (fp16 bits)
     float *part_lse;     // [wave_q, splits, 128]
     int *status;
 };

@@ -242,6 +242,16 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t a_fmt, uint32_t b_fmt
 }
 
 // ------------------------------------------------------------------- misc
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel in the stream is still
+// running; grid_dependency_wait() blocks until that kernel has completed and
+// its memory is visible, so nothing the previous kernel (or anything before
+// it) produced may be read before it.  grid_launch_dependents() lets the
+// next kernel start launching once every CTA of this grid has called it or
+// exited.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Two independent round-to-nearest FMAs on a pair of floats (d.x = a.x * b.x +
 // c.x, d.y likewise): the same results as two fmaf calls, in one instruction.
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {

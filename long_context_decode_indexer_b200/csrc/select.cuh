@@ -10,6 +10,7 @@
 // {V >= threshold}.
 #pragma once
 
+#include "kernels.h"
 #include "ptx.cuh"
 
 namespace dsa {
@@ -149,38 +150,46 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
 // Ordered block-wide compaction: the elements i in [0, n) with pred(v) true
 // are handed to out(slot, v) with consecutive slots base, base + 1, ... in
 // increasing i.  Warp w owns a contiguous slice (a multiple of 128
-// elements); each lane takes four consecutive elements per 128-element step
-// (one src.load4), and a warp works on kEmitUnroll steps at once so that
-// their loads and predicate chains overlap.  Pass 1 counts, one block-wide
-// scan of the warp counts gives every warp its first slot, pass 2 emits in
-// order: four ballots per step (one per element of the lanes' quads) give
-// each lane the number of matches in lower lanes without a shuffle chain.
-// Returns the next free slot.  `wsum`: 32 shared words.
-constexpr int kEmitUnroll = 4;
-
+// elements) in steps of 128: each lane tests four consecutive elements per
+// step (one src.load4), and four ballots (one per element of the lanes'
+// quads) record the step's matches.  The ballot loop has no divergent branch
+// (a diverged warp must reconverge before every ballot, which costs more
+// than the test itself): loads are clamped into the slice and lane t keeps
+// the ballots of step t in a register, written to `bal` after each batch of
+// 32 steps.  After one block-wide scan of the warps' match counts, the
+// second pass walks the recorded ballots: a step without a match costs a
+// shuffle, and only lanes with a match reload their quad; a lane's slot is
+// the number of matches in lower lanes (popc of the ballots below it).
+// Returns the next free slot.  `wsum`: 32 shared words; `bal`: shared, at
+// least emit_ballot_words(n, warps) / 4 uint4.
 template <class Src, class Pred, class Out>
 __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
-                                 uint32_t base, uint32_t *wsum) {
-    constexpr int U = kEmitUnroll;
+                                 uint32_t base, uint32_t *wsum, uint4 *bal) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int per = ((n + nw - 1) / nw + 127) & ~127;
     const int lo = min(warp * per, n), hi = min(lo + per, n);
-    uint32_t cnt = 0;
-    for (int b0 = lo; b0 < hi; b0 += 128 * U) {
-        uint64_t v[U][4];
+    const int steps = (hi - lo + 127) / 128;
+    uint4 *wb = bal + warp * (per / 128);
+    uint32_t cnt = 0;  // warp-uniform
+    for (int b0 = 0; b0 < steps; b0 += 32) {
+        const int nb = min(32, steps - b0);
+        uint4 mine = make_uint4(0, 0, 0, 0);
+        for (int t = 0; t < nb; ++t) {
+            const int i0 = lo + 128 * (b0 + t) + 4 * lane;
+            uint64_t v[4];
+            src.load4(i0 < hi ? i0 : lo, v);  // clamped: no branch around the load
+            uint32_t m = 0;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i0 = b0 + 128 * u + 4 * lane;
-            if (i0 < hi) src.load4(i0, v[u]);
+            for (int e = 0; e < 4; ++e) m |= ((i0 + e < hi) & pred(v[e])) ? (1u << e) : 0u;
+            const uint32_t q0 = __ballot_sync(0xffffffffu, m & 1u);
+            const uint32_t q1 = __ballot_sync(0xffffffffu, m & 2u);
+            const uint32_t q2 = __ballot_sync(0xffffffffu, m & 4u);
+            const uint32_t q3 = __ballot_sync(0xffffffffu, m & 8u);
+            mine = lane == t ? make_uint4(q0, q1, q2, q3) : mine;
+            cnt += __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
         }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i0 = b0 + 128 * u + 4 * lane;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) cnt += (i0 + e < hi && pred(v[u][e])) ? 1u : 0u;
-        }
+        if (lane < nb) wb[b0 + lane] = mine;
     }
-    cnt = warp_sum(cnt);
     if (lane == 0) wsum[warp] = cnt;
     __syncthreads();
     uint32_t before = 0, total = 0;
@@ -191,31 +200,29 @@ __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const 
     }
     uint32_t slot = base + before;
     const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
-    for (int b0 = lo; b0 < hi; b0 += 128 * U) {
-        uint64_t v[U][4];
-        uint32_t mask[U];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int i0 = b0 + 128 * u + 4 * lane;
-            mask[u] = 0;
-            if (i0 < hi) {
-                src.load4(i0, v[u]);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (i0 + e < hi && pred(v[u][e])) mask[u] |= 1u << e;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const uint32_t q0 = __ballot_sync(0xffffffffu, mask[u] & 1u);
-            const uint32_t q1 = __ballot_sync(0xffffffffu, mask[u] & 2u);
-            const uint32_t q2 = __ballot_sync(0xffffffffu, mask[u] & 4u);
-            const uint32_t q3 = __ballot_sync(0xffffffffu, mask[u] & 8u);
-            uint32_t s0 = slot + __popc(q0 & lt) + __popc(q1 & lt) + __popc(q2 & lt) + __popc(q3 & lt);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                if ((mask[u] >> e) & 1u) out(s0++, v[u][e]);
-            slot += __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
+    for (int b0 = 0; b0 < steps; b0 += 32) {
+        const int nb = min(32, steps - b0);
+        const uint4 mine = lane < nb ? wb[b0 + lane] : make_uint4(0, 0, 0, 0);
+        for (int t = 0; t < nb; ++t) {
+            const uint32_t q0 = __shfl_sync(0xffffffffu, mine.x, t);
+            const uint32_t q1 = __shfl_sync(0xffffffffu, mine.y, t);
+            const uint32_t q2 = __shfl_sync(0xffffffffu, mine.z, t);
+            const uint32_t q3 = __shfl_sync(0xffffffffu, mine.w, t);
+            const uint32_t tot = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
+            if (tot == 0u) continue;  // warp-uniform
+            // every lane reloads its quad and computes the four slots; the
+            // stores are predicated, not branched around
+            uint64_t v[4];
+            src.load4(lo + 128 * (b0 + t) + 4 * lane, v);
+            const uint32_t o0 = (q0 >> lane) & 1u, o1 = (q1 >> lane) & 1u;
+            const uint32_t o2 = (q2 >> lane) & 1u, o3 = (q3 >> lane) & 1u;
+            const uint32_t s0 = slot + __popc(q0 & lt) + __popc(q1 & lt) + __popc(q2 & lt) + __popc(q3 & lt);
+            const uint32_t s1 = s0 + o0, s2 = s1 + o1, s3 = s2 + o2;
+            if (o0) out(s0, v[0]);
+            if (o1) out(s1, v[1]);
+            if (o2) out(s2, v[2]);
+            if (o3) out(s3, v[3]);
+            slot += tot;
         }
     }
     __syncthreads();

@@ -9,9 +9,12 @@
 // ("split"); all 128 heads form the MMA's M dimension.
 //   pass 1  S[128 x R] = Q . K^T over 9 chunks of 64 key columns.  Each ring
 //           stage holds a Q chunk (TMA tile, 16 KB) and the R rows' matching
-//           128-byte pieces, gathered by four warps with 16-byte cp.async
-//           into the 128B-swizzled layout (the rows were first prefetched
-//           whole into L2).  S accumulates in TMEM.
+//           128-byte pieces, gathered by eight warps (the softmax warps help:
+//           they have nothing else to do yet) with 16-byte cp.async into the
+//           128B-swizzled layout (the rows were first prefetched whole into
+//           L2).  A gather thread owns one 16-byte piece of a fixed set of
+//           rows, so its addresses are computed once for all nine chunks.
+//           S accumulates in TMEM.
 //   softmax one thread per head reads its S row from TMEM, takes the exact
 //           max over the split, writes P = exp(S - max) into shared memory
 //           as a pair of bf16 tiles P_hi = bf16(P), P_lo = bf16(P - P_hi)
@@ -22,10 +25,15 @@
 //           warps (32-row tiles, L2 hits) into an MN-major swizzled layout; O
 //           takes all 512 TMEM columns, which is why S and O are not live at
 //           the same time.
-// A split writes O / l and its log-sum-exp; the combine kernel merges splits
-// by their log-sum-exp.  With one split the CTA writes the final output.
+// Epilogue: the softmax warps write columns 0..255 of O / l, the gather warps
+// columns 256..511, each thread straight from TMEM to its head's row.  A split writes O / l in fp16 (its values are convex
+// combinations of bf16 rows, so fp16's range suffices and its rounding,
+// 2^-12 relative, is far below the bf16 output's) and its log-sum-exp; the
+// combine kernel merges splits by their log-sum-exp.  With one split the CTA
+// writes the final output.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -43,11 +51,12 @@ constexpr int kNumKChunks = kDqk / 64;              // 9
 constexpr int kVTileBytes = kMlaVRows * kDv * 2;    // 32 KB
 constexpr int kVBlockBytes = kMlaVRows * 128;       // one 64-column block of a V tile
 constexpr int kPBlockBytes = 128 * 128;             // 128 heads x 64 rows bf16
-constexpr int kGatherWarp0 = 6;                     // warps 6..9 gather rows
+constexpr int kGatherWarp0 = 6;                     // warps 6..9 gather rows (and 0..3 in pass 1)
 constexpr int kGatherThreads = 128;
+constexpr int kPass1Threads = 256;                  // pass-1 gather threads (warps 0-3, 6-9)
+constexpr int kPass1Rows = kMlaMaxRows / (kPass1Threads / 8);  // rows per pass-1 gather thread
 constexpr int kGatherLag = 3;                       // pass-1 chunks in flight per gather thread
 constexpr int kVLag = 2;                            // pass-2 tiles in flight per gather thread
-constexpr int kStageRowFloats = 68;                 // epilogue staging row (64 + 4 pad)
 
 struct MlaSmem {
     uint64_t full[kMlaStages];
@@ -63,6 +72,7 @@ struct MlaSmem {
     int32_t rows[kMlaMaxRows];
     uint8_t valid[kMlaMaxRows];
     uint32_t vmask[kMlaMaxRows / 32];  // bit j of word w: entry 32w + j is valid
+    float inv_l[128];                  // 1 / row sum per head (softmax -> second epilogue group)
 };
 
 static_assert(sizeof(MlaSmem) <= 2048, "MlaSmem must fit the reserve in mla_layout()");
@@ -71,10 +81,100 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+// Named barrier `id` over `count` threads that also ANDs `pred` across them.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const uint32_t a = __half_as_ushort(__float2half_rn(lo));
+    const uint32_t b = __half_as_ushort(__float2half_rn(hi));
+    return a | (b << 16);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
     const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
     return a | (b << 16);
+}
+
+// Pass-1 row gathers by one of the kPass1Threads gather threads (gt): it
+// owns the 16-byte piece j = gt % 8 of rows gt / 8 + 32 k, and copies that
+// piece of chunk c (key columns 64c .. 64c+63) of each of its rows into the
+// stage's K area, 128B-swizzled.  Chunk c - kGatherLag is published (the
+// warp arrives on its full barrier) once this thread's copies of it landed.
+// Returns false if a wait timed out.
+__device__ bool gather_pass1(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int gt, int Rp) {
+    const int j = gt & 7, r0 = gt >> 3, lane = threadIdx.x & 31;
+    const uint16_t *src[kPass1Rows];
+    uint32_t dst[kPass1Rows];
+#pragma unroll
+    for (int k = 0; k < kPass1Rows; ++k) {
+        const int r = r0 + 32 * k;
+        src[k] = a.kv + static_cast<int64_t>(sm.rows[r]) * a.kv_row_stride + j * 8;
+        dst[k] = static_cast<uint32_t>(r * 128 + ((j ^ (r & 7)) << 4));
+    }
+    bool ok = true;
+    for (int c = 0; c < kNumKChunks + kGatherLag; ++c) {
+        if (c < kNumKChunks) {
+            const int s = c % kMlaStages;
+            const uint32_t ph = (c / kMlaStages) & 1;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1) && !sm.abort);
+            if (ok) {
+                uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
+#pragma unroll
+                for (int k = 0; k < kPass1Rows; ++k)
+                    if (r0 + 32 * k < Rp) cp_async16(kst + dst[k], src[k] + c * 64);
+            }
+            cp_async_commit();
+        }
+        if (c >= kGatherLag) {
+            // chunk c - lag is complete for this thread: publish it
+            if (c < kNumKChunks) cp_async_wait<kGatherLag>();
+            else cp_async_wait<0>();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.full[(c - kGatherLag) % kMlaStages]);
+        }
+    }
+    return ok;
+}
+
+// O / l of this thread's head row, columns [c_begin, c_begin + 256): TMEM ->
+// registers -> 16-byte stores of the row (bf16 output, or fp16 partials).
+// A thread writes whole 32-byte sectors of its own row, so the stores need
+// no staging and no barrier.  The TMEM loads are warp-collective: every lane
+// runs them, and only the stores are skipped for padding heads (hrow >= h).
+__device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, int q, int wq, int sp,
+                             float inv_l, int c_begin) {
+    const bool live = hrow < a.h;
+    uint16_t *dst = a.splits == 1
+                        ? a.out + (static_cast<int64_t>(q) * a.h + (live ? hrow : 0)) * kDv
+                        : a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+    for (int c1 = c_begin; c1 < c_begin + 256; c1 += 64) {
+        uint32_t v2[2][32];
+        tmem_ld32(lane_addr + c1, v2[0]);
+        tmem_ld32(lane_addr + c1 + 32, v2[1]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const uint32_t *u = &v2[g >> 2][(g & 3) * 8];
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = __uint_as_float(u[2 * e]) * inv_l, x1 = __uint_as_float(u[2 * e + 1]) * inv_l;
+                w[e] = a.splits == 1 ? pack_bf16x2(x0, x1) : pack_half2(x0, x1);
+            }
+            if (live) *reinterpret_cast<uint4 *>(dst + c1 + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
 }
 
 }  // namespace
@@ -104,7 +204,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         sm.abort = 0;
         sm.nvalid = 0;
         for (int s = 0; s < kMlaStages; ++s) {
-            mbar_init(&sm.full[s], 1 + 4);  // Q TMA (with its bytes) + four gather warps
+            mbar_init(&sm.full[s], 1 + kPass1Threads / 32);  // Q TMA (with its bytes) + eight gather warps
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.s_full, 1);
@@ -116,6 +216,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         mbar_init(&sm.o_full, 1);
         fence_mbar_init();
     }
+    // rows h..127 of every Q chunk are never written by TMA: zero them once
+    if (hbox < 128) {
+        for (int s = 0; s < kMlaStages; ++s)
+            for (int i = tid; i < (128 - hbox) * 8; i += blockDim.x)
+                *reinterpret_cast<uint4 *>(ring + s * kStageBytes + hbox * 128 + i * 16) = make_uint4(0, 0, 0, 0);
+    }
+    if (warp == 5) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    // everything above touches no input: with programmatic dependent launch
+    // it overlaps the end of the kernel that produced the indices
+    grid_dependency_wait();
     // cache rows of this split's entries (invalid entries read row 0 and are
     // masked; P = 0 there)
     const int n = a.q_n[q];
@@ -146,16 +259,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         const unsigned bits = __ballot_sync(0xffffffffu, ok != 0);
         if ((i & 31) == 0) sm.vmask[i >> 5] = bits;
     }
-    // rows h..127 of every Q chunk are never written by TMA: zero them once
-    if (hbox < 128) {
-        for (int s = 0; s < kMlaStages; ++s)
-            for (int i = tid; i < (128 - hbox) * 8; i += blockDim.x)
-                *reinterpret_cast<uint4 *>(ring + s * kStageBytes + hbox * 128 + i * 16) = make_uint4(0, 0, 0, 0);
-    }
-    if (warp == 5) {
-        tmem_alloc(&sm.tmem_base, 512);
-        tmem_relinquish();
-    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -185,34 +288,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             for (int i = gt; i < R; i += kGatherThreads)
                 if (sm.valid[i])
                     prefetch_l2_bulk(a.kv + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
-            bool ok = true;
-            // pass 1: chunk c of every row -> K area of ring stage c % kMlaStages
-            for (int c = 0; c < kNumKChunks + kGatherLag; ++c) {
-                if (c < kNumKChunks) {
-                    const int s = c % kMlaStages;
-                    const uint32_t ph = (c / kMlaStages) & 1;
-                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1) && !sm.abort);
-                    if (ok) {
-                        uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
-                        for (int i = gt; i < Rp * 8; i += kGatherThreads) {
-                            const int r = i >> 3, j = i & 7;
-                            const uint16_t *src = a.kv + static_cast<int64_t>(sm.rows[r]) * a.kv_row_stride + c * 64 + j * 8;
-                            cp_async16(kst + r * 128 + ((j ^ (r & 7)) << 4), src);
-                        }
-                    }
-                    cp_async_commit();
-                }
-                if (c >= kGatherLag) {
-                    // chunk c - lag is complete for this thread: publish it
-                    if (c < kNumKChunks) cp_async_wait<kGatherLag>();
-                    else cp_async_wait<0>();
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.full[(c - kGatherLag) % kMlaStages]);
-                }
-            }
-            // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is done
+            bool ok = gather_pass1(a, sm, ring, kPass1Threads / 2 + gt, Rp);
+            // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is
+            // done.  Thread gt owns row r = gt / 4 of every tile and its
+            // pieces u, u + 4, ..., u + 60 (u = gt % 4): one row lookup per tile.
             ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
+            const int vr = gt >> 2, vu = gt & 3;
             const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
             for (int vt = 0; vt < nvt + kVLag; ++vt) {
                 if (vt < nvt) {
@@ -220,13 +301,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     const uint32_t ph = (vt / kMlaVStages) & 1;
                     ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1) && !sm.abort);
                     if (ok) {
-                        uint8_t *vt_base = vring + v * kVTileBytes;
-                        // 32 rows x 8 column blocks x 8 pieces of 16 bytes
-                        for (int i = gt; i < kMlaVRows * 64; i += kGatherThreads) {
-                            const int r = i >> 6, blk = (i >> 3) & 7, j = i & 7;
-                            const int e = vt * kMlaVRows + r;
-                            const uint16_t *src = a.kv + static_cast<int64_t>(sm.rows[e]) * a.kv_row_stride + blk * 64 + j * 8;
-                            cp_async16(vt_base + blk * kVBlockBytes + r * 128 + ((j ^ (r & 7)) << 4), src);
+                        uint8_t *vdst = vring + v * kVTileBytes + vr * 128;
+                        const uint16_t *vsrc = a.kv + static_cast<int64_t>(sm.rows[vt * kMlaVRows + vr]) * a.kv_row_stride;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const int pc = vu + 4 * m;  // 16-byte piece of the 512 value columns
+                            const int blk = pc >> 3, j = pc & 7;
+                            cp_async16(vdst + blk * kVBlockBytes + ((j ^ (vr & 7)) << 4), vsrc + pc * 8);
                         }
                     }
                     cp_async_commit();
@@ -242,6 +323,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             if (!ok && lane == 0) {
                 record_status(a.status, DSA_ERR_TIMEOUT);
                 sm.abort = 1;
+            }
+            // second epilogue group: value columns 256..511
+            const int hrow = (warp & 3) * 32 + lane;
+            const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0) && !sm.abort);
+            // inv_l of every head is in shared memory; both groups agree on ok
+            // (the epilogue's named barriers need all 128 threads of a group)
+            ok = bar_and(3, 256, ok);
+            if (ok) {
+                tc_fence_after();
+                store_output(a, lane_addr, hrow, q, wq, sp, sm.inv_l[hrow], 256);
             }
         } else if (warp == 5) {
             // ------------------------------------------------ MMA issuer
@@ -309,10 +401,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 }
             }
         } else if (warp < 4) {
-            // ------------------------------------- softmax, then epilogue
+            // ------------------- pass-1 gathers, softmax, then epilogue
+            bool ok = gather_pass1(a, sm, ring, tid, Rp);
             const int hrow = warp * 32 + lane;  // head = TMEM lane
             const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.s_full, 0) && !sm.abort);
             float m = -INFINITY, l = 0.f;
             if (ok) {
                 tc_fence_after();
@@ -366,46 +459,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full);
+            const bool has = l > 0.f;
+            const float inv_l = has ? 1.f / l : 0.f;
+            sm.inv_l[hrow] = inv_l;
             ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0) && !sm.abort);
+            ok = bar_and(3, 256, ok);  // hand inv_l to the second group; agree on ok
             if (ok) {
                 tc_fence_after();
-                const bool has = l > 0.f;
-                const float inv_l = has ? 1.f / l : 0.f;
                 const float lse_v = has ? (m * a.scale + logf(l)) : -INFINITY;
                 if (hrow < a.h) {
                     if (a.splits == 1) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
                     else a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
                 }
-                // O / l, 64 columns at a time: TMEM -> padded staging rows ->
-                // coalesced row stores (a warp writes one output row per step)
-                float *stage = reinterpret_cast<float *>(ptile);  // pass-2 area is free now
-                const int64_t prow0 = (static_cast<int64_t>(wq) * a.splits + sp) * 128;
-                for (int c1 = 0, blk = 0; c1 < kDv; c1 += 64, ++blk) {
-                    float *buf = stage + (blk & 1) * (128 * kStageRowFloats);
-                    uint32_t v2[2][32];
-                    tmem_ld32(lane_addr + c1, v2[0]);
-                    tmem_ld32(lane_addr + c1 + 32, v2[1]);
-                    tmem_wait_ld();
-                    float *row = buf + hrow * kStageRowFloats;
-#pragma unroll
-                    for (int g4 = 0; g4 < 16; ++g4) {
-                        const uint32_t *u = &v2[g4 >> 3][(g4 & 7) * 4];
-                        *reinterpret_cast<float4 *>(row + g4 * 4) =
-                            make_float4(__uint_as_float(u[0]) * inv_l, __uint_as_float(u[1]) * inv_l,
-                                        __uint_as_float(u[2]) * inv_l, __uint_as_float(u[3]) * inv_l);
-                    }
-                    asm volatile("bar.sync 1, 128;" ::: "memory");
-                    for (int rr = 0; rr < 32; ++rr) {
-                        const int r = warp * 32 + rr;
-                        if (r >= a.h) break;
-                        const float2 f = *reinterpret_cast<const float2 *>(buf + r * kStageRowFloats + 2 * lane);
-                        if (a.splits == 1)
-                            *reinterpret_cast<uint32_t *>(a.out + (static_cast<int64_t>(q) * a.h + r) * kDv + c1 + 2 * lane) =
-                                pack_bf16x2(f.x, f.y);
-                        else
-                            *reinterpret_cast<float2 *>(a.part_o + (prow0 + r) * kDv + c1 + 2 * lane) = f;
-                    }
-                }
+                store_output(a, lane_addr, hrow, q, wq, sp, inv_l, 0);
             } else if (lane == 0) {
                 record_status(a.status, DSA_ERR_TIMEOUT);
             }
@@ -419,8 +485,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int c0 = 0; c0 < kDv; c0 += 8) *reinterpret_cast<uint4 *>(o + c0) = make_uint4(0, 0, 0, 0);
                 a.lse[static_cast<int64_t>(q) * a.h + hrow] = -INFINITY;
             } else {
-                float *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
-                for (int c0 = 0; c0 < kDv; c0 += 4) *reinterpret_cast<float4 *>(o + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                uint16_t *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+                for (int c0 = 0; c0 < kDv; c0 += 8) *reinterpret_cast<uint4 *>(o + c0) = make_uint4(0, 0, 0, 0);
                 a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = -INFINITY;
             }
         }
@@ -433,35 +499,60 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 }
 
 // Merge the splits of one (query, head): out = sum_s w_s o_s / sum_s w_s with
-// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.
+// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  Warp 0 reads the
+// splits' log-sum-exps (one lane each; splits <= 32) and publishes the
+// weights; then each thread combines 4 columns, its partial loads issued in
+// batches of 8 splits so that they are in flight together.
 __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a) {
+    __shared__ float wts[32];
+    __shared__ float stot, smx;
+    grid_dependency_wait();  // the partials come from the preceding attention kernel
     const int wq = blockIdx.x / a.h, hh = blockIdx.x % a.h;
     const int q = a.q0 + wq;
-    float mx = -INFINITY;
-    for (int s = 0; s < a.splits; ++s)
-        mx = fmaxf(mx, a.part_lse[(static_cast<int64_t>(wq) * a.splits + s) * 128 + hh]);
-    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv;
-    if (mx == -INFINITY) {
-        for (int d = threadIdx.x * 4; d < kDv; d += blockDim.x * 4) {
-            *reinterpret_cast<uint2 *>(o + d) = make_uint2(0, 0);
+    const int64_t row0 = static_cast<int64_t>(wq) * a.splits * 128 + hh;  // split s: row0 + 128 s
+    if (threadIdx.x < 32) {
+        const int s = threadIdx.x;
+        const float ls = s < a.splits ? a.part_lse[row0 + 128 * s] : -INFINITY;
+        float mx = ls;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float w = (mx == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - mx);
+        float t = w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        wts[s] = w;
+        if (s == 0) {
+            stot = t;
+            smx = mx;
         }
+    }
+    __syncthreads();
+    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv;
+    const int d = threadIdx.x * 4;
+    const float tot = stot, mx = smx;
+    if (mx == -INFINITY) {
+        *reinterpret_cast<uint2 *>(o + d) = make_uint2(0, 0);
         if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
         return;
     }
-    float tot = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    const int d = threadIdx.x * 4;
-    for (int s = 0; s < a.splits; ++s) {
-        const int64_t row = (static_cast<int64_t>(wq) * a.splits + s) * 128 + hh;
-        const float ls = a.part_lse[row];
-        if (ls == -INFINITY) continue;
-        const float wgt = __expf(ls - mx);
-        tot += wgt;
-        const float4 v = *reinterpret_cast<const float4 *>(a.part_o + row * kDv + d);
-        acc.x = fmaf(wgt, v.x, acc.x);
-        acc.y = fmaf(wgt, v.y, acc.y);
-        acc.z = fmaf(wgt, v.z, acc.z);
-        acc.w = fmaf(wgt, v.w, acc.w);
+    for (int s0 = 0; s0 < a.splits; s0 += 8) {
+        uint2 raw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            raw[u] = s0 + u < a.splits
+                         ? *reinterpret_cast<const uint2 *>(a.part_o + (row0 + 128 * (s0 + u)) * kDv + d)
+                         : make_uint2(0, 0);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float wgt = s0 + u < a.splits ? wts[s0 + u] : 0.f;
+            const float2 lo2 = __half22float2(*reinterpret_cast<const __half2 *>(&raw[u].x));
+            const float2 hi2 = __half22float2(*reinterpret_cast<const __half2 *>(&raw[u].y));
+            acc.x = fmaf(wgt, lo2.x, acc.x);
+            acc.y = fmaf(wgt, lo2.y, acc.y);
+            acc.z = fmaf(wgt, hi2.x, acc.z);
+            acc.w = fmaf(wgt, hi2.y, acc.w);
+        }
     }
     const float inv = 1.f / tot;
     uint2 u;
@@ -469,6 +560,27 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a) {
     u.y = pack_bf16x2(acc.z * inv, acc.w * inv);
     *reinterpret_cast<uint2 *>(o + d) = u;
     if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
+}
+
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel in the stream finishes; it calls grid_dependency_wait()
+// before reading anything.
+template <class... KArgs, class... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_t smem, cudaStream_t st,
+                              const Args &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
 }
 
 cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap, const MlaParams &a,
@@ -480,15 +592,13 @@ cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap,
     if (e != cudaSuccess) return e;
     const int grid = nq_wave * a.splits;
     if (grid == 0) return cudaSuccess;
-    k3_sparse_mla<<<grid, kMlaThreads, smem, st>>>(qmap, kvmap, a);
-    return cudaGetLastError();
+    return launch_pdl(k3_sparse_mla, grid, kMlaThreads, smem, st, qmap, kvmap, a);
 }
 
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st) {
     const int grid = nq_wave * a.h;
     if (grid == 0 || a.splits <= 1) return cudaSuccess;
-    k4_mla_combine<<<grid, 128, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k4_mla_combine, grid, 128, 0, st, a);
 }
 
 }  // namespace dsa
