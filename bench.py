@@ -158,18 +158,27 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- helpers
-def dist_init():
+def dist_init(backend: str = "nccl"):
+    """Rank, world and local rank from the torchrun environment; one process
+    per GPU over NCCL (gloo runs the same host logic on CPU, in tests)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
+
+
+def replica_inputs(cid: int, rank: int):
+    """Each rank runs its own replica batch (the path has no exchange step):
+    the same workload shape, its own seeded draw."""
+    return make_inputs(cid, seed_offset=rank * 101)
 
 
 def barrier(world):
@@ -179,12 +188,19 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The job's time is the slowest rank's (a device-timed value per rank)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_rate(units_per_rank: int, steps: int, world: int, t_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * steps * world / t_max
 
 
 def algorithmic_bytes(inp):
@@ -210,7 +226,7 @@ def algorithmic_bytes(inp):
 def run_ours(args, world, rank):
     cid = WORKLOADS[args.workload]
     t_gen = time.time()
-    inp = make_inputs(cid, seed_offset=rank * 101)
+    inp = replica_inputs(cid, rank)
     db = upload(inp)
     torch.cuda.synchronize()
     gen_s = time.time() - t_gen
@@ -331,7 +347,7 @@ def run_ours(args, world, rank):
     mla_tflops = alg["flops_attention"] / (t_mla / args.steps) / 1e12
     step_gbs = (alg["indexer"] + alg["attention"]) / (t_total / args.steps) / 1e9
     total_q = inp.nq * args.steps * world
-    qps = total_q / t_max
+    qps = job_rate(inp.nq, args.steps, world, t_max)
     res = {
         "metric": METRIC,
         "value": qps,
