@@ -23,11 +23,11 @@ constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
 constexpr int kSelBinsHost = 2048;
 constexpr long long kHistWaitCycles = 100000;  // ~50 us: bounded wait for a query's full histogram
 
-// Shared words an ordered emission over n elements by `nwarps` warps needs
-// for its recorded ballots (one uint4 per 128-element step of each warp's
-// slice; see emit_ordered).
+// Shared words an ordered emission over n elements by `nwarps` warps needs:
+// one uint4 of ballots per 128-element step of each warp's slice, then 32
+// words of step prefixes per warp (see emit_ordered).
 __host__ __device__ constexpr int emit_ballot_words(int n, int nwarps) {
-    return 4 * nwarps * ((((n + nwarps - 1) / nwarps + 127) & ~127) / 128);
+    return 4 * nwarps * ((((n + nwarps - 1) / nwarps + 127) & ~127) / 128) + 32 * nwarps;
 }
 
 struct K1Params {

@@ -107,6 +107,19 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// Bulk store of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from shared to global memory, tracked by this thread's bulk groups.  The
+// shared source must be made visible to the async proxy first
+// (fence_proxy_async_smem), and must not be reused or freed before
+// bulk_wait_read() returns.
+__device__ __forceinline__ void bulk_store(void *gdst, const void *ssrc, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(smem_u32(ssrc)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has read its source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Ask L2 to fetch [ptr, ptr + bytes) (bytes a multiple of 16, ptr 16-aligned).
 __device__ __forceinline__ void prefetch_l2_bulk(const void *ptr, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");

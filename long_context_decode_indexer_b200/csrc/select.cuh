@@ -151,17 +151,21 @@ __device__ uint64_t radix_refine(const Src &src, int n, uint64_t prefix, int pas
 // are handed to out(slot, v) with consecutive slots base, base + 1, ... in
 // increasing i.  Warp w owns a contiguous slice (a multiple of 128
 // elements) in steps of 128: each lane tests four consecutive elements per
-// step (one src.load4), and four ballots (one per element of the lanes'
-// quads) record the step's matches.  The ballot loop has no divergent branch
-// (a diverged warp must reconverge before every ballot, which costs more
-// than the test itself): loads are clamped into the slice and lane t keeps
-// the ballots of step t in a register, written to `bal` after each batch of
-// 32 steps.  After one block-wide scan of the warps' match counts, the
-// second pass walks the recorded ballots: a step without a match costs a
-// shuffle, and only lanes with a match reload their quad; a lane's slot is
-// the number of matches in lower lanes (popc of the ballots below it).
+// step (one src.load4), giving a 4-bit match mask; four ballots (one per
+// element of the lanes' quads) record the step's matches for the warp.
+//
+// Pass 1 keeps each lane's masks in registers (up to 32 steps: two 64-bit
+// words) and the step ballots in `bal`; a warp scan of the steps' match
+// counts gives every step its first slot within the warp, and one
+// block-wide scan of the warps' totals gives every warp its first slot.
+// Pass 2 is per lane: a lane visits only the steps where it has a match
+// (usually none or one), reads that step's ballots and prefix, reloads its
+// quad and emits.  No loop in either pass branches on data while the warp
+// must stay converged.  Slices longer than 32 steps (never planned) take a
+// slower path that re-tests every step.
 // Returns the next free slot.  `wsum`: 32 shared words; `bal`: shared, at
-// least emit_ballot_words(n, warps) / 4 uint4.
+// least emit_ballot_words(n, warps) / 4 uint4, plus one word per step for the
+// step prefixes when a slice has at most 32 steps (emit_ballot_words covers it).
 template <class Src, class Pred, class Out>
 __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const Out &out,
                                  uint32_t base, uint32_t *wsum, uint4 *bal) {
@@ -169,61 +173,110 @@ __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const 
     const int per = ((n + nw - 1) / nw + 127) & ~127;
     const int lo = min(warp * per, n), hi = min(lo + per, n);
     const int steps = (hi - lo + 127) / 128;
-    uint4 *wb = bal + warp * (per / 128);
-    uint32_t cnt = 0;  // warp-uniform
-    for (int b0 = 0; b0 < steps; b0 += 32) {
-        const int nb = min(32, steps - b0);
+    const int wsteps = per / 128;  // steps of every full slice (same for all warps)
+    uint4 *wb = bal + warp * wsteps;
+    const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
+    uint32_t before = 0, total = 0;
+
+    if (wsteps <= 32) {
+        // ---- pass 1: masks in registers, ballots and step prefixes in shared
+        uint64_t mask01 = 0, mask23 = 0;  // 4 bits per step: steps 0-15, 16-31
         uint4 mine = make_uint4(0, 0, 0, 0);
-        for (int t = 0; t < nb; ++t) {
-            const int i0 = lo + 128 * (b0 + t) + 4 * lane;
+        for (int t = 0; t < steps; ++t) {
+            const int i0 = lo + 128 * t + 4 * lane;
             uint64_t v[4];
             src.load4(i0 < hi ? i0 : lo, v);  // clamped: no branch around the load
             uint32_t m = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) m |= ((i0 + e < hi) & pred(v[e])) ? (1u << e) : 0u;
+            if (t < 16) mask01 |= static_cast<uint64_t>(m) << (4 * t);
+            else mask23 |= static_cast<uint64_t>(m) << (4 * (t - 16));
             const uint32_t q0 = __ballot_sync(0xffffffffu, m & 1u);
             const uint32_t q1 = __ballot_sync(0xffffffffu, m & 2u);
             const uint32_t q2 = __ballot_sync(0xffffffffu, m & 4u);
             const uint32_t q3 = __ballot_sync(0xffffffffu, m & 8u);
             mine = lane == t ? make_uint4(q0, q1, q2, q3) : mine;
-            cnt += __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
         }
-        if (lane < nb) wb[b0 + lane] = mine;
+        // lane t: matches of step t -> exclusive prefix over steps
+        const uint32_t tot_t = __popc(mine.x) + __popc(mine.y) + __popc(mine.z) + __popc(mine.w);
+        const uint32_t incl = warp_incl_scan(tot_t);
+        uint32_t *wpre = reinterpret_cast<uint32_t *>(bal + nw * wsteps) + warp * 32;
+        if (lane < steps) {
+            wb[lane] = mine;
+            wpre[lane] = incl - tot_t;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        for (int w = 0; w < nw; ++w) {
+            const uint32_t c = wsum[w];
+            before += (w < warp) ? c : 0u;
+            total += c;
+        }
+        // ---- pass 2: each lane visits only its own matching steps
+        const uint32_t wbase = base + before;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            uint64_t mm = half == 0 ? mask01 : mask23;
+            while (mm != 0) {
+                const int bit = __ffsll(static_cast<long long>(mm)) - 1;
+                const int t = (bit >> 2) + 16 * half;
+                const uint32_t own = static_cast<uint32_t>(mm >> (bit & ~3)) & 0xFu;
+                mm &= ~(static_cast<uint64_t>(0xFu) << (bit & ~3));
+                const uint4 q = wb[t];
+                const uint32_t s0 = wbase + wpre[t] + __popc(q.x & lt) + __popc(q.y & lt) +
+                                    __popc(q.z & lt) + __popc(q.w & lt);
+                uint64_t v[4];
+                src.load4(lo + 128 * t + 4 * lane, v);
+                const uint32_t o0 = own & 1u, o1 = (own >> 1) & 1u, o2 = (own >> 2) & 1u;
+                const uint32_t s1 = s0 + o0, s2 = s1 + o1, s3 = s2 + o2;
+                if (own & 1u) out(s0, v[0]);
+                if (own & 2u) out(s1, v[1]);
+                if (own & 4u) out(s2, v[2]);
+                if (own & 8u) out(s3, v[3]);
+            }
+        }
+        __syncthreads();
+        return base + total;
+    }
+
+    // ---- slices of more than 32 steps: count, scan, then re-test every step
+    uint32_t cnt = 0;  // warp-uniform
+    for (int t = 0; t < steps; ++t) {
+        const int i0 = lo + 128 * t + 4 * lane;
+        uint64_t v[4];
+        src.load4(i0 < hi ? i0 : lo, v);
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m |= ((i0 + e < hi) & pred(v[e])) ? (1u << e) : 0u;
+        cnt += __popc(__ballot_sync(0xffffffffu, m & 1u)) + __popc(__ballot_sync(0xffffffffu, m & 2u)) +
+               __popc(__ballot_sync(0xffffffffu, m & 4u)) + __popc(__ballot_sync(0xffffffffu, m & 8u));
     }
     if (lane == 0) wsum[warp] = cnt;
     __syncthreads();
-    uint32_t before = 0, total = 0;
     for (int w = 0; w < nw; ++w) {
         const uint32_t c = wsum[w];
         before += (w < warp) ? c : 0u;
         total += c;
     }
     uint32_t slot = base + before;
-    const uint32_t lt = (1u << lane) - 1u;  // lanes below this one
-    for (int b0 = 0; b0 < steps; b0 += 32) {
-        const int nb = min(32, steps - b0);
-        const uint4 mine = lane < nb ? wb[b0 + lane] : make_uint4(0, 0, 0, 0);
-        for (int t = 0; t < nb; ++t) {
-            const uint32_t q0 = __shfl_sync(0xffffffffu, mine.x, t);
-            const uint32_t q1 = __shfl_sync(0xffffffffu, mine.y, t);
-            const uint32_t q2 = __shfl_sync(0xffffffffu, mine.z, t);
-            const uint32_t q3 = __shfl_sync(0xffffffffu, mine.w, t);
-            const uint32_t tot = __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
-            if (tot == 0u) continue;  // warp-uniform
-            // every lane reloads its quad and computes the four slots; the
-            // stores are predicated, not branched around
-            uint64_t v[4];
-            src.load4(lo + 128 * (b0 + t) + 4 * lane, v);
-            const uint32_t o0 = (q0 >> lane) & 1u, o1 = (q1 >> lane) & 1u;
-            const uint32_t o2 = (q2 >> lane) & 1u, o3 = (q3 >> lane) & 1u;
-            const uint32_t s0 = slot + __popc(q0 & lt) + __popc(q1 & lt) + __popc(q2 & lt) + __popc(q3 & lt);
-            const uint32_t s1 = s0 + o0, s2 = s1 + o1, s3 = s2 + o2;
-            if (o0) out(s0, v[0]);
-            if (o1) out(s1, v[1]);
-            if (o2) out(s2, v[2]);
-            if (o3) out(s3, v[3]);
-            slot += tot;
-        }
+    for (int t = 0; t < steps; ++t) {
+        const int i0 = lo + 128 * t + 4 * lane;
+        uint64_t v[4];
+        src.load4(i0 < hi ? i0 : lo, v);
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m |= ((i0 + e < hi) & pred(v[e])) ? (1u << e) : 0u;
+        const uint32_t q0 = __ballot_sync(0xffffffffu, m & 1u);
+        const uint32_t q1 = __ballot_sync(0xffffffffu, m & 2u);
+        const uint32_t q2 = __ballot_sync(0xffffffffu, m & 4u);
+        const uint32_t q3 = __ballot_sync(0xffffffffu, m & 8u);
+        const uint32_t s0 = slot + __popc(q0 & lt) + __popc(q1 & lt) + __popc(q2 & lt) + __popc(q3 & lt);
+        const uint32_t s1 = s0 + (m & 1u), s2 = s1 + ((m >> 1) & 1u), s3 = s2 + ((m >> 2) & 1u);
+        if (m & 1u) out(s0, v[0]);
+        if (m & 2u) out(s1, v[1]);
+        if (m & 4u) out(s2, v[2]);
+        if (m & 8u) out(s3, v[3]);
+        slot += __popc(q0) + __popc(q1) + __popc(q2) + __popc(q3);
     }
     __syncthreads();
     return base + total;

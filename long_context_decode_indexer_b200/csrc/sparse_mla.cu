@@ -55,6 +55,8 @@ constexpr int kGatherWarp0 = 6;                     // warps 6..9 gather rows (a
 constexpr int kGatherThreads = 128;
 constexpr int kPass1Threads = 256;                  // pass-1 gather threads (warps 0-3, 6-9)
 constexpr int kPass1Rows = kMlaMaxRows / (kPass1Threads / 8);  // rows per pass-1 gather thread
+constexpr int kEpiPitch = 512 + 16;                 // epilogue staging row pitch (bytes)
+constexpr int kEpiGroupBytes = 128 * kEpiPitch;     // one epilogue group's staging rows
 constexpr int kGatherLag = 3;                       // pass-1 chunks in flight per gather thread
 constexpr int kVLag = 2;                            // pass-2 tiles in flight per gather thread
 
@@ -76,6 +78,8 @@ struct MlaSmem {
 };
 
 static_assert(sizeof(MlaSmem) <= 2048, "MlaSmem must fit the reserve in mla_layout()");
+static_assert(2 * kEpiGroupBytes <= 2 * 128 * kMlaMaxRows * 2 + kMlaVStages * kVTileBytes,
+              "epilogue staging must fit the pass-2 area (free once O is complete)");
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -148,16 +152,14 @@ __device__ bool gather_pass1(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int
 }
 
 // O / l of this thread's head row, columns [c_begin, c_begin + 256): TMEM ->
-// registers -> 16-byte stores of the row (bf16 output, or fp16 partials).
-// A thread writes whole 32-byte sectors of its own row, so the stores need
-// no staging and no barrier.  The TMEM loads are warp-collective: every lane
-// runs them, and only the stores are skipped for padding heads (hrow >= h).
+// registers -> this thread's staging row in shared memory (`srow`, 512 bytes,
+// rows kEpiPitch apart so that the 16-byte writes of a warp spread over the
+// banks) -> one 512-byte bulk store into the row of the output (bf16) or of
+// the split partials (fp16).  The TMEM loads are warp-collective: every lane
+// runs them; only the store is skipped for padding heads (hrow >= h).  The
+// caller waits for the bulk store (bulk_wait_read) before the CTA exits.
 __device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, int q, int wq, int sp,
-                             float inv_l, int c_begin) {
-    const bool live = hrow < a.h;
-    uint16_t *dst = a.splits == 1
-                        ? a.out + (static_cast<int64_t>(q) * a.h + (live ? hrow : 0)) * kDv
-                        : a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+                             float inv_l, int c_begin, uint8_t *srow) {
     for (int c1 = c_begin; c1 < c_begin + 256; c1 += 64) {
         uint32_t v2[2][32];
         tmem_ld32(lane_addr + c1, v2[0]);
@@ -172,8 +174,16 @@ __device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, i
                 const float x0 = __uint_as_float(u[2 * e]) * inv_l, x1 = __uint_as_float(u[2 * e + 1]) * inv_l;
                 w[e] = a.splits == 1 ? pack_bf16x2(x0, x1) : pack_half2(x0, x1);
             }
-            if (live) *reinterpret_cast<uint4 *>(dst + c1 + g * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4 *>(srow + (c1 - c_begin) * 2 + g * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+    }
+    fence_proxy_async_smem();  // the staging row is read by the bulk copy
+    if (hrow < a.h) {
+        uint16_t *dst = a.splits == 1
+                            ? a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv
+                            : a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+        bulk_store(dst + c_begin, srow, 512);
+        bulk_commit();
     }
 }
 
@@ -333,7 +343,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             ok = bar_and(3, 256, ok);
             if (ok) {
                 tc_fence_after();
-                store_output(a, lane_addr, hrow, q, wq, sp, sm.inv_l[hrow], 256);
+                store_output(a, lane_addr, hrow, q, wq, sp, sm.inv_l[hrow], 256,
+                             ptile + kEpiGroupBytes + hrow * kEpiPitch);
             }
         } else if (warp == 5) {
             // ------------------------------------------------ MMA issuer
@@ -442,11 +453,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                         uint32_t hi[4], lo[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
+                            // one paired conversion each for P_hi and P_lo
                             const float a0 = p[g8 * 8 + 2 * e], a1 = p[g8 * 8 + 2 * e + 1];
-                            const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-                            hi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                                    (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-                            lo[e] = pack_bf16x2(a0 - __bfloat162float(h0), a1 - __bfloat162float(h1));
+                            const __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+                            const float2 hf = __bfloat1622float2(h2);
+                            const __nv_bfloat162 l2 = __floats2bfloat162_rn(a0 - hf.x, a1 - hf.y);
+                            hi[e] = *reinterpret_cast<const uint32_t *>(&h2);
+                            lo[e] = *reinterpret_cast<const uint32_t *>(&l2);
                         }
                         const uint32_t off = rowoff + ((ch ^ (hrow & 7)) << 4);
                         *reinterpret_cast<uint4 *>(ptile + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -471,7 +484,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     if (a.splits == 1) a.lse[static_cast<int64_t>(q) * a.h + hrow] = lse_v;
                     else a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = lse_v;
                 }
-                store_output(a, lane_addr, hrow, q, wq, sp, inv_l, 0);
+                store_output(a, lane_addr, hrow, q, wq, sp, inv_l, 0, ptile + hrow * kEpiPitch);
             } else if (lane == 0) {
                 record_status(a.status, DSA_ERR_TIMEOUT);
             }
@@ -492,6 +505,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
         }
     }
 
+    bulk_wait_read();  // the epilogue's bulk stores have read their staging rows
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
