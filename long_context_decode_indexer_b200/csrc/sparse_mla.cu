@@ -513,67 +513,63 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 }
 
 // Merge the splits of one (query, head): out = sum_s w_s o_s / sum_s w_s with
-// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  Warp 0 reads the
-// splits' log-sum-exps (one lane each; splits <= 32) and publishes the
-// weights; then each thread combines 4 columns, its partial loads issued in
-// batches of 8 splits so that they are in flight together.
-__global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a) {
-    __shared__ float wts[32];
-    __shared__ float stot, smx;
+// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  One warp covers 256
+// value columns of one head (8 per lane, 16-byte loads and stores), so a
+// head takes two warps and a 128-thread CTA two heads.  Every warp reads the
+// head's split log-sum-exps itself (lane s holds split s; splits <= 32) and
+// gets the weights by shuffles: no shared memory, no CTA barrier.  The
+// partial loads of all splits are issued before any is used.
+__global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_slots) {
     grid_dependency_wait();  // the partials come from the preceding attention kernel
-    const int wq = blockIdx.x / a.h, hh = blockIdx.x % a.h;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int head_slot = blockIdx.x * 2 + (warp >> 1);  // (query in wave) * h + head
+    if (head_slot >= n_slots) return;                     // whole warp: odd head count
+    const int wq = head_slot / a.h, hh = head_slot % a.h;
     const int q = a.q0 + wq;
     const int64_t row0 = static_cast<int64_t>(wq) * a.splits * 128 + hh;  // split s: row0 + 128 s
-    if (threadIdx.x < 32) {
-        const int s = threadIdx.x;
-        const float ls = s < a.splits ? a.part_lse[row0 + 128 * s] : -INFINITY;
-        float mx = ls;
+    const int d = (warp & 1) * 256 + lane * 8;
+    const float ls = lane < a.splits ? a.part_lse[row0 + 128 * lane] : -INFINITY;
+    float mx = ls;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        const float w = (mx == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - mx);
-        float t = w;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float w = (mx == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - mx);
+    float tot = w;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        wts[s] = w;
-        if (s == 0) {
-            stot = t;
-            smx = mx;
-        }
-    }
-    __syncthreads();
-    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv;
-    const int d = threadIdx.x * 4;
-    const float tot = stot, mx = smx;
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv + d;
     if (mx == -INFINITY) {
-        *reinterpret_cast<uint2 *>(o + d) = make_uint2(0, 0);
-        if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
+        *reinterpret_cast<uint4 *>(o) = make_uint4(0, 0, 0, 0);
+        if (lane == 0 && (warp & 1) == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
         return;
     }
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int s0 = 0; s0 < a.splits; s0 += 8) {
-        uint2 raw[8];
+        uint4 raw[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
             raw[u] = s0 + u < a.splits
-                         ? *reinterpret_cast<const uint2 *>(a.part_o + (row0 + 128 * (s0 + u)) * kDv + d)
-                         : make_uint2(0, 0);
+                         ? *reinterpret_cast<const uint4 *>(a.part_o + (row0 + 128 * (s0 + u)) * kDv + d)
+                         : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const float wgt = s0 + u < a.splits ? wts[s0 + u] : 0.f;
-            const float2 lo2 = __half22float2(*reinterpret_cast<const __half2 *>(&raw[u].x));
-            const float2 hi2 = __half22float2(*reinterpret_cast<const __half2 *>(&raw[u].y));
-            acc.x = fmaf(wgt, lo2.x, acc.x);
-            acc.y = fmaf(wgt, lo2.y, acc.y);
-            acc.z = fmaf(wgt, hi2.x, acc.z);
-            acc.w = fmaf(wgt, hi2.y, acc.w);
+            const float wgt = __shfl_sync(0xffffffffu, w, (s0 + u) & 31);
+            const uint32_t r4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r4[e]));
+                acc[2 * e] = fmaf(wgt, f.x, acc[2 * e]);
+                acc[2 * e + 1] = fmaf(wgt, f.y, acc[2 * e + 1]);
+            }
         }
     }
     const float inv = 1.f / tot;
-    uint2 u;
-    u.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    u.y = pack_bf16x2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2 *>(o + d) = u;
-    if (threadIdx.x == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
+    uint4 res;
+    res.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    res.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    res.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+    res.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+    *reinterpret_cast<uint4 *>(o) = res;
+    if (lane == 0 && (warp & 1) == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
 }
 
 // Launch with programmatic stream serialization: the kernel may begin while
@@ -610,9 +606,9 @@ cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap,
 }
 
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st) {
-    const int grid = nq_wave * a.h;
+    const int grid = (nq_wave * a.h + 1) / 2;  // two heads per CTA
     if (grid == 0 || a.splits <= 1) return cudaSuccess;
-    return launch_pdl(k4_mla_combine, grid, 128, 0, st, a);
+    return launch_pdl(k4_mla_combine, grid, 128, 0, st, a, nq_wave * a.h);
 }
 
 }  // namespace dsa
