@@ -56,7 +56,7 @@ K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
               "long_context_decode_indexer_b200/csrc/select.cuh",
               "long_context_decode_indexer_b200/csrc/ptx.cuh",
               "long_context_decode_indexer_b200/csrc/kernels.h")
-K1_PROFILED = {"sha256_16": "2966f871998939ba", "bytes_per_position": 131.23763020833334}
+K1_PROFILED = {"sha256_16": "8a4b7d790e67b55e", "bytes_per_position": 131.10498046875}
 
 
 def k1_traffic(inp):

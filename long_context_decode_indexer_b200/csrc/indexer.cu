@@ -514,9 +514,13 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             int b = grp;
             uint32_t aph = 0;
             for (int t = grp; t < ntiles; t += 2) {
-                // every lane waits; the warp proceeds only if all saw the
-                // phase complete (tcgen05.ld below is warp-collective)
-                const bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], aph) && !sm.abort);
+                // lane 0 polls (eight warps polling with every lane would
+                // steal issue slots from the producer and MMA threads); then
+                // every lane observes the completed phase itself -- its own
+                // acquire, which cannot fail: the buffer's next phase needs
+                // this warp's release below.  The warp proceeds only if all
+                // lanes saw it (tcgen05.ld below is warp-collective).
+                const bool ok = warp_wait(&sm.acc_full[b], aph, &sm.abort);
                 if (!ok) {
                     if (lane == 0) {
                         record_status(a.status, DSA_ERR_TIMEOUT);

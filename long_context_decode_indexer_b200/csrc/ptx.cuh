@@ -75,6 +75,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// Whole-warp wait: lane 0 polls (bounded), then every lane observes the
+// completed phase itself, so each lane has its own acquire.  Valid only when
+// the barrier cannot complete its following phase before this warp acts
+// (the usual ring protocol: the next phase needs this warp's arrival).
+// Returns the same value in every lane; false on timeout or `abort` set.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const volatile int32_t *abort) {
+    bool seen = true;
+    if ((threadIdx.x & 31) == 0) seen = mbar_wait(bar, parity) && !*abort;
+    seen = __shfl_sync(0xffffffffu, seen, 0);
+    if (seen) seen = mbar_try_wait(bar, parity);
+    return __all_sync(0xffffffffu, seen);
+}
+
 // --------------------------------------------------------------------- TMA
 // 2-D tiled load of a box into shared memory; completion is counted in bytes
 // on `bar`.  c0 is the innermost coordinate (elements), c1 the row.
