@@ -84,16 +84,17 @@ def peaks():
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """Samples SM clock, max clock, power and clock-event reasons while the
-    timed loops run: NVML polled every ~1 ms from a thread (read-only), plus
-    an nvidia-smi CSV record in gpurun_out/clocks.csv."""
+    timed loops run: NVML polled every ~1 ms from a thread (read-only), plus,
+    when `csv_path` is given, an nvidia-smi CSV record (every 200 ms)."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
     SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                   "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                   "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, csv_path: str = None):
         self.dev = device_index
+        self.csv_path = csv_path
         self.samples = []
         self.active = False
         self.stop = False
@@ -114,8 +115,10 @@ class ClockSampler:
             self.thread = threading.Thread(target=self._poll, daemon=True)
             self.thread.start()
         try:
-            os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-            self.fh = open(os.path.join(ROOT, "gpurun_out", "clocks.csv"), "w")
+            if not self.csv_path:
+                raise RuntimeError("no clock record requested")
+            os.makedirs(os.path.dirname(os.path.abspath(self.csv_path)), exist_ok=True)
+            self.fh = open(self.csv_path, "w")
             self.smi = subprocess.Popen(
                 ["stdbuf", "-oL", "nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.SMI_FIELDS,
                  "--format=csv", "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
@@ -270,7 +273,7 @@ def run_ours(args, world, rank):
     assert dsa.check_status(ws) == dsa.DSA_OK, dsa.last_error()
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(torch.cuda.current_device(), args.clocks_csv) as clk:
         clk.active = True
         t_total = timed(step, args.steps)
         torch.cuda.synchronize()
@@ -464,6 +467,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also record nvidia-smi clock samples (CSV) during the timed loops")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, _ = dist_init() if args.impl == "ours" else (
