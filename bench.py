@@ -206,6 +206,17 @@ def job_rate(units_per_rank: int, steps: int, world: int, t_max: float) -> float
     return units_per_rank * steps * world / t_max
 
 
+def workload_config(inp, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": inp.name, "nq": inp.nq, "context": int(inp.q_n.max()),
+            "topk": inp.topk, "h_idx": inp.h_idx, "d_idx": inp.d_idx, "heads": inp.h,
+            "d_qk": inp.d_qk, "d_v": inp.d_v, "paged": inp.page_table is not None,
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2: each step streams the %.0f MB index-K cache; "
+                  "no flush between steps (attention-only stage: L2 evicted by a 256 MiB "
+                  "read before each call)" % (algorithmic_bytes(inp)["indexer"] / 1e6)}
+
+
 def algorithmic_bytes(inp):
     """Bytes the three steps must move at minimum (per batch)."""
     n = inp.q_n.astype(np.int64)
@@ -366,13 +377,7 @@ def run_ours(args, world, rank):
         "data": "synthetic",
         "impl": "ours",
         "tokens_per_s": qps,
-        "config": {"workload": inp.name, "nq": inp.nq, "context": int(inp.q_n.max()),
-                   "topk": inp.topk, "h_idx": inp.h_idx, "d_idx": inp.d_idx, "heads": inp.h,
-                   "d_qk": inp.d_qk, "d_v": inp.d_v, "paged": paged,
-                   "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "inputs larger than L2: each step streams the %.0f MB index-K cache; "
-                         "no flush between steps (attention-only stage: L2 evicted by a 256 MiB "
-                         "read before each call)" % (alg["indexer"] / 1e6)},
+        "config": workload_config(inp, world),
         "roofline": {"bound": "hbm", "achieved": idx_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": idx_gbs / hbm, "traffic": k1_traffic(inp),
                      "kernel": "k1_indexer (fused indexer + TopK)",
@@ -447,10 +452,7 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": {"workload": inp.name, "nq": inp.nq, "context": int(inp.q_n.max()),
-                   "topk": inp.topk, "h_idx": inp.h_idx, "d_idx": inp.d_idx, "heads": inp.h,
-                   "d_qk": inp.d_qk, "d_v": inp.d_v, "paged": inp.page_table is not None,
-                   "parallelism": "single"},
+        "config": workload_config(inp, world),
         "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
                          "sample": "1 query of %s per step (full context), fp64 C oracle"
                                    % inp.name},
