@@ -429,7 +429,19 @@ def cpu_baseline(inp, target_s=15.0):
         qps, dt = qps1, dt1
     return {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
             "sample": "%d of %d queries of %s (full context), fp64 C oracle, %.1f s"
-                      % (n, inp.nq, inp.name, dt)}
+                      % (n, inp.nq, inp.name, dt),
+            "cpu": cpu_model()}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def run_reference(args, world, rank):
