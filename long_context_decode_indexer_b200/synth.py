@@ -113,7 +113,8 @@ def _normal_bf16(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.nd
 def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = None,
                 L: Optional[int] = None, ragged: bool = False, paged: Optional[bool] = None,
                 lengths: Optional[np.ndarray] = None, with_k_scale: bool = False,
-                topk: Optional[int] = None, h: Optional[int] = None) -> Inputs:
+                topk: Optional[int] = None, h: Optional[int] = None,
+                h_idx: Optional[int] = None, d_idx: Optional[int] = None) -> Inputs:
     """Inputs of workload ``config_id`` (1..5), optionally resized for tests.
 
     decode  : one query per sequence; query n = L (rows 0..L-1 visible).
@@ -128,7 +129,8 @@ def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = N
     kind = c["kind"]
     nseq = c["nseq"] if nseq is None else int(nseq)
     L = c["L"] if L is None else int(L)
-    h_idx, d_idx = c["h_idx"], c["d_idx"]
+    h_idx = c["h_idx"] if h_idx is None else int(h_idx)
+    d_idx = c["d_idx"] if d_idx is None else int(d_idx)
     h = c["h"] if h is None else int(h)
     k = c["topk"] if topk is None else int(topk)
     if paged is None:

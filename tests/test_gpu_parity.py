@@ -87,12 +87,19 @@ def test_fused_indexer_topk_equals_scores_then_topk(case):
         check_index_set_exact(idx_f[qi], idx_u[qi], int(inp.q_n[qi]), inp.topk)
 
 
-@pytest.mark.parametrize("case", ["tiny", "v32_multichunk", "prefill_pairs"])
+@pytest.mark.parametrize("case", ["tiny", "v32_multichunk", "prefill_pairs", "heads64_dim64",
+                                  "heads16_dim128", "key_scale"])
 def test_fused_indexer_topk_recall_against_oracle(case):
     if case == "tiny":
         inp = make_inputs(1)
     elif case == "v32_multichunk":
         inp = make_inputs(2, lengths=[20000, 2049, 9000])
+    elif case == "heads64_dim64":      # H_I = 64 with d_I = 64 (64-byte swizzle, N = 64)
+        inp = make_inputs(2, lengths=[9000, 3000], d_idx=64)
+    elif case == "heads16_dim128":     # H_I = 16 with d_I = 128 (N = 16)
+        inp = make_inputs(2, lengths=[9000, 3000], h_idx=16)
+    elif case == "key_scale":          # per-row key scales in the fused path
+        inp = make_inputs(2, lengths=[12000, 2500], with_k_scale=True)
     else:
         inp = make_inputs(4, L=2600)   # queries t = 0..2599: fallback and scored
     db = upload(inp)
@@ -102,7 +109,7 @@ def test_fused_indexer_topk_recall_against_oracle(case):
     else:
         sel = np.arange(inp.nq)
     ref = oracle.indexer_scores(inp.q_idx[sel], inp.w[sel], inp.kidx, inp.q_seq[sel], inp.q_n[sel],
-                                seq_row0=inp.seq_row0, ld=inp.max_n)
+                                seq_row0=inp.seq_row0, ld=inp.max_n, k_scale=inp.k_scale)
     check_recall(idx[sel], ref, inp.q_n[sel], inp.topk)
 
 
@@ -170,9 +177,10 @@ def test_forward_matches_oracle(case):
     check_attention(out[sel], lse[sel], ref_out, ref_lse)
 
 
-def test_paged_forward_equals_contiguous_bit_for_bit():
+@pytest.mark.parametrize("page_size", [64, 128])
+def test_paged_forward_equals_contiguous_bit_for_bit(page_size):
     inp = make_inputs(3, lengths=[3000, 2049, 700])
-    pg = to_paged(inp)
+    pg = to_paged(inp, page_size=page_size)
     a = gpu_forward(upload(inp))
     b = gpu_forward(upload(pg))
     for qi in range(inp.nq):
