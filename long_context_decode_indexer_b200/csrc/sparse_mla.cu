@@ -57,8 +57,8 @@ constexpr int kPass1Threads = 256;                  // pass-1 gather threads (wa
 constexpr int kPass1Rows = kMlaMaxRows / (kPass1Threads / 8);  // rows per pass-1 gather thread
 constexpr int kEpiPitch = 512 + 16;                 // epilogue staging row pitch (bytes)
 constexpr int kEpiGroupBytes = 128 * kEpiPitch;     // one epilogue group's staging rows
-constexpr int kGatherLag = 3;                       // pass-1 chunks in flight per gather thread
-constexpr int kVLag = 2;                            // pass-2 tiles in flight per gather thread
+constexpr int kGatherLag = 2;                       // pass-1 chunks a gather thread publishes behind its newest
+constexpr int kVLag = 1;                            // pass-2 tiles a gather thread publishes behind its newest
 
 struct MlaSmem {
     uint64_t full[kMlaStages];
