@@ -21,16 +21,20 @@
 //           (the A operands of pass 2) and keeps the row sum.  A single bf16
 //           P would add ~1e-3 relative error on top of the ~1.7e-3 that the
 //           bf16 output itself carries; the pair makes P exact to ~2^-16.
-//   pass 2  O[128 x 512] = P_hi . V + P_lo . V, V re-gathered by the same
-//           warps (32-row tiles, L2 hits) into an MN-major swizzled layout; O
+//   pass 2  O[128 x 512] = P_hi . V + P_lo . V, V re-gathered by warps 6-9
+//           (32-row tiles, L2 hits) into an MN-major swizzled layout; O
 //           takes all 512 TMEM columns, which is why S and O are not live at
 //           the same time.
+// The gather threads publish each staged chunk or tile as soon as the
+// following one is requested (a lag of two chunks / one tile): publishing
+// later kept the tensor cores waiting on data that had already landed.
 // Epilogue: the softmax warps write columns 0..255 of O / l, the gather warps
-// columns 256..511, each thread straight from TMEM to its head's row.  A split writes O / l in fp16 (its values are convex
-// combinations of bf16 rows, so fp16's range suffices and its rounding,
-// 2^-12 relative, is far below the bf16 output's) and its log-sum-exp; the
-// combine kernel merges splits by their log-sum-exp.  With one split the CTA
-// writes the final output.
+// columns 256..511; each thread moves its head's row from TMEM to a staging
+// row in shared memory and issues one 512-byte bulk store.  A split writes
+// O / l in fp16 (its values are convex combinations of bf16 rows, so fp16's
+// range suffices and its rounding, 2^-12 relative, is far below the bf16
+// output's) and its log-sum-exp; the combine kernel merges splits by their
+// log-sum-exp.  With one split the CTA writes the final output.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
