@@ -180,7 +180,10 @@ int dsa_indexer_topk(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  *   out          [nq, h, d_v] bf16;  lse [nq, h] fp32 (natural log)
  * A query with no valid entry gets out = 0 and lse = -inf.
  * Arithmetic: bf16 tensor-core products with fp32 accumulation; softmax in
- * fp32; P rounded to bf16 for the P.V product. */
+ * fp32; P enters the P.V product as a pair of bf16 tiles (P_hi + P_lo,
+ * together exact to about 2^-16).  When a query's rows are split over
+ * several CTAs, each split's normalised output is kept in ws as fp16 and
+ * the splits are merged by their log-sum-exp. */
 int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q,
                           const void *kv_cache, int64_t kv_row_stride,
                           const int32_t *idx, void *out, float *lse, void *ws,
