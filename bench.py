@@ -404,6 +404,7 @@ def run_ours(args, world, rank):
         "stages": {
             "indexer_topk_us": t_idx / args.steps * 1e6,
             "indexer_topk_gbs": idx_gbs,
+            "indexer_topk_frac_nominal_8tbs": idx_gbs / 8000.0,
             "sparse_mla_us": t_mla / args.steps * 1e6,
             "sparse_mla_gbs": mla_gbs,
             "sparse_mla_tflops": mla_tflops,
