@@ -72,6 +72,12 @@ def _load():
             lib.dsa_oracle_forward.argtypes = [
                 _I32, _I32, _I32, _I32, _I32, _I32, _I32, _F64, _P, _P, _P, _P,
                 _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32]
+            lib.dsa_oracle_f64_to_e4m3.restype = ctypes.c_uint8
+            lib.dsa_oracle_f64_to_e4m3.argtypes = [_F64]
+            lib.dsa_oracle_indexer_project.restype = ctypes.c_int
+            lib.dsa_oracle_indexer_project.argtypes = [
+                _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _F64,
+                _P, _F64, _P, _P, _P, _P, _P, _P, _P, _P, _I32]
             _lib = lib
     return _lib
 
@@ -214,3 +220,39 @@ def forward(q_idx, w, kidx, q, kv, q_seq, q_n, *, k, scale, d_v=512,
     if rc != 0:
         raise RuntimeError("dsa_oracle_forward failed: %d" % rc)
     return idx, out, lse
+
+
+def f64_to_e4m3(x: float) -> int:
+    """E4M3 code nearest to x after clamping to [-448, 448] (ties to even)."""
+    return int(_load().dsa_oracle_f64_to_e4m3(float(x)))
+
+
+def indexer_project(x, q_lora, w_qb, w_k, w_proj, ln_gamma, ln_beta, positions, *,
+                    h_idx, d_idx, rope_dim=64, ln_eps=1e-6, rope_theta=10000.0, nthreads=0):
+    """The indexer's q^I / k^I / w producer for nt tokens (see the C source).
+
+    x [nt, hidden] and q_lora [nt, q_lora_rank] bf16 bits; w_qb
+    [h_idx*d_idx, q_lora_rank], w_k [d_idx, hidden], w_proj [h_idx, hidden]
+    bf16 bits ([out, in]); ln_gamma / ln_beta [d_idx] float32; positions [nt]
+    int32.  Returns a dict: q_f, k_f, w_f (fp64 before quantisation), q_code,
+    q_scale, k_code, k_scale (FP8 codes and power-of-two scales), w_bf16.
+    """
+    x = _c(x, np.uint16)
+    nt, hidden = x.shape
+    q_lora = _c(q_lora, np.uint16)
+    rank = q_lora.shape[1]
+    w_qb, w_k, w_proj = _c(w_qb, np.uint16), _c(w_k, np.uint16), _c(w_proj, np.uint16)
+    ln_gamma, ln_beta = _c(ln_gamma, np.float32), _c(ln_beta, np.float32)
+    positions = _c(positions, np.int32)
+    out = dict(q_f=np.empty((nt, h_idx, d_idx)), k_f=np.empty((nt, d_idx)), w_f=np.empty((nt, h_idx)),
+               q_code=np.empty((nt, h_idx, d_idx), np.uint8), q_scale=np.empty((nt, h_idx), np.float32),
+               k_code=np.empty((nt, d_idx), np.uint8), k_scale=np.empty(nt, np.float32),
+               w_bf16=np.empty((nt, h_idx), np.uint16))
+    rc = _load().dsa_oracle_indexer_project(
+        nt, hidden, rank, int(h_idx), int(d_idx), int(rope_dim), _ptr(x), _ptr(q_lora), _ptr(w_qb),
+        _ptr(w_k), _ptr(w_proj), _ptr(ln_gamma), _ptr(ln_beta), float(ln_eps), _ptr(positions),
+        float(rope_theta), _ptr(out["q_f"]), _ptr(out["k_f"]), _ptr(out["w_f"]), _ptr(out["q_code"]),
+        _ptr(out["q_scale"]), _ptr(out["k_code"]), _ptr(out["k_scale"]), _ptr(out["w_bf16"]), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_indexer_project failed: %d" % rc)
+    return out

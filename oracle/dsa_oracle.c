@@ -60,6 +60,28 @@ double dsa_oracle_e4m3_to_f64(uint8_t code)
     return sign ? -v : v;
 }
 
+/* E4M3 encoding of a real number: the nearest finite E4M3 value after
+ * clamping to [-448, 448], ties to the code with an even mantissa; NaN maps
+ * to the NaN code.  Found by trying all 127 non-negative finite codes
+ * (plain rather than clever).  Used by the q^I / k^I producer below. */
+uint8_t dsa_oracle_f64_to_e4m3(double x)
+{
+    if (isnan(x)) return 0x7F;
+    int sign = signbit(x) ? 1 : 0;
+    double a = fabs(x);
+    if (a > 448.0) a = 448.0;
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c < 0x7F; ++c) {
+        double d = fabs(dsa_oracle_e4m3_to_f64((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(best | (sign << 7));
+}
+
 /* bfloat16: the upper 16 bits of an IEEE-754 binary32.  Widening is exact. */
 double dsa_oracle_bf16_to_f64(uint16_t bits)
 {
@@ -396,4 +418,156 @@ int dsa_oracle_forward(int32_t nq, int32_t h_idx, int32_t d_idx, int32_t h,
     return dsa_oracle_sparse_mla(nq, h, d_qk, d_v, scale, q, kv, kv_row_stride,
                                  q_seq, q_n, seq_row0, page_table, max_pages,
                                  page_size, idx_out, k, out, lse, nthreads);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Next step on the path: the indexer's q^I / k^I / w producer                 */
+/* ------------------------------------------------------------------------- */
+
+/* The indexer's own projections, per token t ([yuyanqi] sections 4.1-4.3):
+ *   q^I[t]   = W_qb . q_lora[t], reshaped to [H_I, d_I]        (wq_b)
+ *   k^I[t]   = LayerNorm(W_k . x[t])                            (wk, k_norm)
+ *   the first rope_dim dims of every q^I head and of k^I get the indexer's
+ *   own RoPE at the token's position (split [rope_head_dim, ...], then
+ *   rotary_emb(positions, q_rope, k_rope))
+ *   w[t]     = (W_proj . x[t]) * H_I^-1/2 * d_I^-1/2 * q_scale   (weights_proj,
+ *              the n_heads^-0.5 and softmax_scale factors, the q scale)
+ * then q^I and k^I go to FP8 with a scale ("q_scale" folded into w; "k_s",
+ * e8m0, multiplying the score).
+ *
+ * Readings where the pages are silent: linear layers are y = W x with W
+ * stored [out, in] (bf16), x bf16; LayerNorm is (k - mean) / sqrt(var + eps)
+ * * gamma + beta with the biased variance; RoPE rotates the pairs (2i, 2i+1)
+ * of the rope dims by pos * theta^(-2i / rope_dim) (the rotary embedding's
+ * own definition); both scales are powers of two (the e8m0 of k_s, and the
+ * same for q so that folding it into w is exact): s = 2^ceil(log2(amax /
+ * 448)), 1 when amax = 0, one per (token, head) for q and one per token for
+ * k; codes = e4m3(value / s).  w is then rounded to bf16.
+ *
+ * Outputs (any may be NULL): q_f [nt, H_I, d_I] and k_f [nt, d_I] (fp64,
+ * after RoPE, before quantisation), w_f [nt, H_I] (fp64, folded), q_code /
+ * q_scale, k_code / k_scale (the FP8 codes and their scales), w_bf16. */
+static double bf(const uint16_t *p, int64_t i) { return dsa_oracle_bf16_to_f64(p[i]); }
+
+static double pow2_scale(double amax)
+{
+    if (!(amax > 0.0)) return 1.0;
+    return ldexp(1.0, (int)ceil(log2(amax / 448.0)));
+}
+
+/* bfloat16 nearest to v (ties to even), rounded once from fp64: 8
+ * significant bits, spacing 2^(e-7) for |v| in [2^e, 2^(e+1)), 2^-133 below
+ * the smallest normal; beyond the largest finite value -> infinity. */
+static uint16_t f64_to_bf16_rne(double v)
+{
+    if (isnan(v)) return 0x7FC0;
+    double a = fabs(v);
+    double r = 0.0;
+    if (a > 0.0) {
+        int e;
+        frexp(a, &e);        /* a = f * 2^e, f in [0.5, 1): a in [2^(e-1), 2^e) */
+        int lo = e - 1 - 7;  /* spacing exponent of the 8-significant-bit grid */
+        if (lo < -133) lo = -133;
+        r = ldexp(rint(ldexp(a, -lo)), lo);  /* rint: ties to even */
+        if (r > ldexp(255.0, 120)) r = INFINITY;  /* largest finite: (2 - 2^-7) * 2^127 */
+    }
+    float f = (float)(signbit(v) ? -r : r);  /* exact: r has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    return (uint16_t)(u >> 16);
+}
+
+static void rope_rotate(double *v, int32_t rope_dim, int32_t pos, double theta)
+{
+    for (int32_t i = 0; i < rope_dim / 2; ++i) {
+        double ang = (double)pos * pow(theta, -2.0 * (double)i / (double)rope_dim);
+        double c = cos(ang), sn = sin(ang);
+        double x0 = v[2 * i], x1 = v[2 * i + 1];
+        v[2 * i] = x0 * c - x1 * sn;
+        v[2 * i + 1] = x0 * sn + x1 * c;
+    }
+}
+
+int dsa_oracle_indexer_project(int32_t nt, int32_t hidden, int32_t q_lora_rank,
+                               int32_t h_idx, int32_t d_idx, int32_t rope_dim,
+                               const uint16_t *x, const uint16_t *q_lora,
+                               const uint16_t *w_qb, const uint16_t *w_k,
+                               const uint16_t *w_proj, const float *ln_gamma,
+                               const float *ln_beta, double ln_eps,
+                               const int32_t *positions, double rope_theta,
+                               double *q_f, double *k_f, double *w_f,
+                               uint8_t *q_code, float *q_scale,
+                               uint8_t *k_code, float *k_scale,
+                               uint16_t *w_bf16, int32_t nthreads)
+{
+    if (nt < 0 || hidden <= 0 || q_lora_rank <= 0 || h_idx <= 0 || d_idx <= 0) return -1;
+    if (rope_dim < 0 || rope_dim > d_idx || (rope_dim & 1)) return -1;
+    set_threads(nthreads);
+    int rc = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int32_t t = 0; t < nt; ++t) {
+        double *qv = (double *)malloc((size_t)h_idx * d_idx * sizeof(double));
+        double *kv = (double *)malloc((size_t)d_idx * sizeof(double));
+        if (!qv || !kv) {
+            free(qv);
+            free(kv);
+            rc = -2;
+            continue;
+        }
+        /* q^I = W_qb . q_lora, one output row at a time */
+        for (int64_t o = 0; o < (int64_t)h_idx * d_idx; ++o) {
+            double acc = 0.0;
+            for (int32_t r = 0; r < q_lora_rank; ++r)
+                acc += bf(w_qb, o * q_lora_rank + r) * bf(q_lora, (int64_t)t * q_lora_rank + r);
+            qv[o] = acc;
+        }
+        /* k^I = LayerNorm(W_k . x) */
+        for (int32_t o = 0; o < d_idx; ++o) {
+            double acc = 0.0;
+            for (int32_t i = 0; i < hidden; ++i)
+                acc += bf(w_k, (int64_t)o * hidden + i) * bf(x, (int64_t)t * hidden + i);
+            kv[o] = acc;
+        }
+        double mean = 0.0, var = 0.0;
+        for (int32_t o = 0; o < d_idx; ++o) mean += kv[o];
+        mean /= d_idx;
+        for (int32_t o = 0; o < d_idx; ++o) var += (kv[o] - mean) * (kv[o] - mean);
+        var /= d_idx;
+        for (int32_t o = 0; o < d_idx; ++o)
+            kv[o] = (kv[o] - mean) / sqrt(var + ln_eps) * (double)ln_gamma[o] + (double)ln_beta[o];
+        /* RoPE on the first rope_dim dims of every q head and of k */
+        for (int32_t j = 0; j < h_idx; ++j) rope_rotate(qv + (int64_t)j * d_idx, rope_dim, positions[t], rope_theta);
+        rope_rotate(kv, rope_dim, positions[t], rope_theta);
+        /* k: one power-of-two scale per token */
+        double kmax = 0.0;
+        for (int32_t o = 0; o < d_idx; ++o) kmax = fmax(kmax, fabs(kv[o]));
+        double ks = pow2_scale(kmax);
+        for (int32_t o = 0; o < d_idx; ++o) {
+            if (k_f) k_f[(int64_t)t * d_idx + o] = kv[o];
+            if (k_code) k_code[(int64_t)t * d_idx + o] = dsa_oracle_f64_to_e4m3(kv[o] / ks);
+        }
+        if (k_scale) k_scale[t] = (float)ks;
+        /* q: one power-of-two scale per (token, head); w folds it */
+        for (int32_t j = 0; j < h_idx; ++j) {
+            const double *qh = qv + (int64_t)j * d_idx;
+            double qmax = 0.0;
+            for (int32_t o = 0; o < d_idx; ++o) qmax = fmax(qmax, fabs(qh[o]));
+            double qs = pow2_scale(qmax);
+            double wp = 0.0;
+            for (int32_t i = 0; i < hidden; ++i)
+                wp += bf(w_proj, (int64_t)j * hidden + i) * bf(x, (int64_t)t * hidden + i);
+            double wv = wp / sqrt((double)h_idx) / sqrt((double)d_idx) * qs;
+            int64_t tj = (int64_t)t * h_idx + j;
+            if (w_f) w_f[tj] = wv;
+            if (w_bf16) w_bf16[tj] = f64_to_bf16_rne(wv);
+            if (q_scale) q_scale[tj] = (float)qs;
+            for (int32_t o = 0; o < d_idx; ++o) {
+                if (q_f) q_f[tj * d_idx + o] = qh[o];
+                if (q_code) q_code[tj * d_idx + o] = dsa_oracle_f64_to_e4m3(qh[o] / qs);
+            }
+        }
+        free(qv);
+        free(kv);
+    }
+    return rc;
 }
