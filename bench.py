@@ -3,25 +3,36 @@
 MLA attention over a 16 x 128K-context batch (one query per sequence).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload long_decode_16x128k|batched_decode_64x32k|paged_mtp_decode_128seq]
+                    [--workload NAME] [--ragged] [--nseq S] [--L CTX]
+                    [--no-cpu-baseline] [--no-e2e] [--clocks-csv PATH]
+    python bench.py --profile [--workload NAME] [--nseq S] [--L CTX] [--warmup W] [--steps K]
+
+Workloads: long_decode_16x128k (default: the headline), batched_decode_64x32k,
+paged_mtp_decode_128seq, causal_prefill_16k, tiny_decode_4k; --ragged draws
+the long-decode context lengths from U[1024, L] (sequence 0 at 2048 and 1 at
+2049); --nseq / --L resize a workload.
 
 One step = one dsa_forward call over the batch (fused FP8 indexer + exact TopK,
 sparse MLA, split combine), inputs resident in HBM.  Every timed step is
 bracketed by CUDA events on the launching stream.  No L2 flush runs between
-steps: each step streams the whole index-K cache (268 MB at 16 x 128K, more
-than twice the 126 MB L2) through L2, which evicts the previous step's data.
-(A flush by writing a buffer would leave ~126 MB of dirty lines that the next
-step pays to write back.)  The attention-only stage timing, whose inputs are
-smaller than L2, evicts L2 before each call by reading a 256 MiB buffer,
-outside the timed interval.  With
-N > 1 (torchrun) every rank runs its own replica batch (the path has no
-exchange step) and the time is the max over ranks.
+steps of the decode workloads: each step streams the whole index-K cache (268
+MB at 16 x 128K, more than twice the 126 MB L2) through L2, which evicts the
+previous step's data.  (A flush by writing a buffer would leave ~126 MB of
+dirty lines that the next step pays to write back.)  Smaller workloads, and
+the attention-only stage, evict L2 before each timed call by reading a 256 MiB
+buffer, outside the timed interval.  With N > 1 (torchrun) every rank runs its
+own replica batch (the path has no exchange step) and the time is the max over
+ranks.
 
 Printed: one JSON line (rank 0).  `roofline` is for the dominant kernel (the
-fused indexer), timed alone over the same workload; `e2e` repeats the step
+fused indexer), timed alone over the same workload; `stages` gives each
+stage's time and its fraction of the binding roofline; `e2e` repeats the step
 through the C ABI from pinned host buffers (query-side inputs in, outputs
 out; the caches are resident state); `cpu_baseline` is the fp64 oracle timed
-on a bounded sample on this host.
+on a bounded sample on this host, on all cores and on one.
+
+--profile runs warm-up + K forward steps with no timing and checks the
+device status: the command the ncu captures run.
 """
 from __future__ import annotations
 
@@ -44,14 +55,16 @@ from long_context_decode_indexer_b200.batch import upload, workspace  # noqa: E4
 from long_context_decode_indexer_b200.synth import CONFIGS, make_inputs  # noqa: E402
 
 METRIC = "DSA decode queries/s at 128K ctx (indexer+TopK+sparse MLA); % of HBM/TC roofline"
-WORKLOADS = {c["name"]: cid for cid, c in CONFIGS.items() if c["kind"] in ("decode", "paged2")}
+WORKLOADS = {c["name"]: cid for cid, c in CONFIGS.items()}
 DEFAULT_WORKLOAD = CONFIGS[3]["name"]
 L2_BYTES = 126 * 1024 * 1024
+STAGE_ITERS = 200  # iterations of each stage-alone timing loop (more clock samples)
 
 
-# DRAM traffic of the fused indexer from one ncu capture (see
-# profiles/k1_indexer_long_decode_16x96k.md): read + write bytes per scored
-# position, valid only while the kernel sources hash to the captured build.
+# DRAM traffic of the fused indexer from one ncu capture of the 16 x 98304
+# decode case (dram__bytes_read.sum + dram__bytes_write.sum per launch over
+# the scored positions), valid only while the kernel sources hash to the
+# captured build; the capture is summarised under profiles/.
 K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
               "long_context_decode_indexer_b200/csrc/select.cuh",
               "long_context_decode_indexer_b200/csrc/ptx.cuh",
@@ -59,26 +72,32 @@ K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
 K1_PROFILED = {"sha256_16": "8a4b7d790e67b55e", "bytes_per_position": 131.10498046875}
 
 
-def k1_traffic(inp):
+def k1_sources_hash() -> str:
     import hashlib
     h = hashlib.sha256()
     for f in K1_SOURCES:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
-    if h.hexdigest()[:16] != K1_PROFILED["sha256_16"]:
+    return h.hexdigest()[:16]
+
+
+def k1_traffic(inp):
+    if k1_sources_hash() != K1_PROFILED["sha256_16"]:
         return None
     n = inp.q_n.astype(np.int64)
     return float(K1_PROFILED["bytes_per_position"] * n[n > inp.topk].sum())
 
 
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+        return (float(d["hbm_gbs"]), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 # ----------------------------------------------------------------- clocks
@@ -178,6 +197,20 @@ def dist_init(backend: str = "nccl"):
     return world, rank, local
 
 
+def workload_inputs(args, seed_offset: int = 0):
+    """The workload's seeded batch (resized by --nseq / --L, ragged lengths
+    with --ragged)."""
+    cid = WORKLOADS[args.workload]
+    kw = {}
+    if getattr(args, "nseq", None) is not None and CONFIGS[cid]["kind"] != "prefill":
+        kw["nseq"] = args.nseq
+    if getattr(args, "L", None) is not None:
+        kw["L"] = args.L
+    if getattr(args, "ragged", False):
+        kw["ragged"] = True
+    return make_inputs(cid, seed_offset=seed_offset, **kw)
+
+
 def replica_inputs(cid: int, rank: int):
     """Each rank runs its own replica batch (the path has no exchange step):
     the same workload shape, its own seeded draw."""
@@ -206,29 +239,46 @@ def job_rate(units_per_rank: int, steps: int, world: int, t_max: float) -> float
     return units_per_rank * steps * world / t_max
 
 
-def workload_config(inp, world):
+def workload_name(inp, ragged=False):
+    return inp.name + ("_ragged" if ragged else "")
+
+
+def workload_config(inp, world, ragged=False, flush=False):
     """The `config` object of the JSON line (the same for both arms)."""
-    return {"workload": inp.name, "nq": inp.nq, "context": int(inp.q_n.max()),
-            "topk": inp.topk, "h_idx": inp.h_idx, "d_idx": inp.d_idx, "heads": inp.h,
-            "d_qk": inp.d_qk, "d_v": inp.d_v, "paged": inp.page_table is not None,
-            "parallelism": "replicas" if world > 1 else "single",
-            "l2": "inputs larger than L2: each step streams the %.0f MB index-K cache; "
-                  "no flush between steps (attention-only stage: L2 evicted by a 256 MiB "
-                  "read before each call)" % (algorithmic_bytes(inp)["indexer"] / 1e6)}
+    l2 = ("inputs larger than L2: each step streams the %.0f MB index-K cache; no flush "
+          "between steps (attention-only stage: L2 evicted by a 256 MiB read before each call)"
+          % (algorithmic_bytes(inp)["indexer"] / 1e6)) if not flush else \
+         "L2 evicted by a 256 MiB read before every timed call (outside the timed interval)"
+    return {"workload": workload_name(inp, ragged), "nq": inp.nq, "context": int(inp.q_n.max()),
+            "context_min": int(inp.q_n.min()), "topk": inp.topk, "h_idx": inp.h_idx,
+            "d_idx": inp.d_idx, "heads": inp.h, "d_qk": inp.d_qk, "d_v": inp.d_v,
+            "queries_per_sequence": inp.q_per_seq, "paged": inp.page_table is not None,
+            "parallelism": "replicas" if world > 1 else "single", "l2": l2}
 
 
 def algorithmic_bytes(inp):
-    """Bytes the three steps must move at minimum (per batch)."""
+    """Bytes and FLOPs the three steps must move / compute at minimum (per
+    batch).  The index-K rows of a sequence are read once however many of
+    its queries score them; a query whose history fits in k reads none."""
     n = inp.q_n.astype(np.int64)
     k = inp.topk
     scored = n > k
-    kI = int(n[scored].sum()) * inp.d_idx                        # k^I rows streamed once
-    if inp.q_per_seq == 2:                                       # two queries share a stream
-        kI = int(np.maximum(n[0::2], n[1::2])[scored[0::2] | scored[1::2]].sum()) * inp.d_idx
-    idx_in = inp.nq * (inp.h_idx * inp.d_idx + inp.h_idx * 2)    # q^I + w
+    kI = 0
+    for s in range(inp.nseq):
+        m = (inp.q_seq == s) & scored
+        if m.any():
+            kI += int(n[m].max()) * inp.d_idx                    # rows streamed once per sequence
+    idx_in = int(scored.sum()) * (inp.h_idx * inp.d_idx + inp.h_idx * 2)   # q^I + w
     idx_out = inp.nq * k * 4                                     # selected positions
     sel = np.minimum(n, k)
-    gather = int(sel.sum()) * inp.d_qk * 2                       # latent rows
+    rows = 0
+    for s in range(inp.nseq):                                    # distinct latent rows per sequence
+        m = inp.q_seq == s
+        if m.any():
+            rows += int(sel[m].max()) if inp.kind != "prefill" else int(n[m].max())
+    if inp.kind != "prefill":
+        rows = int(sel.sum())                                    # every query gathers its own rows
+    gather = rows * inp.d_qk * 2
     att_io = inp.nq * inp.h * (inp.d_qk * 2 + inp.d_v * 2 + 4) + inp.nq * k * 4
     flops_idx = 2 * int(n[scored].sum()) * inp.h_idx * inp.d_idx
     flops_att = 2 * int(sel.sum()) * inp.h * (inp.d_qk + inp.d_v)
@@ -236,25 +286,50 @@ def algorithmic_bytes(inp):
                 flops_indexer=flops_idx, flops_attention=flops_att)
 
 
+def stage_fraction(bytes_, flops, t, hbm_gbs, tflops):
+    """max(t_bytes, t_flops) / t: the stage's fraction of its binding roofline."""
+    t_b = bytes_ / (hbm_gbs * 1e9)
+    t_f = flops / (tflops * 1e12) if flops else 0.0
+    return max(t_b, t_f) / t, ("hbm" if t_b >= t_f else "tensor")
+
+
+def count_our_launches(fn) -> int:
+    """Kernels of libdsa_b200 that one call of fn launches (torch profiler)."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            fn()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if str(e.device_type).endswith("CUDA")]
+        return sum(1 for nm in names if "dsa::" in nm)
+    except Exception:
+        return -1
+
+
 # -------------------------------------------------------------- our arm
 def run_ours(args, world, rank):
-    cid = WORKLOADS[args.workload]
     t_gen = time.time()
-    inp = replica_inputs(cid, rank)
+    inp = workload_inputs(args, seed_offset=rank * 101)
     db = upload(inp)
     torch.cuda.synchronize()
     gen_s = time.time() - t_gen
     p = db.params()
     kv = db.kvdesc()
     paged = db.page_table is not None
+    prefill = inp.kind == "prefill"
     st = torch.cuda.current_stream()
     ws = workspace(dsa.workspace_size(p, kv, dsa.OP_FORWARD))
     ws_idx = workspace(dsa.workspace_size(p, kv, dsa.OP_INDEXER_TOPK))
-    ws_mla = workspace(dsa.workspace_size(p, kv, dsa.OP_SPARSE_MLA_DECODE))
+    mla_op = dsa.OP_SPARSE_MLA_PREFILL if prefill else dsa.OP_SPARSE_MLA_DECODE
+    ws_mla = workspace(dsa.workspace_size(p, kv, mla_op))
+    mla_fn = dsa.sparse_mla_prefill if prefill else dsa.sparse_mla_decode
     out = torch.empty((inp.nq, inp.h, inp.d_v), dtype=torch.int16, device="cuda")
     lse = torch.empty((inp.nq, inp.h), dtype=torch.float32, device="cuda")
     idx = torch.empty((inp.nq, inp.topk), dtype=torch.int32, device="cuda")
     evict_buf = torch.ones(2 * L2_BYTES // 4, dtype=torch.int32, device="cuda")
+    alg = algorithmic_bytes(inp)
+    flush = alg["indexer"] < 2 * L2_BYTES   # the step's own stream does not evict L2
 
     def evict():
         # read (not write) a buffer twice the size of L2: evicts the cache
@@ -279,26 +354,129 @@ def run_ours(args, world, rank):
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in evs) / 1e3
 
+    if args.profile:
+        for _ in range(args.warmup + args.steps):
+            step()
+        status = dsa.check_status(ws)
+        print(json.dumps({"profile": workload_name(inp, args.ragged), "nq": inp.nq,
+                          "max_n": inp.max_n, "steps": args.warmup + args.steps,
+                          "device_status": status}))
+        return None, inp
+
     for _ in range(args.warmup):
         step()
     assert dsa.check_status(ws) == dsa.DSA_OK, dsa.last_error()
+    launches_per_step = count_our_launches(step)
     barrier(world)
     torch.cuda.synchronize()
+    stage_iters = max(args.steps, STAGE_ITERS)
     with ClockSampler(torch.cuda.current_device(), args.clocks_csv) as clk:
         clk.active = True
-        t_total = timed(step, args.steps)
+        t_total = timed(step, args.steps, before=evict if flush else None)
         torch.cuda.synchronize()
         barrier(world)
         # stage timings (same workload, same stream) for the roofline
         t_idx = timed(lambda: dsa.indexer_topk(p, kv, db.q_idx, db.w, db.kidx, db.k_scale, idx,
-                                               None, ws_idx, stream=st), args.steps)
-        t_mla = timed(lambda: dsa.sparse_mla_decode(p, kv, db.q, db.kv, db.kv_row_stride, idx,
-                                                    out, lse, ws_mla, stream=st), args.steps,
-                      before=evict)
+                                               None, ws_idx, stream=st), stage_iters,
+                      before=evict if flush else None)
+        t_mla = timed(lambda: mla_fn(p, kv, db.q, db.kv, db.kv_row_stride, idx, out, lse, ws_mla,
+                                     stream=st), stage_iters, before=evict)
     status = dsa.check_status(ws)
     t_max = max_over_ranks(t_total, world)
 
-    # end to end through the C ABI from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, world, inp, db, p, idx, out, lse, ws_idx, ws_mla, mla_fn, timed)
+    for w_ in (ws, ws_idx, ws_mla):
+        assert dsa.check_status(w_) == dsa.DSA_OK, dsa.last_error()
+
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    us_idx = t_idx / stage_iters * 1e6
+    us_mla = t_mla / stage_iters * 1e6
+    idx_gbs = alg["indexer"] / (us_idx * 1e-6) / 1e9
+    mla_gbs = alg["attention"] / (us_mla * 1e-6) / 1e9
+    mla_tflops = alg["flops_attention"] / (us_mla * 1e-6) / 1e12
+    idx_tflops = alg["flops_indexer"] / (us_idx * 1e-6) / 1e12
+    step_s = t_total / args.steps
+    step_gbs = (alg["indexer"] + alg["attention"]) / step_s / 1e9
+    mla_frac, mla_bound = stage_fraction(alg["attention"], alg["flops_attention"], us_mla * 1e-6,
+                                         hbm, bf16)
+    mla_frac_sus, _ = stage_fraction(alg["attention"], alg["flops_attention"], us_mla * 1e-6,
+                                     hbm, bf16_sus)
+    # FP8 dense peak: the recipe's nominal FP8 / bf16 ratio (2x) times the
+    # measured bf16 burst peak
+    fp8 = 2.0 * bf16
+    idx_frac, idx_bound = stage_fraction(alg["indexer"], alg["flops_indexer"], us_idx * 1e-6, hbm, fp8)
+    total_q = inp.nq * args.steps * world
+    qps = job_rate(inp.nq, args.steps, world, t_max)
+    if idx_bound == "hbm":
+        roof = {"bound": "hbm", "achieved": idx_gbs, "peak": hbm, "unit": "GB/s",
+                "frac": idx_gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": idx_tflops, "peak": fp8, "unit": "TFLOP/s",
+                "frac": idx_tflops / fp8}
+    roof.update({"traffic": k1_traffic(inp) if not prefill else None,
+                 "kernel": "k1_indexer (fused indexer + TopK)", "peak_source": peak_kind,
+                 "kernel_sources_sha16": k1_sources_hash()})
+    res = {
+        "metric": METRIC,
+        "value": qps,
+        "unit": "queries/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t_max / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3+bf16",
+        "data": "synthetic",
+        "impl": "ours",
+        "tokens_per_s": qps,
+        "config": workload_config(inp, world, args.ragged, flush),
+        "roofline": roof,
+        "stages": {
+            "indexer_topk_us": us_idx,
+            "indexer_topk_gbs": idx_gbs,
+            "indexer_topk_tflops_fp8": idx_tflops,
+            "indexer_topk_bound": idx_bound,
+            "indexer_topk_frac": idx_frac,
+            "indexer_topk_frac_nominal_8tbs": idx_gbs / 8000.0,
+            "sparse_mla_us": us_mla,
+            "sparse_mla_gbs": mla_gbs,
+            "sparse_mla_tflops": mla_tflops,
+            "sparse_mla_bound": mla_bound,
+            "sparse_mla_frac": mla_frac,
+            "sparse_mla_frac_sustained_bf16": mla_frac_sus,
+            "sparse_mla_frac_hbm": mla_gbs / hbm,
+            "sparse_mla_frac_bf16": mla_tflops / bf16,
+            "step_us": step_s * 1e6,
+            "step_gbs": step_gbs,
+            "step_frac_hbm": step_gbs / hbm,
+            "algorithmic_bytes_per_step": alg["indexer"] + alg["attention"],
+            "flops_per_step": alg["flops_indexer"] + alg["flops_attention"],
+            "fp8_peak_tflops": fp8,
+            "fp8_peak_source": "2 x measured bf16 burst (nominal FP8/bf16 ratio)",
+            "stage_iters": stage_iters,
+        },
+        "gpu_launches": launches_per_step * args.steps if launches_per_step >= 0 else None,
+        "gpu_launches_per_step": launches_per_step,
+        "device_status": status,
+        "input_gen_s": gen_s,
+        "clocks": clk.summary(),
+    }
+    if e2e is not None:
+        e2e["value"] = total_q / e2e.pop("t")
+        e2e["eager_value"] = total_q / e2e.pop("t_eager")
+        res["e2e"] = e2e
+    return res, inp
+
+
+def run_e2e(args, world, inp, db, p, idx, out, lse, ws_idx, ws_mla, mla_fn, timed):
+    """The step end to end through the C ABI from pinned host buffers: the
+    query-side inputs go up, the indices and the attention output come back,
+    every step (the caches are resident state)."""
+    st = torch.cuda.current_stream()
     h_qidx = torch.from_numpy(inp.q_idx).pin_memory()
     h_w = torch.from_numpy(inp.w.view(np.int16)).pin_memory()
     h_q = torch.from_numpy(inp.q.view(np.int16)).pin_memory()
@@ -319,9 +497,9 @@ def run_ours(args, world, rank):
 
     def e2e_step():
         # The same two stages through the public entry points (dsa_indexer_topk,
-        # then dsa_sparse_mla_decode, which is what dsa_forward runs), with the
-        # copies overlapped on a second stream: the 2.4 MB attention query goes
-        # up while the indexer runs, the indices come down while the attention
+        # then the sparse attention, which is what dsa_forward runs), with the
+        # copies overlapped on a second stream: the attention query goes up
+        # while the indexer runs, the indices come down while the attention
         # runs.  `cur` is the capture stream while a graph is recorded.
         cur = torch.cuda.current_stream()
         copy_stream.wait_stream(cur)                 # the previous step is done with d_q
@@ -334,7 +512,7 @@ def run_ours(args, world, rank):
         copy_stream.wait_stream(cur)                 # the indices are final
         with torch.cuda.stream(copy_stream):
             h_idx.copy_(idx, non_blocking=True)
-        dsa.sparse_mla_decode(p, kv_e, d_q, db.kv, db.kv_row_stride, idx, out, lse, ws_mla)
+        mla_fn(p, kv_e, d_q, db.kv, db.kv_row_stride, idx, out, lse, ws_mla)
         h_out.copy_(out, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
         cur.wait_stream(copy_stream)                 # join the copy stream
@@ -343,11 +521,11 @@ def run_ours(args, world, rank):
         e2e_step()
     torch.cuda.synchronize()
     barrier(world)
-    t_e2e_eager = max_over_ranks(timed(e2e_step, args.steps), world)
+    t_eager = max_over_ranks(timed(e2e_step, args.steps), world)
     # The same step recorded once as a CUDA graph (copies from the pinned
     # buffers, the two stages' launches, copies back, both streams) and
     # replayed: one host launch per step, as a decode loop would run it.
-    e2e_launch = "cuda_graph"
+    launch = "cuda_graph"
     try:
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
@@ -362,96 +540,60 @@ def run_ours(args, world, rank):
             graph.replay()
         torch.cuda.synchronize()
         barrier(world)
-        t_e2e = max_over_ranks(timed(graph.replay, args.steps), world)
+        t = max_over_ranks(timed(graph.replay, args.steps), world)
         del graph
     except RuntimeError as exc:  # capture refused: report the eager loop
         print("e2e graph capture failed (%s); reporting the eager loop" % exc, file=sys.stderr)
-        e2e_launch, t_e2e = "eager", t_e2e_eager
-    assert dsa.check_status(ws) == dsa.DSA_OK, dsa.last_error()
-    assert dsa.check_status(ws_idx) == dsa.DSA_OK, dsa.last_error()
-    assert dsa.check_status(ws_mla) == dsa.DSA_OK, dsa.last_error()
+        launch, t = "eager", t_eager
     torch.cuda.synchronize()
-    e2e_same = bool(torch.equal(h_out, ref_out.cpu()))  # host copy == device-resident result
-
-    alg = algorithmic_bytes(inp)
-    hbm, bf16, peak_kind = peaks()
-    idx_gbs = alg["indexer"] / (t_idx / args.steps) / 1e9
-    mla_gbs = alg["attention"] / (t_mla / args.steps) / 1e9
-    mla_tflops = alg["flops_attention"] / (t_mla / args.steps) / 1e12
-    step_gbs = (alg["indexer"] + alg["attention"]) / (t_total / args.steps) / 1e9
-    total_q = inp.nq * args.steps * world
-    qps = job_rate(inp.nq, args.steps, world, t_max)
-    res = {
-        "metric": METRIC,
-        "value": qps,
-        "unit": "queries/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": t_max / args.steps * 1e3,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "e4m3+bf16",
-        "data": "synthetic",
-        "impl": "ours",
-        "tokens_per_s": qps,
-        "config": workload_config(inp, world),
-        "roofline": {"bound": "hbm", "achieved": idx_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": idx_gbs / hbm, "traffic": k1_traffic(inp),
-                     "kernel": "k1_indexer (fused indexer + TopK)",
-                     "peak_source": peak_kind},
-        "stages": {
-            "indexer_topk_us": t_idx / args.steps * 1e6,
-            "indexer_topk_gbs": idx_gbs,
-            "indexer_topk_frac_nominal_8tbs": idx_gbs / 8000.0,
-            "sparse_mla_us": t_mla / args.steps * 1e6,
-            "sparse_mla_gbs": mla_gbs,
-            "sparse_mla_tflops": mla_tflops,
-            "sparse_mla_frac_hbm": mla_gbs / hbm,
-            "sparse_mla_frac_bf16": mla_tflops / bf16,
-            "step_gbs": step_gbs,
-            "step_frac_hbm": step_gbs / hbm,
-            "algorithmic_bytes_per_step": alg["indexer"] + alg["attention"],
-        },
-        "e2e": {"value": total_q / t_e2e, "unit": "queries/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "launch": e2e_launch,
-                "copies": "overlapped with the kernels on a second stream",
-                "eager_value": total_q / t_e2e_eager, "matches_device_result": e2e_same},
-        "gpu_launches": 3 * args.steps,
-        "device_status": status,
-        "input_gen_s": gen_s,
-        "clocks": clk.summary(),
-    }
-    return res, inp
+    same = bool(torch.equal(h_out, ref_out.cpu()))  # host copy == device-resident result
+    return {"t": t, "t_eager": t_eager, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "launch": launch,
+            "copies": "overlapped with the kernels on a second stream",
+            "matches_device_result": same}
 
 
 # --------------------------------------------------------- oracle timing
-def oracle_sample(inp, n_queries, nthreads=0):
-    """Time the fp64 oracle (score -> TopK -> attention) on the first
-    n_queries queries of the batch; returns (queries/s, cores, seconds)."""
+def _oracle_queries(inp, sel, nthreads):
     import oracle
-    sel = np.arange(min(n_queries, inp.nq))
     t0 = time.time()
     oracle.forward(inp.q_idx[sel], inp.w[sel], inp.kidx, inp.q[sel], inp.kv, inp.q_seq[sel],
                    inp.q_n[sel], k=inp.topk, scale=inp.scale, seq_row0=inp.seq_row0,
-                   page_table=inp.page_table, page_size=inp.page_size, nthreads=nthreads)
-    dt = time.time() - t0
-    return len(sel) / dt, oracle.max_threads(), dt
+                   page_table=inp.page_table, page_size=inp.page_size, k_scale=inp.k_scale,
+                   nthreads=nthreads)
+    return time.time() - t0
 
 
-def cpu_baseline(inp, target_s=15.0):
-    """Bounded sample: one query first, then as many more as ~target_s allows."""
-    qps1, cores, dt1 = oracle_sample(inp, 1)
+def oracle_sample(inp, n_queries, nthreads=0, seed=0):
+    """Time the fp64 oracle (score -> TopK -> attention) on n_queries queries
+    of the batch (the first ones; a seeded random subset for a prefill, whose
+    queries differ in length); returns (queries/s, threads, seconds, sel)."""
+    import oracle
+    n_queries = min(n_queries, inp.nq)
+    if inp.kind == "prefill":
+        sel = np.sort(np.random.default_rng(1000 + seed).choice(inp.nq, n_queries, replace=False))
+    else:
+        sel = np.arange(n_queries)
+    dt = _oracle_queries(inp, sel, nthreads)
+    threads = oracle.max_threads() if nthreads == 0 else nthreads
+    return len(sel) / dt, threads, dt, sel
+
+
+def cpu_baseline(inp, target_s=12.0):
+    """Bounded samples of the oracle on this host: as many queries as ~target_s
+    allows on all cores, and one query on one core."""
+    qps1, cores, dt1, _ = oracle_sample(inp, 1)
     n = max(1, min(inp.nq, int(target_s / max(dt1, 1e-3))))
     if n > 1:
-        qps, cores, dt = oracle_sample(inp, n)
+        qps, cores, dt, sel = oracle_sample(inp, n)
     else:
         qps, dt = qps1, dt1
+    qps_1c, _, dt_1c, _ = oracle_sample(inp, 1, nthreads=1)
+    kind = "a seeded random subset" if inp.kind == "prefill" else "the first"
     return {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
-            "sample": "%d of %d queries of %s (full context), fp64 C oracle, %.1f s"
-                      % (n, inp.nq, inp.name, dt),
-            "cpu": cpu_model()}
+            "sample": "%s %d of %d queries of %s (full context), fp64 C oracle, %.1f s on %d threads; "
+                      "1 query on 1 thread: %.1f s" % (kind, n, inp.nq, inp.name, dt, cores, dt_1c),
+            "value_1core": qps_1c, "cpu": cpu_model()}
 
 
 def cpu_model() -> str:
@@ -466,18 +608,19 @@ def cpu_model() -> str:
 
 
 def run_reference(args, world, rank):
+    """The oracle as the reference arm: rank 0 alone; every step is a bounded
+    sample (one query of the workload)."""
     if rank != 0:
         return None
-    cid = WORKLOADS[args.workload]
-    inp = make_inputs(cid)
+    inp = workload_inputs(args)
     import oracle
     oracle.build()
-    # each "step" is a bounded sample: one query of the batch
     for _ in range(min(args.warmup, 1)):
         oracle_sample(inp, 1)
     times = []
-    for _ in range(args.steps):
-        _, cores, dt = oracle_sample(inp, 1)
+    cores = 0
+    for i in range(args.steps):
+        _, cores, dt, _ = oracle_sample(inp, 1, seed=i)
         times.append(dt)
     qps = args.steps / sum(times)
     return {
@@ -485,7 +628,7 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sum(times) / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
-        "config": workload_config(inp, world),
+        "config": workload_config(inp, world, getattr(args, "ragged", False)),
         "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": cores, "kind": "oracle",
                          "sample": "1 query of %s per step (full context), fp64 C oracle"
                                    % inp.name},
@@ -494,18 +637,31 @@ def run_reference(args, world, rank):
     }
 
 
-def main():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--ragged", action="store_true",
+                    help="decode context lengths ~ U[1024, L] (sequence 0 at 2048, 1 at 2049)")
+    ap.add_argument("--nseq", type=int, default=None, help="resize: number of sequences")
+    ap.add_argument("--L", type=int, default=None, help="resize: context length (median for paged)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="run warm-up + steps forward calls untimed (for profiler captures)")
     ap.add_argument("--clocks-csv", default=None,
                     help="also record nvidia-smi clock samples (CSV) during the timed loops")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+    args = ap.parse_args(argv)
+    if not args.profile:
+        args.warmup = max(args.warmup, 3)
+    return args
+
+
+def main():
+    args = parse_args()
     world, rank, _ = dist_init() if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
     if args.impl == "reference":
@@ -514,7 +670,7 @@ def main():
             print(json.dumps(res))
         return
     res, inp = run_ours(args, world, rank)
-    if rank == 0:
+    if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(res))

@@ -228,8 +228,10 @@ int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  *     dsa_workspace_size(DSA_OP_INDEXER_TOPK) gives a shape's need.
  *   - The call allocates nothing (no cudaMalloc, no allocating library
  *     call).  The first call on each device resolves the array's device
- *     address (cudaGetSymbolAddress); make that first call outside any
- *     stream capture.
+ *     address (cudaGetSymbolAddress) and keeps it for the life of the
+ *     process; make that first call outside any stream capture.  Do not use
+ *     this entry point after cudaDeviceReset (or anything else that tears
+ *     down the device's primary context): the kept address would be stale.
  *   - All calls share the array and it keeps the last call's contents: the
  *     call clears what must start at zero itself, but calls whose work
  *     overlaps on the GPU (other streams, other threads) race; serialise them.

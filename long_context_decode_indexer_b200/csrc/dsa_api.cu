@@ -214,7 +214,7 @@ MlaPlan plan_mla(const dsa_params *p) {
     if (m.splits == 1) {
         m.wave = p->nq;
     } else {
-        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv * 2 + 4);
+        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv * 2 + 4 + 8);
         size_t w = kPartialBudget / per_q;
         if (w < 1) w = 1;
         m.wave = p->nq < static_cast<int>(w) ? p->nq : static_cast<int>(w);
@@ -224,7 +224,7 @@ MlaPlan plan_mla(const dsa_params *p) {
 
 // -------------------------------------------------------------- workspace
 struct WsLayout {
-    size_t status, ghist, gtot, cand, cand_cnt, done, idx, part_o, part_lse, total;
+    size_t status, ghist, gtot, cand, cand_cnt, done, idx, part_o, part_lse, part_scale, total;
     size_t zero_begin, zero_end;  // cleared at the start of every call
 };
 
@@ -247,12 +247,14 @@ size_t indexer_ws(const dsa_params *p, const IndexerPlan &pl, int mode, size_t o
 }
 
 size_t mla_ws(const dsa_params *p, const MlaPlan &m, size_t off, WsLayout &w) {
-    w.part_o = w.part_lse = off;
+    w.part_o = w.part_lse = w.part_scale = off;
     if (m.splits <= 1) return off;
     w.part_o = off;
     off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * dsa::kDv * 2, 256);  // fp16
     w.part_lse = off;
     off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 4, 256);
+    w.part_scale = off;
+    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 2 * 4, 256);
     return off;
 }
 
@@ -387,14 +389,11 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
             int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
             const WsLayout &wl, const MlaPlan &m, cudaStream_t st) {
     if (p->nq == 0) return DSA_OK;
-    CUtensorMap qmap, kvmap;
+    CUtensorMap qmap;
     const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
     int rc = make_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dsa::kDqk,
                          static_cast<uint64_t>(p->nq) * p->h, dsa::kDqk * 2, 64, hbox,
                          CU_TENSOR_MAP_SWIZZLE_128B);
-    if (rc) return rc;
-    rc = make_map_2d(&kvmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, kv_cache, dsa::kDqk, kv->cache_rows,
-                     static_cast<uint64_t>(kv_row_stride) * 2, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     dsa::MlaParams a;
     memset(&a, 0, sizeof a);
@@ -419,11 +418,12 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.lse = lse;
     a.part_o = m.splits > 1 ? at<uint16_t>(ws, wl.part_o) : nullptr;
     a.part_lse = m.splits > 1 ? at<float>(ws, wl.part_lse) : nullptr;
+    a.part_scale = m.splits > 1 ? at<float>(ws, wl.part_scale) : nullptr;
     a.status = at<int>(ws, wl.status);
     for (int q0 = 0; q0 < p->nq; q0 += m.wave) {
         const int nw = (p->nq - q0) < m.wave ? (p->nq - q0) : m.wave;
         a.q0 = q0;
-        cudaError_t e = dsa::launch_sparse_mla(qmap, kvmap, a, nw, st);
+        cudaError_t e = dsa::launch_sparse_mla(qmap, a, nw, st);
         if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
         e = dsa::launch_mla_combine(a, nw, st);
         if (e != cudaSuccess) return cuda_fail(e, "split combine launch");

@@ -145,8 +145,9 @@ struct MlaParams {
     // outputs
     uint16_t *out;       // [nq, h, d_v] bf16
     float *lse;          // [nq, h]
-    uint16_t *part_o;    // [wave_q, splits, 128, d_v] normalised partial outputs (fp16 bits)
+    uint16_t *part_o;    // [wave_q, splits, 128, d_v] normalised partial outputs / part_scale (fp16 bits)
     float *part_lse;     // [wave_q, splits, 128]
+    float *part_scale;   // [wave_q, splits, 128, 2] power of two of each half row of part_o
     int *status;
 };
 
@@ -174,8 +175,7 @@ __host__ __device__ inline MlaLayout mla_layout() {
     return L;
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap, const MlaParams &a,
-                              int nq_wave, cudaStream_t st);
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st);
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st);
 
 }  // namespace dsa

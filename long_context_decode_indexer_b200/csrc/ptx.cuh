@@ -1,5 +1,5 @@
 // ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarrier, TMA (tiled and
-// gather4), tcgen05 (TMEM alloc, MMA, commit, loads, fences) and the shared
+// bulk), tcgen05 (TMEM alloc, MMA, commit, loads, fences) and the shared
 // memory matrix descriptors the 5th-generation tensor cores read.
 #pragma once
 
@@ -97,18 +97,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
-        : "memory");
-}
-// Row gather: four rows r0..r3 (each one box row high) at column c0, written
-// as four consecutive box rows of shared memory.
-__device__ __forceinline__ void tma_gather4(void *dst, const CUtensorMap *map, uint64_t *bar,
-                                            int32_t c0, int32_t r0, int32_t r1, int32_t r2,
-                                            int32_t r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-        "r"(smem_u32(bar))
         : "memory");
 }
 // Contiguous global -> shared copy by the TMA engine (both addresses 16-byte

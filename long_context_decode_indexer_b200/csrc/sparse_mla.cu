@@ -31,10 +31,13 @@
 // Epilogue: the softmax warps write columns 0..255 of O / l, the gather warps
 // columns 256..511; each thread moves its head's row from TMEM to a staging
 // row in shared memory and issues one 512-byte bulk store.  A split writes
-// O / l in fp16 (its values are convex combinations of bf16 rows, so fp16's
-// range suffices and its rounding, 2^-12 relative, is far below the bf16
-// output's) and its log-sum-exp; the combine kernel merges splits by their
-// log-sum-exp.  With one split the CTA writes the final output.
+// O / l as fp16 values times a power-of-two scale per (split, head, half
+// row), chosen from that half row's largest magnitude: the values keep
+// fp16's precision (2^-12 relative, far below the bf16 output's rounding)
+// over the whole bf16 range of the latent cache, which plain fp16 (max
+// 65504, subnormal below 6e-5) would not.  Each split also writes its
+// log-sum-exp; the combine kernel merges splits by their log-sum-exp.  With
+// one split the CTA writes the final output.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -159,11 +162,37 @@ __device__ bool gather_pass1(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int
 // registers -> this thread's staging row in shared memory (`srow`, 512 bytes,
 // rows kEpiPitch apart so that the 16-byte writes of a warp spread over the
 // banks) -> one 512-byte bulk store into the row of the output (bf16) or of
-// the split partials (fp16).  The TMEM loads are warp-collective: every lane
-// runs them; only the store is skipped for padding heads (hrow >= h).  The
-// caller waits for the bulk store (bulk_wait_read) before the CTA exits.
+// the split partials (fp16 times 2^e, e from the half row's largest
+// magnitude m: m * 2^-e lies in [2^14, 2^15), below fp16's 65504).  The TMEM
+// loads are warp-collective: every lane runs them; only the stores are
+// skipped for padding heads (hrow >= h).  The caller waits for the bulk
+// store (bulk_wait_read) before the CTA exits.
 __device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, int q, int wq, int sp,
                              float inv_l, int c_begin, uint8_t *srow) {
+    const bool partial = a.splits > 1;
+    float mul = inv_l;
+    if (partial) {
+        float mx = 0.f;
+        for (int c1 = c_begin; c1 < c_begin + 256; c1 += 64) {
+            uint32_t v2[2][32];
+            tmem_ld32(lane_addr + c1, v2[0]);
+            tmem_ld32(lane_addr + c1 + 32, v2[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(v2[0][j])), fabsf(__uint_as_float(v2[1][j]))));
+        }
+        mx *= inv_l;
+        // exponent of mx minus 14 (0 for an all-zero row); a subnormal or
+        // tiny mx is clamped (its values then stay below 2^14, still exact
+        // enough), so that both 2^-e and 2^e are normal floats
+        int e = mx > 0.f ? static_cast<int>((__float_as_uint(mx) >> 23) & 0xFFu) - 127 - 14 : 0;
+        e = min(max(e, -100), 113);
+        mul = inv_l * __int_as_float((127 - e) << 23);
+        if (hrow < a.h)
+            a.part_scale[((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * 2 + (c_begin >> 8)] =
+                __int_as_float((127 + e) << 23);
+    }
     for (int c1 = c_begin; c1 < c_begin + 256; c1 += 64) {
         uint32_t v2[2][32];
         tmem_ld32(lane_addr + c1, v2[0]);
@@ -175,15 +204,15 @@ __device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, i
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float x0 = __uint_as_float(u[2 * e]) * inv_l, x1 = __uint_as_float(u[2 * e + 1]) * inv_l;
-                w[e] = a.splits == 1 ? pack_bf16x2(x0, x1) : pack_half2(x0, x1);
+                const float x0 = __uint_as_float(u[2 * e]) * mul, x1 = __uint_as_float(u[2 * e + 1]) * mul;
+                w[e] = partial ? pack_half2(x0, x1) : pack_bf16x2(x0, x1);
             }
             *reinterpret_cast<uint4 *>(srow + (c1 - c_begin) * 2 + g * 16) = make_uint4(w[0], w[1], w[2], w[3]);
         }
     }
     fence_proxy_async_smem();  // the staging row is read by the bulk copy
     if (hrow < a.h) {
-        uint16_t *dst = a.splits == 1
+        uint16_t *dst = !partial
                             ? a.out + (static_cast<int64_t>(q) * a.h + hrow) * kDv
                             : a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
         bulk_store(dst + c_begin, srow, 512);
@@ -194,8 +223,7 @@ __device__ void store_output(const MlaParams &a, uint32_t lane_addr, int hrow, i
 }  // namespace
 
 __global__ void __launch_bounds__(kMlaThreads, 1)
-    k3_sparse_mla(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kvmap,
-                  const MlaParams a) {
+    k3_sparse_mla(const __grid_constant__ CUtensorMap qmap, const MlaParams a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     const MlaLayout L = mla_layout();
@@ -502,9 +530,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int c0 = 0; c0 < kDv; c0 += 8) *reinterpret_cast<uint4 *>(o + c0) = make_uint4(0, 0, 0, 0);
                 a.lse[static_cast<int64_t>(q) * a.h + hrow] = -INFINITY;
             } else {
-                uint16_t *o = a.part_o + ((static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow) * kDv;
+                const int64_t row = (static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow;
+                uint16_t *o = a.part_o + row * kDv;
                 for (int c0 = 0; c0 < kDv; c0 += 8) *reinterpret_cast<uint4 *>(o + c0) = make_uint4(0, 0, 0, 0);
-                a.part_lse[(static_cast<int64_t>(wq) * a.splits + sp) * 128 + hrow] = -INFINITY;
+                a.part_lse[row] = -INFINITY;
+                a.part_scale[row * 2] = 1.f;
+                a.part_scale[row * 2 + 1] = 1.f;
             }
         }
     }
@@ -517,7 +548,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
 }
 
 // Merge the splits of one (query, head): out = sum_s w_s o_s / sum_s w_s with
-// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  One warp covers 256
+// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  A split's stored
+// half row is o_s * 2^-e_s (fp16), so it enters with the weight w_s * 2^e_s.  One warp covers 256
 // value columns of one head (8 per lane, 16-byte loads and stores), so a
 // head takes two warps and a 128-thread CTA two heads.  Every warp reads the
 // head's split log-sum-exps itself (lane s holds split s; splits <= 32) and
@@ -533,10 +565,12 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_s
     const int64_t row0 = static_cast<int64_t>(wq) * a.splits * 128 + hh;  // split s: row0 + 128 s
     const int d = (warp & 1) * 256 + lane * 8;
     const float ls = lane < a.splits ? a.part_lse[row0 + 128 * lane] : -INFINITY;
+    const float sc = lane < a.splits ? a.part_scale[(row0 + 128 * lane) * 2 + (warp & 1)] : 0.f;
     float mx = ls;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     const float w = (mx == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - mx);
+    const float wsc = w > 0.f ? w * sc : 0.f;  // weight of the stored (scaled) values
     float tot = w;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
@@ -556,7 +590,7 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_s
                          : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-            const float wgt = __shfl_sync(0xffffffffu, w, (s0 + u) & 31);
+            const float wgt = __shfl_sync(0xffffffffu, wsc, (s0 + u) & 31);
             const uint32_t r4[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -597,8 +631,7 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_
     return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap, const MlaParams &a,
-                              int nq_wave, cudaStream_t st) {
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st) {
     const MlaLayout L = mla_layout();
     const size_t smem = smem_for_tmem(L.total, 512);
     cudaError_t e = cudaFuncSetAttribute(k3_sparse_mla, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -606,7 +639,7 @@ cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const CUtensorMap &kvmap,
     if (e != cudaSuccess) return e;
     const int grid = nq_wave * a.splits;
     if (grid == 0) return cudaSuccess;
-    return launch_pdl(k3_sparse_mla, grid, kMlaThreads, smem, st, qmap, kvmap, a);
+    return launch_pdl(k3_sparse_mla, grid, kMlaThreads, smem, st, qmap, a);
 }
 
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st) {

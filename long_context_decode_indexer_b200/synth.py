@@ -9,7 +9,7 @@ sides never have to agree on a quantisation step.
 Every tensor comes from its own PCG64 stream seeded by
 ``SeedSequence([1000 + config_id + seed_offset, stream])`` with these streams:
   0 context lengths, 1 page permutation, 2 q^I, 3 w, 4 k^I, 5 heavy-tail rows,
-  6 q (attention query), 7 latent KV.
+  6 q (attention query), 7 latent KV, 8 per-row key scales.
 Encodings: e4m3 via torch's float8_e4m3fn cast after clamping to +-448 (round
 to nearest even, saturating); bf16 via torch's round-to-nearest-even cast.
 """
@@ -110,11 +110,43 @@ def _normal_bf16(rng: np.random.Generator, shape, chunk: int = 1 << 24) -> np.nd
     return out.reshape(shape)
 
 
+def context_lengths(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = None,
+                    L: Optional[int] = None, ragged: bool = False,
+                    lengths: Optional[np.ndarray] = None) -> np.ndarray:
+    """Context length of every sequence of workload ``config_id`` (stream 0).
+
+    decode : L for every sequence; ragged: U[1024, L] with sequence 0 at 2048
+             and sequence 1 at 2049 (the short-history boundary).
+    paged2 : round(exp(ln L + N(0,1))) clipped to [512, 131071] (the
+             speculative token then sees at most 131072 positions).
+    prefill: the one sequence of L tokens.
+    """
+    c = CONFIGS[config_id]
+    kind = c["kind"]
+    nseq = c["nseq"] if nseq is None else int(nseq)
+    L = c["L"] if L is None else int(L)
+    r_len = _rng(config_id, seed_offset, 0)
+    if lengths is not None:
+        return np.asarray(lengths, np.int64).copy()
+    if kind == "paged2":
+        z = r_len.standard_normal(nseq)
+        return np.clip(np.round(np.exp(math.log(L) + 1.0 * z)), 512, 131071).astype(np.int64)
+    if ragged:
+        seq_ctx = r_len.integers(1024, L, size=nseq, endpoint=True).astype(np.int64)
+        if nseq > 0:
+            seq_ctx[0] = min(2048, L)
+        if nseq > 1:
+            seq_ctx[1] = min(2049, L)
+        return seq_ctx
+    return np.full(nseq, L, np.int64)
+
+
 def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = None,
                 L: Optional[int] = None, ragged: bool = False, paged: Optional[bool] = None,
                 lengths: Optional[np.ndarray] = None, with_k_scale: bool = False,
                 topk: Optional[int] = None, h: Optional[int] = None,
-                h_idx: Optional[int] = None, d_idx: Optional[int] = None) -> Inputs:
+                h_idx: Optional[int] = None, d_idx: Optional[int] = None,
+                with_attention: bool = True) -> Inputs:
     """Inputs of workload ``config_id`` (1..5), optionally resized for tests.
 
     decode  : one query per sequence; query n = L (rows 0..L-1 visible).
@@ -124,6 +156,8 @@ def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = N
               physical pages a random permutation).
     ragged  : decode lengths ~ U[1024, L] per sequence, with sequence 0 at
               2048 and sequence 1 at 2049 (the short-history boundary).
+    with_attention=False leaves q and the latent cache empty (indexer-only
+    tests of long histories).
     """
     c = dict(CONFIGS[config_id])
     kind = c["kind"]
@@ -136,22 +170,9 @@ def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = N
     if paged is None:
         paged = kind == "paged2"
 
-    # context lengths (stream 0)
-    r_len = _rng(config_id, seed_offset, 0)
-    if lengths is not None:
-        seq_ctx = np.asarray(lengths, np.int64).copy()
-        nseq = len(seq_ctx)
-    elif kind == "paged2":
-        z = r_len.standard_normal(nseq)
-        seq_ctx = np.clip(np.round(np.exp(math.log(L) + 1.0 * z)), 512, 131072).astype(np.int64)
-    elif ragged:
-        seq_ctx = r_len.integers(1024, L, size=nseq, endpoint=True).astype(np.int64)
-        if nseq > 0:
-            seq_ctx[0] = min(2048, L)
-        if nseq > 1:
-            seq_ctx[1] = min(2049, L)
-    else:
-        seq_ctx = np.full(nseq, L, np.int64)
+    seq_ctx = context_lengths(config_id, seed_offset=seed_offset, nseq=nseq, L=L,
+                              ragged=ragged, lengths=lengths)
+    nseq = len(seq_ctx)
 
     if kind == "prefill":
         assert nseq == 1
@@ -216,11 +237,15 @@ def make_inputs(config_id: int, *, seed_offset: int = 0, nseq: Optional[int] = N
     k_scale = None
     if with_k_scale:
         # powers of two in [1/4, 4] (e8m0-style block scales)
-        k_scale = np.exp2(_rng(config_id, seed_offset, 5).integers(-2, 3, size=rows)).astype(np.float32)
+        k_scale = np.exp2(_rng(config_id, seed_offset, 8).integers(-2, 3, size=rows)).astype(np.float32)
 
     # attention query and latent cache (streams 6, 7)
-    q = _normal_bf16(_rng(config_id, seed_offset, 6), (nq, h, D_QK))
-    kv = _normal_bf16(_rng(config_id, seed_offset, 7), (rows, D_QK))
+    if with_attention:
+        q = _normal_bf16(_rng(config_id, seed_offset, 6), (nq, h, D_QK))
+        kv = _normal_bf16(_rng(config_id, seed_offset, 7), (rows, D_QK))
+    else:
+        q = np.zeros((nq, h, D_QK), np.uint16)
+        kv = np.zeros((1, D_QK), np.uint16)
 
     return Inputs(config_id=config_id, name=c["name"], kind=kind, h_idx=h_idx,
                   d_idx=d_idx, h=h, d_qk=D_QK, d_v=D_V, topk=k,

@@ -25,6 +25,7 @@ from long_context_decode_indexer_b200.synth import CONFIGS, make_inputs
 pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not cuda_ok(), reason="needs a CUDA GPU")]
 
 WORKLOADS = {c["name"]: cid for cid, c in CONFIGS.items() if cid != 1}
+WORKLOADS["long_decode_16x128k_ragged"] = 3   # L ~ U[1024, 131072], sequences 0/1 at 2048/2049
 
 
 def _forward(db):
@@ -53,10 +54,57 @@ def _sample(inp, cid, count=4):
     return np.array(sorted(pick))
 
 
+def test_indexer_scores_at_full_context_element_by_element():
+    """dsa_indexer_scores over two 131072-position histories (the long-decode
+    shapes, heavy tail included), every score against the oracle."""
+    from gpu_util import check_scores, gpu_scores, oracle_scores
+    inp = make_inputs(3, nseq=2, with_attention=False)
+    db = upload(inp)
+    g = gpu_scores(db, ld=inp.max_n + 64).cpu().numpy()
+    ref, absref = oracle_scores(inp, ld=inp.max_n + 64)
+    check_scores(g, ref, absref, inp.q_n)
+
+
+def test_indexer_scores_beyond_a_million_positions():
+    """160 queries (more groups than SMs: one chunk per query, capped at 2^20
+    positions, so the 1,100,000-position history takes two chunks) over one
+    shared sequence; sampled windows, the chunk seam and the last tile are
+    checked against the oracle, position by position."""
+    import dataclasses
+    from gpu_util import check_scores, gpu_scores
+    from long_context_decode_indexer_b200.synth import encode_bf16, encode_e4m3
+    n = 1_100_000
+    base = make_inputs(3, lengths=[n], with_attention=False)
+    nq = 160
+    rng = np.random.default_rng(77)
+    q_idx = encode_e4m3(rng.standard_normal((nq, base.h_idx, base.d_idx), dtype=np.float32))
+    w = encode_bf16(rng.standard_normal((nq, base.h_idx), dtype=np.float32) * np.float32(0.125))
+    q_n = np.full(nq, n, np.int32)
+    q_n[1::7] = n - 12345                                   # some shorter histories
+    inp = dataclasses.replace(base, q_idx=q_idx, w=w, q_seq=np.zeros(nq, np.int32), q_n=q_n,
+                              q=np.zeros((nq, base.h, base.d_qk), np.uint16))
+    db = upload(inp)
+    g = gpu_scores(db, ld=n)
+    sel = np.array([0, 1, 57, 159])
+    windows = [(0, 3000), (n // 2 - 1500, 3000), ((1 << 20) - 1500, 3000), (n - 12345 - 700, 1400),
+               (n - 3000, 3000)]
+    for a, wlen in windows:
+        view = dataclasses.replace(inp, q_idx=q_idx[sel], w=w[sel], q_seq=np.zeros(len(sel), np.int32),
+                                   q_n=np.clip(q_n[sel].astype(np.int64) - a, 0, wlen).astype(np.int32),
+                                   seq_row0=np.array([a], np.int64))
+        ref, absref = oracle.indexer_scores(view.q_idx, view.w, view.kidx, view.q_seq, view.q_n,
+                                            seq_row0=view.seq_row0, ld=wlen, with_abs=True)
+        got = g[torch.from_numpy(sel).cuda(), a:a + wlen].cpu().numpy()
+        got = np.where(np.arange(wlen)[None, :] < view.q_n[:, None], got, -np.inf)
+        check_scores(got, ref, absref, view.q_n)
+    tail = g[:, n - 12345:].cpu().numpy()                    # beyond n for the shorter queries
+    assert np.all(np.isneginf(tail[1::7]))
+
+
 @pytest.mark.parametrize("workload", sorted(WORKLOADS))
 def test_full_size_forward_on_sampled_queries(workload):
     cid = WORKLOADS[workload]
-    inp = make_inputs(cid)
+    inp = make_inputs(cid, ragged=workload.endswith("_ragged"))
     db = upload(inp)
     idx, out, lse = _forward(db)
     sel = _sample(inp, cid)

@@ -140,6 +140,30 @@ def test_sparse_mla_matches_oracle(case):
     check_attention(out, lse, ref_out, ref_lse)
 
 
+@pytest.mark.parametrize("magnitude", [1e9, 1e5, 1e-6])
+def test_sparse_mla_split_partials_keep_the_bf16_range(magnitude):
+    """Latents far outside fp16's range (|c| ~ 1e5 and 1e9: outputs beyond
+    fp16's 65504) or deep in its subnormals (|c| ~ 1e-6), with the query scaled inversely so that the scores stay
+    those of the standard workload: two queries give 32 splits each, so every
+    output goes through the split partials and the combine."""
+    import dataclasses
+    from long_context_decode_indexer_b200.synth import encode_bf16
+    inp = make_inputs(2, lengths=[3000, 2500])
+
+    def scaled(bits, f):
+        x = (bits.astype(np.uint32) << 16).view(np.float32) * np.float32(f)
+        return encode_bf16(x)
+
+    inp = dataclasses.replace(inp, kv=scaled(inp.kv, magnitude), q=scaled(inp.q, 1.0 / magnitude))
+    rng = np.random.default_rng(21)
+    idx = np.stack([rng.choice(int(n), size=inp.topk, replace=False) for n in inp.q_n]).astype(np.int32)
+    db = upload(inp)
+    out, lse = gpu_mla(db, idx)
+    ref_out, ref_lse = oracle_attention(inp, idx)
+    assert np.all(np.isfinite(out))
+    check_attention(out, lse, ref_out, ref_lse, magnitude=magnitude)
+
+
 def test_sparse_mla_prefill_entry_matches_oracle():
     inp = make_inputs(4, L=600, topk=256)
     rng = np.random.default_rng(9)

@@ -36,8 +36,8 @@ def _worker(rank, world, port, out):
     inp = bench.replica_inputs(1, r)
     digest = hashlib.sha256(inp.q_idx.tobytes() + inp.kidx.tobytes()).hexdigest()
     rate = bench.job_rate(inp.nq, 10, w, t_max)
-    args = type("A", (), {"workload": "tiny_decode_4k", "warmup": 3, "steps": 1})()
-    ref = bench.run_reference(args, w, r) if r != 0 else "skipped on rank 0"
+    args = type("A", (), {"workload": "tiny_decode_4k", "warmup": 1, "steps": 1})()
+    ref = bench.run_reference(args, w, r)
     out.put((r, w, t_max, digest, inp.nq, rate, ref))
     dist.destroy_process_group()
 
@@ -77,3 +77,9 @@ def test_job_rate_counts_every_rank(results):
 
 def test_reference_arm_runs_on_rank_zero_only(results):
     assert results[1][5] is None                   # rank 1 does no work and prints nothing
+    line = results[0][5]                           # rank 0 times the oracle and returns its line
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["value"] > 0 and line["unit"] == "queries/s"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    assert line["config"]["workload"] == "tiny_decode_4k"

@@ -4,7 +4,8 @@ the index keys, the short-history boundary of the ragged variant, the
 lognormal lengths and the page tables of the paged workload."""
 import numpy as np
 
-from long_context_decode_indexer_b200.synth import CONFIGS, PAGE_SIZE, make_inputs, to_paged
+from long_context_decode_indexer_b200.synth import (CONFIGS, PAGE_SIZE, context_lengths,
+                                                    make_inputs, to_paged)
 
 
 def _dec_e4m3(codes):
@@ -31,6 +32,15 @@ def test_streams_are_independent_per_tensor():
     assert np.array_equal(a.kv, b.kv)
     c = make_inputs(2, nseq=2, L=600, seed_offset=1)  # another replica
     assert not np.array_equal(a.kidx, c.kidx)
+    # the key scales have a stream of their own: asking for them changes no
+    # other tensor, and they are not a function of the heavy-tail draw
+    d = make_inputs(2, nseq=2, L=600, with_k_scale=True)
+    assert np.array_equal(a.kidx, d.kidx) and np.array_equal(a.q_idx, d.q_idx)
+    assert np.array_equal(a.kv, d.kv) and np.array_equal(a.w, d.w)
+    tail_rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence([1002, 5])))
+    same_as_tail = np.exp2(tail_rng.integers(-2, 3, size=d.rows)).astype(np.float32)
+    assert not np.array_equal(d.k_scale, same_as_tail)
+    assert set(np.unique(d.k_scale).tolist()) <= {0.25, 0.5, 1.0, 2.0, 4.0}
 
 
 def test_heavy_tail_scales_one_percent_of_each_sequence():
@@ -52,10 +62,15 @@ def test_ragged_variant_pins_the_short_history_boundary():
 def test_paged_workload_lengths_and_page_tables():
     inp = make_inputs(5, nseq=16)
     L = inp.seq_len.astype(np.int64) - 1             # context of the first query
-    assert np.all((L >= 512) & (L <= 131072))
+    assert np.all((L >= 512) & (L <= 131071))
+    assert inp.q_n.max() <= 131072                   # the speculative token too
     assert abs(np.median(np.log(L)) - np.log(16384)) < 0.6   # median 16384, sigma 1
     assert np.array_equal(inp.q_n[0::2], L) and np.array_equal(inp.q_n[1::2], L + 1)
     assert inp.page_size == PAGE_SIZE
+    assert context_lengths(5).max() <= 131071        # the full 128-sequence draw
+    clipped = context_lengths(5, L=1 << 22, nseq=8)  # a median far above the clip
+    assert clipped.max() == 131071                   # n <= 131072 for the speculative token too
+    assert np.array_equal(context_lengths(5, nseq=16), L)
     pages = (inp.seq_len.astype(np.int64) + PAGE_SIZE - 1) // PAGE_SIZE
     used = np.concatenate([inp.page_table[i, :pages[i]] for i in range(len(pages))])
     assert np.array_equal(np.sort(used), np.arange(pages.sum()))   # a permutation of all pages
