@@ -38,17 +38,21 @@ def _stale() -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, defines=()) -> str:
+    """Compile the library (to `out`, default the in-tree libdsa_b200.so),
+    with extra -D `defines`."""
+    target = out or LIB
+    if not force and out is None and not defines and not _stale():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
+    tmp = target + ".tmp%d" % os.getpid()
     cmd = [NVCC, *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "--expt-relaxed-constexpr",
-           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+           "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
+           *["-D" + d for d in defines], "-o", tmp, *sources()]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, target)
+    return target
 
 
 if __name__ == "__main__":

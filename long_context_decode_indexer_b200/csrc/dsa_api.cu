@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -31,6 +32,20 @@ int cuda_fail(cudaError_t e, const char *what) {
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Test hook for the bounded waits.  DSA_TEST_INJECT_TIMEOUT=indexer (or
+// =attention) makes the calls that launch that kernel run it with a short
+// wait budget (1e5 SM cycles, ~50 us) and with one arrival its first CTA's
+// MMA issuer waits for never made, so the wait runs out: the kernel records
+// DSA_ERR_TIMEOUT in the status word, lets its other waits run out the same
+// way, waits for its own copies in flight and returns.  Unset, every wait
+// has the ~1 s budget and nothing is skipped.
+constexpr long long kTestWaitBudget = 100000;
+
+bool inject_timeout(const char *kernel) {
+    const char *v = getenv("DSA_TEST_INJECT_TIMEOUT");
+    return v != nullptr && strcmp(v, kernel) == 0;
+}
 
 size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -116,6 +131,7 @@ int check_kv(const dsa_params *p, const dsa_kv *kv) {
 // ----------------------------------------------------------------- planning
 struct IndexerPlan {
     int hp, qg, gpb, n_groups, P, chunk, stages, acc_bufs;
+    bool parallel;  // fused, several chunks, every CTA resident: each chunk selects its own part
     uint32_t tmem_cols;
     size_t smem;
 };
@@ -146,19 +162,30 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     int64_t P = p_fill < p_small ? p_fill : p_small;
     if (P < p_min) P = p_min;
     if (P < 1) P = 1;
+    pl.parallel = false;
     if (mode != dsa::kModeScores) {
-        // the merge list (P * topk composites) must fit on chip
-        int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
-        if (p_cap > dsa::kMaxChunks) p_cap = dsa::kMaxChunks;
-        if (P > p_cap) {
-            if (p_min > p_cap) return fail(DSA_ERR_UNSUPPORTED, "history too long for topk=%d (max_n=%d)", p->topk, p->max_n);
-            P = p_cap;
+        // Parallel selection (fused, the grid resident at once) keeps no
+        // merge list in one CTA: up to kMaxChunks chunks.  Otherwise the
+        // last CTA's merge list (P * topk composites) must fit on chip.
+        const int64_t p_par = P < dsa::kMaxChunks ? P : dsa::kMaxChunks;
+        if (mode == dsa::kModeFused && p_par > 1 && p_par >= p_min &&
+            static_cast<int64_t>(pl.n_groups) * p_par <= num_sms()) {
+            P = p_par;
+            pl.parallel = true;
+        } else {
+            int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
+            if (p_cap > dsa::kMaxChunks) p_cap = dsa::kMaxChunks;
+            if (P > p_cap) {
+                if (p_min > p_cap) return fail(DSA_ERR_UNSUPPORTED, "history too long for topk=%d (max_n=%d)", p->topk, p->max_n);
+                P = p_cap;
+            }
         }
     }
     int64_t chunk = (sp + P - 1) / P;
     chunk = (chunk + 127) / 128 * 128;
     if (chunk > chunk_max) chunk = chunk_max;
     P = (sp + chunk - 1) / chunk;
+    if (P <= 1) pl.parallel = false;
     pl.P = static_cast<int>(P);
     pl.chunk = static_cast<int>(chunk);
     if (mode != dsa::kModeScores) {
@@ -167,7 +194,7 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
         const int nw = (mode == dsa::kModeTopk ? dsa::kK2Threads : dsa::kK1Threads) / 32;
         const int merge_n = pl.P * (p->topk + 2);
         if (dsa::emit_ballot_words(pl.chunk, nw) > dsa::kSelBinsHost ||
-            dsa::emit_ballot_words(merge_n, nw) > (pl.qg + 1) * dsa::kSelBinsHost)
+            (!pl.parallel && dsa::emit_ballot_words(merge_n, nw) > (pl.qg + 1) * dsa::kSelBinsHost))
             return fail(DSA_ERR_UNSUPPORTED, "selection scratch too small for this plan");
     }
     pl.acc_bufs = (dsa::kK1MaxAcc * pl.qg * pl.hp <= 512) ? dsa::kK1MaxAcc : 2;
@@ -180,12 +207,13 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     if (mode != dsa::kModeTopk) {
         int st = dsa::kK1MaxStages;
         while (st >= 2 &&
-               dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st).total > 232448)
+               dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st, !pl.parallel).total > 232448)
             --st;
         if (st < 2) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
         pl.stages = st;
     }
-    const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, pl.stages);
+    const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, pl.stages,
+                                           !pl.parallel);
     pl.smem = L.total;
     if (pl.smem > 232448) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
     return DSA_OK;
@@ -224,24 +252,31 @@ MlaPlan plan_mla(const dsa_params *p) {
 
 // -------------------------------------------------------------- workspace
 struct WsLayout {
-    size_t status, ghist, gtot, cand, cand_cnt, done, idx, part_o, part_lse, part_scale, total;
+    size_t status, ghist, gtot, published, cand, cand_cnt, cand_above, done, idx, part_o, part_lse,
+        part_scale, total;
     size_t zero_begin, zero_end;  // cleared at the start of every call
 };
 
+int cand_stride(const dsa_params *p) { return (p->topk + 3) & ~3; }
+
 size_t indexer_ws(const dsa_params *p, const IndexerPlan &pl, int mode, size_t off, WsLayout &w) {
-    w.ghist = w.cand = w.cand_cnt = w.done = off;
+    w.ghist = w.gtot = w.published = w.cand = w.cand_cnt = w.cand_above = w.done = off;
     if (mode == dsa::kModeScores || pl.P <= 1) return off;
     w.zero_begin = off;
     w.ghist = off;
     off = up(off + static_cast<size_t>(p->nq) * 2048 * 4, 256);
     w.gtot = off;
     off = up(off + static_cast<size_t>(p->nq) * 4, 256);
+    w.published = off;
+    off = up(off + static_cast<size_t>(p->nq) * 4, 256);
     w.done = off;
     off = up(off + static_cast<size_t>(pl.n_groups) * 4, 256);
     w.zero_end = off;
     w.cand = off;
-    off = up(off + static_cast<size_t>(p->nq) * pl.P * ((p->topk + 1) & ~1) * 8, 256);
+    off = up(off + static_cast<size_t>(p->nq) * pl.P * cand_stride(p) * 8, 256);
     w.cand_cnt = off;
+    off = up(off + static_cast<size_t>(p->nq) * pl.P * 4, 256);
+    w.cand_above = off;
     off = up(off + static_cast<size_t>(p->nq) * pl.P * 4, 256);
     return off;
 }
@@ -346,15 +381,23 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.idx = idx;
     a.nsel = nsel;
     a.status = at<int>(ws, wl.status);
+    a.wait_budget = dsa::kWaitBudgetCycles;
+    if (mode != dsa::kModeTopk && inject_timeout("indexer")) {
+        a.wait_budget = kTestWaitBudget;
+        a.inject = 1;
+    }
     if (mode != dsa::kModeScores && pl.P > 1) {
         a.ghist = at<uint32_t>(ws, wl.ghist);
         a.gtot = at<uint32_t>(ws, wl.gtot);
+        a.published = at<uint32_t>(ws, wl.published);
         a.done = at<uint32_t>(ws, wl.done);
-        // every CTA of the launch is resident at once (one CTA per SM)
-        a.wait_hist = (static_cast<int64_t>(pl.n_groups) * pl.P <= num_sms()) ? 1 : 0;
+        // every CTA of the launch is resident at once (at most one per SM
+        // is needed): each chunk selects its own part of the output
+        a.parallel = pl.parallel ? 1 : 0;
         a.cand = at<uint64_t>(ws, wl.cand);
-        a.cand_stride = (p->topk + 1) & ~1;
+        a.cand_stride = cand_stride(p);
         a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
+        a.cand_above = at<int32_t>(ws, wl.cand_above);
         cudaError_t e = cudaMemsetAsync(static_cast<uint8_t *>(ws) + wl.zero_begin, 0,
                                         wl.zero_end - wl.zero_begin, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
@@ -420,6 +463,11 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.part_lse = m.splits > 1 ? at<float>(ws, wl.part_lse) : nullptr;
     a.part_scale = m.splits > 1 ? at<float>(ws, wl.part_scale) : nullptr;
     a.status = at<int>(ws, wl.status);
+    a.wait_budget = dsa::kWaitBudgetCycles;
+    if (inject_timeout("attention")) {
+        a.wait_budget = kTestWaitBudget;
+        a.inject = 1;
+    }
     for (int q0 = 0; q0 < p->nq; q0 += m.wave) {
         const int nw = (p->nq - q0) < m.wave ? (p->nq - q0) : m.wave;
         a.q0 = q0;

@@ -18,18 +18,28 @@
 // -> MMA completion no longer paces the stream.
 //
 // Fused mode keeps the chunk's scores in shared memory as order-preserving
-// keys.  Exact selection across chunks without a grid barrier:
-//   1. each chunk adds the histogram of its keys' top 11 bits to the query's
-//      global histogram G;
-//   2. it reads G back: any snapshot of G is a lower bound of the final one
-//      bin by bin, so the bin where G's count from the top reaches k is at
-//      most the final threshold bin -- keys in lower bins can never win;
-//   3. it publishes its keys at or above that bin (capped by an exact local
-//      TopK of size k), then bumps the group's done counter;
-//   4. the last CTA of the group takes everything above the final threshold
+// keys; scores never leave the SM.  With one chunk per group the CTA selects
+// directly.  With several chunks, each adds the histogram of its keys' top
+// 11 bits to the query's global histogram G.  Then:
+//
+// Parallel (every CTA of the launch is resident at once, the usual decode
+// case): each chunk waits (bounded) until every chunk has added its
+// histogram, so its snapshot of G is final and gives the threshold bin d*
+// and the number of keys above it.  Each chunk publishes its keys of bin d*
+// (at most the `need` largest) and its count of keys above d*; after a
+// second bounded wait for every chunk's list, each chunk finds the exact
+// threshold among the bin-d* lists itself, derives every chunk's selected
+// count (hence its own offset in the ascending output) and writes its own
+// selected positions.  No CTA waits for another to finish its chunk.
+//
+// Otherwise (more CTAs than can be resident):
+//   1. any snapshot of G is a lower bound of the final one bin by bin, so
+//      the bin where G's count from the top reaches k is at most the final
+//      threshold bin -- keys in lower bins can never win;
+//   2. each chunk publishes its keys at or above that bin (capped by an
+//      exact local TopK of size k), then bumps the group's done counter;
+//   3. the last CTA of the group takes everything above the final threshold
 //      bin and radix-refines the threshold bin among the candidates.
-// Scores never leave the SM.  With one chunk per group the CTA selects
-// directly.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -59,12 +69,17 @@ struct K1Smem {
     uint32_t g_seen;                     // positions counted into G before the snapshot
     int32_t cand_off[kMaxChunks + 1];    // merge: prefix of the chunks' (padded) candidate counts
     int32_t cand_n[kMaxChunks];
+    int32_t cand_above[kMaxChunks];      // parallel: keys of each chunk above the threshold bin
+    int32_t sel_cnt[kMaxChunks];         // parallel: positions each chunk selects
+    int32_t sel_ok;                      // parallel: the bounded waits succeeded
+    unsigned long long t_exact;          // parallel: the need-th largest listed composite
     uint64_t merge_bar;                  // merge: bulk copies of the candidate lists
     uint32_t merge_phase;
+    uint64_t mma_done;                   // every MMA issued by this CTA has completed
     SelectScratch sel;
 };
 
-static_assert(sizeof(K1Smem) <= 1024, "K1Smem must fit the 1 KB misc area of k1_layout");
+static_assert(sizeof(K1Smem) <= kK1MiscBytes, "K1Smem must fit the misc area of k1_layout");
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -108,6 +123,26 @@ struct ListSrc {
     }
 };
 
+// The chunks' candidate lists read in place from global memory (L2), as one
+// list whose chunk segments start at the virtual offsets off[c] (each a
+// multiple of 4; the entries past a chunk's count are zero composites).
+struct GlobalSegSrc {
+    const uint64_t *cand;  // [P, stride]
+    int stride, P;
+    const int32_t *off;    // shared: P + 1 virtual offsets
+    __device__ void load4(int i, uint64_t (&v)[4]) const {
+        int c = 0;
+        while (c + 1 < P && off[c + 1] <= i) ++c;
+        const uint64_t *p = cand + static_cast<int64_t>(c) * stride + (i - off[c]);
+        const uint4 a = __ldcg(reinterpret_cast<const uint4 *>(p));
+        const uint4 b = __ldcg(reinterpret_cast<const uint4 *>(p + 2));
+        v[0] = (static_cast<uint64_t>(a.y) << 32) | a.x;
+        v[1] = (static_cast<uint64_t>(a.w) << 32) | a.z;
+        v[2] = (static_cast<uint64_t>(b.y) << 32) | b.x;
+        v[3] = (static_cast<uint64_t>(b.w) << 32) | b.z;
+    }
+};
+
 // Copy a query's global histogram (2048 words, L2) to shared memory.  All
 // of a thread's loads are issued before any store, so the copy costs one L2
 // round trip instead of one per loop iteration.  Needs blockDim >= 256.
@@ -136,6 +171,165 @@ __device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScrat
     return r;
 }
 
+// Parallel exact selection of query q by chunk c = blockIdx.x % P, once the
+// snapshot of G taken in chunk_select is final (every chunk's histogram in
+// it): d* is the threshold bin, `above` the query's keys in higher bins,
+// need = K - above the keys to take from bin d*.
+//   1. publish this chunk's keys of bin d* (its `need` largest at most: a
+//      key beaten by `need` keys of the bin in its own chunk never wins) and
+//      its count of keys above d*; bump the query's `published` counter;
+//   2. wait (bounded) until every chunk has published, read all the lists
+//      (staged into the free streaming area when they fit, else in place)
+//      and find the exact threshold T: the need-th largest composite among
+//      them;
+//   3. every chunk's selected count is its keys above d* plus its listed
+//      keys >= T; the chunks before this one give its offset, and it writes
+//      its own keys >= T there, in ascending position order.
+// `list` / `list_cap`: shared memory below the chunk's keys (the TMA ring and
+// the q tile, free once streaming is over), in composites.
+__device__ void parallel_select(const K1Params &a, K1Smem &sm, int q, int qi, const uint32_t *keys,
+                                int start, int len, const uint32_t *lhist, uint32_t *scratch,
+                                uint64_t *list, int list_cap) {
+    const int K = a.topk, P = a.P, c = blockIdx.x % P;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+    LocalSrc src{keys, start};
+    const bool complete = sm.sel_ok && sm.g_complete[qi];
+    const uint32_t d = sm.g_digit[qi];
+    const uint32_t need = static_cast<uint32_t>(K) - sm.g_above[qi];
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * P + c) * a.cand_stride;
+    int32_t m = 0;
+    int32_t above_c = 0;
+    if (complete) {
+        above_c = static_cast<int32_t>(hist_sum_from(lhist, d + 1, sm.sel));
+        const uint32_t bucket_c = lhist[d];
+        uint64_t thr = static_cast<uint64_t>(d) << 53;
+        if (bucket_c > need) thr = radix_refine(src, len, d, 1, need, scratch, sm.sel);
+        m = static_cast<int32_t>(emit_ordered(
+            src, len, [thr, d](uint64_t v) { return (v >> 53) == d && v >= thr; },
+            [cand, K](uint32_t slot, uint64_t v) {
+                if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
+            },
+            0u, sm.sel.wsum, reinterpret_cast<uint4 *>(scratch)));
+        if (m > K) m = K;  // cannot happen: at most `need` <= K keys pass
+    }
+    // zero composites pad the list to a multiple of 4 (below every key)
+    if (tid < 4 && m + tid < ((m + 3) & ~3)) cand[m + tid] = 0ull;
+    if (tid == 0) {
+        a.cand_cnt[static_cast<int64_t>(q) * P + c] = m;
+        a.cand_above[static_cast<int64_t>(q) * P + c] = above_c;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) {
+        atomicAdd(&a.published[q], 1u);
+        sm.sel_ok = complete && wait_count(&a.published[q], static_cast<uint32_t>(P), a.wait_budget);
+        if (!sm.sel_ok) record_status(a.status, DSA_ERR_TIMEOUT);
+    }
+    __syncthreads();
+    if (!sm.sel_ok) return;
+    // every chunk's list length (padded to 4) and above-count; offsets
+    const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * P;
+    const int32_t *abv = a.cand_above + static_cast<int64_t>(q) * P;
+    if (warp == 0) {
+        const int m_l = lane < P ? min(__ldcg(&cnt[lane]), K) : 0;
+        const int padded = (m_l + 3) & ~3;
+        const int incl = static_cast<int>(warp_incl_scan(static_cast<uint32_t>(padded)));
+        if (lane < P) {
+            sm.cand_off[lane] = incl - padded;
+            sm.cand_n[lane] = m_l;
+            sm.cand_above[lane] = __ldcg(&abv[lane]);
+        }
+        const int tot = __shfl_sync(0xffffffffu, incl, 31);
+        const int true_tot = static_cast<int>(warp_sum(static_cast<uint32_t>(m_l)));
+        if (lane == 0) {
+            sm.cand_off[P] = tot;
+            sm.sel.res[3] = static_cast<uint32_t>(true_tot);
+            if (tot <= list_cap) {
+                fence_proxy_async_global();
+                mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(tot) * 8u);
+            }
+        }
+    }
+    __syncthreads();
+    const int total = sm.cand_off[P];
+    const uint32_t listed = sm.sel.res[3];
+    const bool staged = total <= list_cap;
+    if (staged) {
+        if (tid < P && sm.cand_n[tid] > 0) {
+            fence_proxy_async_global();
+            bulk_load(list + sm.cand_off[tid], a.cand + (static_cast<int64_t>(q) * P + tid) * a.cand_stride,
+                      static_cast<uint32_t>((sm.cand_n[tid] + 3) & ~3) * 8u, &sm.merge_bar);
+        }
+        const bool ok = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase, a.wait_budget));
+        if (tid == 0) sm.merge_phase ^= 1u;
+        __syncthreads();
+        if (!ok) {
+            if (tid == 0) record_status(a.status, DSA_ERR_TIMEOUT);
+            return;
+        }
+    }
+    // the threshold: the need-th largest listed composite (listed >= need:
+    // a chunk whose bin-d* keys exceed `need` lists `need` of them, else all).
+    // radix_refine gives a bound T with exactly `need` listed composites >= T;
+    // the smallest of them, Te, is the threshold itself.  Selecting own keys
+    // >= Te (not >= T) matters: a chunk's unlisted bin-d* keys lie below its
+    // smallest listed one, which is <= Te, but may lie above T.
+    uint64_t T = static_cast<uint64_t>(d) << 53;
+    if (listed != need) {
+        if (staged) T = radix_refine(ListSrc{list}, total, d, 1, need, scratch, sm.sel);
+        else T = radix_refine(GlobalSegSrc{a.cand + static_cast<int64_t>(q) * P * a.cand_stride,
+                                           a.cand_stride, P, sm.cand_off},
+                              total, d, 1, need, scratch, sm.sel);
+    }
+    if (tid == 0) sm.t_exact = ~0ull;
+    __syncthreads();
+    // selected count of every chunk: keys above d* + listed keys >= T
+    for (int cc = warp; cc < P; cc += nwarps) {
+        const int mm = sm.cand_n[cc];
+        const uint64_t *seg = staged ? list + sm.cand_off[cc]
+                                     : a.cand + (static_cast<int64_t>(q) * P + cc) * a.cand_stride;
+        uint32_t k = 0;
+        unsigned long long lo = ~0ull;
+        for (int j = lane; j < mm; j += 32) {
+            const uint64_t v = staged ? seg[j] : __ldcg(&seg[j]);
+            if (v >= T) {
+                ++k;
+                lo = v < lo ? v : lo;
+            }
+        }
+        k = warp_sum(k);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, lo, o);
+            lo = y < lo ? y : lo;
+        }
+        if (lane == 0) {
+            sm.sel_cnt[cc] = sm.cand_above[cc] + static_cast<int32_t>(k);
+            if (k) atomicMin(&sm.t_exact, lo);
+        }
+    }
+    __syncthreads();
+    const uint64_t Te = sm.t_exact;
+    int off = 0, all = 0;
+    for (int cc = 0; cc < P; ++cc) {
+        off += cc < c ? sm.sel_cnt[cc] : 0;
+        all += sm.sel_cnt[cc];
+    }
+    int32_t *out = a.idx + static_cast<int64_t>(q) * K;
+    const uint32_t got = emit_ordered(
+        src, len, [Te](uint64_t v) { return v >= Te; },
+        [out, K](uint32_t slot, uint64_t v) {
+            if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
+        },
+        static_cast<uint32_t>(off), sm.sel.wsum, reinterpret_cast<uint4 *>(scratch));
+    if (tid == 0) {
+        if (got != static_cast<uint32_t>(off + sm.sel_cnt[c]) || all != K)
+            record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        if (c == 0 && a.nsel) a.nsel[q] = K;
+    }
+    __syncthreads();
+}
+
 // Everything one query of a chunk does after its keys are in shared memory:
 // direct selection (one chunk), or publishing candidates (several chunks).
 // `keys` holds the chunk's keys for positions [start, start + len) and
@@ -144,7 +338,7 @@ __device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScrat
 // same from run to run.
 __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n,
                              const uint32_t *keys, int start, int len, const uint32_t *lhist,
-                             uint32_t *scratch) {
+                             uint32_t *scratch, uint64_t *list, int list_cap) {
     const int K = a.topk;
     LocalSrc src{keys, start};
     if (a.P == 1) {
@@ -170,31 +364,22 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
         return;
     }
 
-    // ---- several chunks: publish this chunk's histogram, then its candidates
+    // ---- several chunks: publish this chunk's histogram, then read G back
     uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
     const int c = blockIdx.x % a.P;
-    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * a.cand_stride;
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
         if (lhist[b]) atomicAdd(&G[b], lhist[b]);
     __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
         atomicAdd(&a.gtot[q], static_cast<uint32_t>(len));
-        // When every chunk of the query runs at the same time, wait (bounded)
-        // until all of them have added their histograms: the bound below is
-        // then the final threshold bin.  Any earlier snapshot is still a valid
-        // (weaker) bound, so running out of time only costs candidates.
-        if (a.wait_hist) {
-            const long long t0 = clock64();
-            while (ld_acquire_u32(&a.gtot[q]) < static_cast<uint32_t>(n)) {
-                if (clock64() - t0 > kHistWaitCycles) break;
-                __nanosleep(64);
-            }
-        }
-        // Read the count BEFORE the snapshot: every chunk adds its histogram
-        // to G before its count to gtot, so if the count already covers all n
-        // positions here, the snapshot below holds every chunk's histogram.
-        // (Read after the snapshot, it could cover chunks the snapshot missed.)
+        // Parallel mode: every chunk runs at the same time, so wait (bounded)
+        // until all of them have added their histograms.  Read the count
+        // BEFORE the snapshot: every chunk adds its histogram to G before its
+        // count to gtot, so a count that covers all n positions here proves
+        // the snapshot below complete.  (Read after the snapshot, it could
+        // cover chunks the snapshot missed.)
+        sm.sel_ok = a.parallel ? wait_count(&a.gtot[q], static_cast<uint32_t>(n), a.wait_budget) : 1;
         sm.g_seen = ld_acquire_u32(&a.gtot[q]);
     }
     __syncthreads();
@@ -210,6 +395,11 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
         sm.g_above[qi] = sm.sel.res[1];
     }
     __syncthreads();
+    if (a.parallel) {
+        parallel_select(a, sm, q, qi, keys, start, len, lhist, scratch, list, list_cap);
+        return;
+    }
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * a.cand_stride;
     const uint32_t at_or_above = hist_sum_from(lhist, dlow, sm.sel);
     uint64_t thr = static_cast<uint64_t>(dlow) << 53;
     if (at_or_above > static_cast<uint32_t>(K)) {
@@ -295,7 +485,7 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
             bulk_load(list + sm.cand_off[c], cand + static_cast<int64_t>(c) * a.cand_stride,
                       static_cast<uint32_t>((m + 1) & ~1) * 8u, &sm.merge_bar);
     }
-    const bool staged = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase));
+    const bool staged = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase, a.wait_budget));
     if (threadIdx.x < a.P && (sm.cand_n[threadIdx.x] & 1)) list[sm.cand_off[threadIdx.x] + sm.cand_n[threadIdx.x]] = 0ull;
     if (threadIdx.x == 0) sm.merge_phase ^= 1u;
     __syncthreads();
@@ -356,7 +546,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     k1_indexer(const __grid_constant__ CUtensorMap kmap, const K1Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages);
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages, !a.parallel);
     uint8_t *stages = base + L.stages;
     uint8_t *qtile = base + L.qtile;
     uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
@@ -390,7 +580,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     // The producer (thread 0) fills the TMA ring as soon as its barriers
     // exist, so the first tiles are in flight during the rest of the set-up.
     const int64_t row0 = (a.page_table == nullptr && nqg > 0) ? a.seq_row0[seq] : 0;
+    // tests only: the first CTA never loads its first tile, so the MMA
+    // issuer's wait for it runs out
+    const bool skip_first = a.inject != 0 && blockIdx.x == 0;
     auto issue_tile = [&](int t, int s) {
+        if (skip_first && t == 0) return;
         const int p0 = start + t * kTileRows;
         uint8_t *dst = stages + s * kTileBytes;
         if (a.page_table == nullptr) {
@@ -412,6 +606,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         sm.is_last = 0;
         for (int i = 0; i < kMaxGroupQueries; ++i) sm.g_complete[i] = 0;
         mbar_init(&sm.merge_bar, 1);
+        mbar_init(&sm.mma_done, 1);
         sm.merge_phase = 0;
         for (int s = 0; s < a.stages; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -466,15 +661,24 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 // in this single-thread loop, which paces the whole stream
                 int s = n_pro == a.stages ? 0 : n_pro;
                 uint32_t ph = n_pro == a.stages ? 1u : 0u;
+                int t_end = n_pro;  // tiles issued (or skipped) so far
                 for (int t = n_pro; t < ntiles; ++t) {
-                    if (!mbar_wait(&sm.empty[s], ph ^ 1) || sm.abort) {
+                    if (!mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
                     }
                     issue_tile(t, s);
+                    t_end = t + 1;
                     if (++s == a.stages) { s = 0; ph ^= 1; }
                 }
+                // before the CTA may exit, every tile load issued must have
+                // landed: wait (bounded) for the newest phase of each stage
+                // (a no-op when the MMA consumed them all)
+                for (int t = max(t_end - a.stages, 0); t < t_end; ++t)
+                    if (!(skip_first && t == 0) &&
+                        !mbar_wait(&sm.full[t % a.stages], static_cast<uint32_t>(t / a.stages) & 1u, a.wait_budget))
+                        record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else if (warp == 1) {
             if (lane == 0) {
@@ -488,7 +692,8 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 int s = 0, b = 0;
                 uint32_t ph = 0, aph = 0;
                 for (int t = 0; t < ntiles; ++t) {
-                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1) || !mbar_wait(&sm.full[s], ph) || sm.abort) {
+                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
+                        !mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
@@ -503,6 +708,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                     if (++s == a.stages) { s = 0; ph ^= 1; }
                     if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
                 }
+                // every MMA issued must complete before TMEM is freed
+                tc_commit(&sm.mma_done);
+                if (!mbar_wait(&sm.mma_done, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else {
             // epilogue: group 0 = warps 2..5 takes even tiles (buffer 0),
@@ -520,7 +728,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 // acquire, which cannot fail: the buffer's next phase needs
                 // this warp's release below.  The warp proceeds only if all
                 // lanes saw it (tcgen05.ld below is warp-collective).
-                const bool ok = warp_wait(&sm.acc_full[b], aph, &sm.abort);
+                const bool ok = warp_wait(&sm.acc_full[b], aph, &sm.abort, a.wait_budget);
                 if (!ok) {
                     if (lane == 0) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
@@ -591,15 +799,19 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 
     // ---- selection (fused mode)
     if (MODE == kModeFused && !sm.abort) {
+        // parallel selection stages the chunks' lists below the keys (the
+        // TMA ring and the q tile, free now)
+        uint64_t *below_keys = reinterpret_cast<uint64_t *>(base);
+        const int below_cap = static_cast<int>(L.keys / sizeof(uint64_t));
         for (int qi = 0; qi < nqg; ++qi) {
             const int n = sm.n_q[qi];
             if (n <= a.topk) continue;
             const int qlen = max(min(end, n) - start, 0);
             chunk_select(a, sm, q0 + qi, qi, n, keys + qi * a.chunk, start, qlen,
-                         lhist + qi * kSelBins, hist);
+                         lhist + qi * kSelBins, hist, below_keys, below_cap);
             __syncthreads();
         }
-        if (a.P > 1) {
+        if (a.P > 1 && !a.parallel) {
             bool any = false;
             for (int qi = 0; qi < nqg; ++qi) any |= sm.n_q[qi] > a.topk;
             if (any && arrive_group(a, sm, g)) {
@@ -626,7 +838,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0);
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0, true);
     uint32_t *keys = reinterpret_cast<uint32_t *>(base + L.keys);
     uint32_t *hist = reinterpret_cast<uint32_t *>(base + L.hist);
     K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
@@ -662,7 +874,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
         }
     }
     __syncthreads();
-    chunk_select(a, sm, q, 0, n, keys, start, len, lhist, hist);
+    chunk_select(a, sm, q, 0, n, keys, start, len, lhist, hist, nullptr, 0);
     __syncthreads();
     if (a.P > 1 && arrive_group(a, sm, q)) {
         uint64_t *list = reinterpret_cast<uint64_t *>(base);
@@ -676,7 +888,7 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
 // ---------------------------------------------------------------------------
 template <int MODE, int HP, int DI>
 static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaStream_t st) {
-    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages);
+    const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages, !a.parallel);
     const size_t smem = smem_for_tmem(L.total, a.tmem_cols);
     auto kern = k1_indexer<MODE, HP, DI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -704,7 +916,7 @@ cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, co
 }
 
 cudaError_t launch_topk(const K1Params &a, cudaStream_t st) {
-    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0);
+    const K1Layout L = k1_layout(kModeTopk, 0, 1, 0, a.chunk, a.P, a.topk, 0, true);
     cudaError_t e = cudaFuncSetAttribute(k2_topk, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(L.total));
     if (e != cudaSuccess) return e;
     const int grid = a.nq * a.P;

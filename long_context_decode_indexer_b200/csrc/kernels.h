@@ -8,6 +8,11 @@
 
 namespace dsa {
 
+// Budget of a bounded wait, in SM clock cycles (about one second at 1.9 GHz).
+// A wait that runs out records DSA_ERR_TIMEOUT and abandons the work instead
+// of hanging the GPU.
+constexpr long long kWaitBudgetCycles = 2000000000LL;
+
 // ---------------------------------------------------------------- indexer
 constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
 constexpr int kModeScores = 1;  // scores written to HBM
@@ -21,7 +26,7 @@ constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 6
 constexpr int kMaxChunks = 32;       // chunks per query group (merge bookkeeping)
 constexpr int kKeysBudget = 96 * 1024;  // bytes of on-chip scores per CTA
 constexpr int kSelBinsHost = 2048;
-constexpr long long kHistWaitCycles = 100000;  // ~50 us: bounded wait for a query's full histogram
+constexpr int kK1MiscBytes = 2048;    // barriers, flags and selection scratch of k1 / k2
 
 // Shared words an ordered emission over n elements by `nwarps` warps needs:
 // one uint4 of ballots per 128-element step of each warp's slice, then 32
@@ -58,12 +63,18 @@ struct K1Params {
     // workspace
     uint32_t *ghist;      // [nq, 2048] global top-digit histograms
     uint32_t *gtot;       // [nq] positions counted into ghist so far
-    int32_t wait_hist;    // all CTAs are co-resident: wait (bounded) for the full histogram
+    int32_t parallel;     // every CTA is co-resident: each chunk selects its own part exactly
     uint64_t *cand;       // [nq, P, cand_stride] candidate composites
-    int32_t cand_stride;  // topk rounded up to even (16-byte aligned chunk lists)
+    int32_t cand_stride;  // topk rounded up to a multiple of 4 (32-byte aligned chunk lists)
     int32_t *cand_cnt;    // [nq, P]
+    int32_t *cand_above;  // [nq, P] (parallel) keys of each chunk above the threshold bin
+    uint32_t *published;  // [nq] (parallel) chunks that published their threshold-bin lists
     uint32_t *done;       // [n_groups] chunks finished
     int *status;
+    // bounded waits: budget in SM cycles; `inject` (tests only) makes one
+    // arrival the first CTA's MMA issuer waits for never happen
+    long long wait_budget;
+    int32_t inject;
 };
 
 struct K1Layout {
@@ -73,8 +84,10 @@ struct K1Layout {
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // Offsets from a 1024-byte aligned base; `total` includes the alignment slack.
+// `merge`: the last CTA of a group stages every chunk's candidates (the
+// selection used when the grid is not resident at once).
 __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, int chunk, int P,
-                                              int topk, int stages) {
+                                              int topk, int stages, bool merge) {
     K1Layout L;
     uint32_t off = 0;
     L.stages = off;
@@ -85,7 +98,7 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
     if (mode != kModeScores) off += static_cast<uint32_t>(qg) * static_cast<uint32_t>(chunk) * 4u;
     // the last CTA of a group stages the threshold-bin candidates in the
     // area below the histogram
-    if (mode != kModeScores && P > 1) {
+    if (mode != kModeScores && P > 1 && merge) {
         const uint32_t need = static_cast<uint32_t>(P) * static_cast<uint32_t>(topk + 1) * 8u;
         if (off < need) off = need;
     }
@@ -96,7 +109,7 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
     off += align_up(static_cast<uint32_t>(qg * hp * 4), 16);
     off = align_up(off, 128);
     L.misc = off;
-    off += 1024;
+    off += kK1MiscBytes;
     L.total = off + 1024;
     return L;
 }
@@ -149,6 +162,8 @@ struct MlaParams {
     float *part_lse;     // [wave_q, splits, 128]
     float *part_scale;   // [wave_q, splits, 128, 2] power of two of each half row of part_o
     int *status;
+    long long wait_budget;  // bounded waits, SM cycles
+    int32_t inject;         // tests only: the first CTA's gathers skip one arrival
 };
 
 struct MlaLayout {

@@ -8,13 +8,9 @@
 #include <stdint.h>
 
 #include "dsa.h"
+#include "kernels.h"
 
 namespace dsa {
-
-// Budget of a bounded wait, in SM clock cycles (about one second at 1.9 GHz).
-// A wait that runs out records DSA_ERR_TIMEOUT and abandons the work instead
-// of hanging the GPU.
-constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -65,12 +61,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
         : "memory");
     return done != 0;
 }
-// Wait for the phase with the given parity to complete; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// Wait for the phase with the given parity to complete; false once `budget`
+// SM cycles have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
+                                          long long budget = kWaitBudgetCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitBudgetCycles) return false;
+        if (clock64() - t0 > budget) return false;
+    }
+    return true;
+}
+
+// Spin (bounded) until the global word *p reaches `target` (acquire).
+__device__ __forceinline__ bool wait_count(const uint32_t *p, uint32_t target, long long budget) {
+    if (ld_acquire_u32(p) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_u32(p) < target) {
+        if (clock64() - t0 > budget) return false;
+        __nanosleep(64);
     }
     return true;
 }
@@ -80,9 +89,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
 // the barrier cannot complete its following phase before this warp acts
 // (the usual ring protocol: the next phase needs this warp's arrival).
 // Returns the same value in every lane; false on timeout or `abort` set.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const volatile int32_t *abort) {
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, const volatile int32_t *abort,
+                                          long long budget = kWaitBudgetCycles) {
     bool seen = true;
-    if ((threadIdx.x & 31) == 0) seen = mbar_wait(bar, parity) && !*abort;
+    if ((threadIdx.x & 31) == 0) seen = mbar_wait(bar, parity, budget) && !*abort;
     seen = __shfl_sync(0xffffffffu, seen, 0);
     if (seen) seen = mbar_try_wait(bar, parity);
     return __all_sync(0xffffffffu, seen);
@@ -136,6 +146,12 @@ __device__ __forceinline__ void cp_async_wait() {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Order this thread's generic-proxy view of global memory (including data
+// other threads released to it) before its later async-proxy (bulk copy)
+// accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ----------------------------------------------------------------- tcgen05

@@ -137,7 +137,7 @@ __device__ bool gather_pass1(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int
         if (c < kNumKChunks) {
             const int s = c % kMlaStages;
             const uint32_t ph = (c / kMlaStages) & 1;
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1) && !sm.abort);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) && !sm.abort);
             if (ok) {
                 uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
 #pragma unroll
@@ -152,7 +152,9 @@ __device__ bool gather_pass1(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int
             else cp_async_wait<0>();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.full[(c - kGatherLag) % kMlaStages]);
+            // tests only: the first CTA never publishes chunk 0
+            const bool skip = a.inject != 0 && blockIdx.x == 0 && c == kGatherLag;
+            if (lane == 0 && !skip) mbar_arrive(&sm.full[(c - kGatherLag) % kMlaStages]);
         }
     }
     return ok;
@@ -312,17 +314,25 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             // ------------------------------------------ Q chunks by TMA
             const uint32_t qbytes = static_cast<uint32_t>(hbox) * 128u;
             if (lane == 0) {
+                int c_end = 0;  // chunks whose Q tile was requested
                 for (int c = 0; c < kNumKChunks; ++c) {
                     const int s = c % kMlaStages;
                     const uint32_t ph = (c / kMlaStages) & 1;
-                    if (sm.abort || !mbar_wait(&sm.empty[s], ph ^ 1)) {
+                    if (sm.abort || !mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget)) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
                     }
                     mbar_arrive_expect_tx(&sm.full[s], qbytes);
                     tma_load_2d(ring + s * kStageBytes, &qmap, &sm.full[s], c * 64, q * a.h);
+                    c_end = c + 1;
                 }
+                // the requested tiles land before the CTA may exit: wait
+                // (bounded) for the newest phase of each stage; a stage whose
+                // row pieces were never published runs out the budget, which
+                // happens only after a wait elsewhere already failed
+                for (int c = max(c_end - kMlaStages, 0); c < c_end; ++c)
+                    mbar_wait(&sm.full[c % kMlaStages], static_cast<uint32_t>(c / kMlaStages) & 1u, a.wait_budget);
             }
         } else if (warp >= kGatherWarp0) {
             // ------------------------------------------ row gathers (cp.async)
@@ -334,14 +344,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             // pass 2: V tiles reuse the pass-1 area once every pass-1 MMA is
             // done.  Thread gt owns row r = gt / 4 of every tile and its
             // pieces u, u + 4, ..., u + 60 (u = gt % 4): one row lookup per tile.
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0) && !sm.abort);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0, a.wait_budget) && !sm.abort);
             const int vr = gt >> 2, vu = gt & 3;
             const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
             for (int vt = 0; vt < nvt + kVLag; ++vt) {
                 if (vt < nvt) {
                     const int v = vt % kMlaVStages;
                     const uint32_t ph = (vt / kMlaVStages) & 1;
-                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1) && !sm.abort);
+                    ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1, a.wait_budget) && !sm.abort);
                     if (ok) {
                         uint8_t *vdst = vring + v * kVTileBytes + vr * 128;
                         const uint16_t *vsrc = a.kv + static_cast<int64_t>(sm.rows[vt * kMlaVRows + vr]) * a.kv_row_stride;
@@ -369,7 +379,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             // second epilogue group: value columns 256..511
             const int hrow = (warp & 3) * 32 + lane;
             const uint32_t lane_addr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-            ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0) && !sm.abort);
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, a.wait_budget) && !sm.abort);
             // inv_l of every head is in shared memory; both groups agree on ok
             // (the epilogue's named barriers need all 128 threads of a group)
             ok = bar_and(3, 256, ok);
@@ -386,7 +396,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 for (int c = 0; c < kNumKChunks; ++c) {
                     const int s = c % kMlaStages;
                     const uint32_t ph = (c / kMlaStages) & 1;
-                    if (sm.abort || !mbar_wait(&sm.full[s], ph)) {
+                    if (sm.abort || !mbar_wait(&sm.full[s], ph, a.wait_budget)) {
                         ok = false;
                         break;
                     }
@@ -402,7 +412,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     tc_commit(&sm.empty[s]);
                 }
                 tc_commit(&sm.s_full);
-                if (ok && mbar_wait(&sm.p_full, 0) && !sm.abort) {
+                if (ok && mbar_wait(&sm.p_full, 0, a.wait_budget) && !sm.abort) {
                     tc_fence_after();
                     // B = V tile, MN-major: LBO = distance between 64-column
                     // blocks, SBO = 1 KB between 8-row groups.  A = P_hi, P_lo:
@@ -412,7 +422,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     for (int vt = 0; vt < nvt; ++vt) {
                         const int v = vt % kMlaVStages;
                         const uint32_t ph = (vt / kMlaVStages) & 1;
-                        if (sm.abort || !mbar_wait(&sm.v_full[v], ph)) {
+                        if (sm.abort || !mbar_wait(&sm.v_full[v], ph, a.wait_budget)) {
                             ok = false;
                             break;
                         }
@@ -442,13 +452,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                     record_status(a.status, DSA_ERR_TIMEOUT);
                     sm.abort = 1;
                 }
+                // every MMA issued completes (o_full's phase) before TMEM is freed
+                if (!mbar_wait(&sm.o_full, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else if (warp < 4) {
             // ------------------- pass-1 gathers, softmax, then epilogue
             bool ok = gather_pass1(a, sm, ring, tid, Rp);
             const int hrow = warp * 32 + lane;  // head = TMEM lane
             const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.s_full, 0) && !sm.abort);
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.s_full, 0, a.wait_budget) && !sm.abort);
             float m = -INFINITY, l = 0.f;
             if (ok) {
                 tc_fence_after();
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             const bool has = l > 0.f;
             const float inv_l = has ? 1.f / l : 0.f;
             sm.inv_l[hrow] = inv_l;
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0) && !sm.abort);
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.o_full, 0, a.wait_budget) && !sm.abort);
             ok = bar_and(3, 256, ok);  // hand inv_l to the second group; agree on ok
             if (ok) {
                 tc_fence_after();
