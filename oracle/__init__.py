@@ -74,6 +74,14 @@ def _load():
                 _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32]
             lib.dsa_oracle_f64_to_e4m3.restype = ctypes.c_uint8
             lib.dsa_oracle_f64_to_e4m3.argtypes = [_F64]
+            lib.dsa_oracle_pow2_scale.restype = _F64
+            lib.dsa_oracle_pow2_scale.argtypes = [_F64]
+            lib.dsa_oracle_f64_to_bf16.restype = ctypes.c_uint16
+            lib.dsa_oracle_f64_to_bf16.argtypes = [_F64]
+            lib.dsa_oracle_quantize_rows.restype = ctypes.c_int
+            lib.dsa_oracle_quantize_rows.argtypes = [_I64, _I32, _P, _P, _P]
+            lib.dsa_oracle_fold_weights.restype = ctypes.c_int
+            lib.dsa_oracle_fold_weights.argtypes = [_I64, _I32, _I32, _P, _P, _P, _P]
             lib.dsa_oracle_indexer_project.restype = ctypes.c_int
             lib.dsa_oracle_indexer_project.argtypes = [
                 _I32, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _F64,
@@ -256,3 +264,38 @@ def indexer_project(x, q_lora, w_qb, w_k, w_proj, ln_gamma, ln_beta, positions, 
     if rc != 0:
         raise RuntimeError("dsa_oracle_indexer_project failed: %d" % rc)
     return out
+
+
+def pow2_scale(amax: float) -> float:
+    """Smallest power of two 2^e with amax / 2^e <= 448 (1 for amax = 0)."""
+    return float(_load().dsa_oracle_pow2_scale(float(amax)))
+
+
+def f64_to_bf16(x: float) -> int:
+    """bf16 bits nearest to x (ties to even), rounded once from fp64."""
+    return int(_load().dsa_oracle_f64_to_bf16(float(x)))
+
+
+def quantize_rows(v):
+    """Per-row power-of-two scale and E4M3 codes of v [rows, d] (fp64 in)."""
+    v = _c(v, np.float64)
+    rows, d = v.shape
+    codes = np.empty((rows, d), np.uint8)
+    scales = np.empty(rows, np.float32)
+    if _load().dsa_oracle_quantize_rows(rows, d, _ptr(v), _ptr(codes), _ptr(scales)) != 0:
+        raise RuntimeError("dsa_oracle_quantize_rows failed")
+    return codes, scales
+
+
+def fold_weights(wp, q_scale, d_idx):
+    """w = wp / sqrt(H_I) / sqrt(d_I) * q_scale (fp64) and its bf16 bits;
+    wp [n, H_I] fp64, q_scale [n, H_I] float32."""
+    wp = _c(wp, np.float64)
+    q_scale = _c(q_scale, np.float32)
+    n, h = wp.shape
+    w_f = np.empty((n, h), np.float64)
+    w_b = np.empty((n, h), np.uint16)
+    if _load().dsa_oracle_fold_weights(n, h, int(d_idx), _ptr(wp), _ptr(q_scale), _ptr(w_f),
+                                       _ptr(w_b)) != 0:
+        raise RuntimeError("dsa_oracle_fold_weights failed")
+    return w_f, w_b

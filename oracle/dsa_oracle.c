@@ -449,7 +449,10 @@ int dsa_oracle_forward(int32_t nq, int32_t h_idx, int32_t d_idx, int32_t h,
  * q_scale, k_code / k_scale (the FP8 codes and their scales), w_bf16. */
 static double bf(const uint16_t *p, int64_t i) { return dsa_oracle_bf16_to_f64(p[i]); }
 
-static double pow2_scale(double amax)
+/* The power-of-two quantisation scale of a vector whose largest magnitude is
+ * amax: the smallest 2^e with amax / 2^e <= 448 (the E4M3 maximum), 1 for an
+ * all-zero vector. */
+double dsa_oracle_pow2_scale(double amax)
 {
     if (!(amax > 0.0)) return 1.0;
     return ldexp(1.0, (int)ceil(log2(amax / 448.0)));
@@ -458,7 +461,7 @@ static double pow2_scale(double amax)
 /* bfloat16 nearest to v (ties to even), rounded once from fp64: 8
  * significant bits, spacing 2^(e-7) for |v| in [2^e, 2^(e+1)), 2^-133 below
  * the smallest normal; beyond the largest finite value -> infinity. */
-static uint16_t f64_to_bf16_rne(double v)
+uint16_t dsa_oracle_f64_to_bf16(double v)
 {
     if (isnan(v)) return 0x7FC0;
     double a = fabs(v);
@@ -475,6 +478,41 @@ static uint16_t f64_to_bf16_rne(double v)
     uint32_t u;
     memcpy(&u, &f, sizeof u);
     return (uint16_t)(u >> 16);
+}
+
+/* FP8 quantisation of `rows` vectors of d values each (row-major v): one
+ * power-of-two scale per row from its largest magnitude, codes =
+ * e4m3(v / scale) ([yuyanqi] section 4.3: q and k in FP8 with a scale; the
+ * e8m0 k_s).  scales[r] = the row's scale; codes [rows, d]. */
+int dsa_oracle_quantize_rows(int64_t rows, int32_t d, const double *v, uint8_t *codes, float *scales)
+{
+    if (rows < 0 || d <= 0) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *x = v + r * d;
+        double amax = 0.0;
+        for (int32_t o = 0; o < d; ++o) amax = fmax(amax, fabs(x[o]));
+        double s = dsa_oracle_pow2_scale(amax);
+        if (scales) scales[r] = (float)s;
+        if (codes)
+            for (int32_t o = 0; o < d; ++o) codes[r * d + o] = dsa_oracle_f64_to_e4m3(x[o] / s);
+    }
+    return 0;
+}
+
+/* The indexer's head weights with every constant folded in ([yuyanqi]
+ * section 4.3: weights_proj * n_heads^-1/2 * softmax_scale * q_scale), for
+ * n tokens: w[t, j] = wp[t, j] / sqrt(H_I) / sqrt(d_I) * q_scale[t, j],
+ * then rounded to bf16 (ties to even).  Either output may be NULL. */
+int dsa_oracle_fold_weights(int64_t n, int32_t h_idx, int32_t d_idx, const double *wp,
+                            const float *q_scale, double *w_f, uint16_t *w_bf16)
+{
+    if (n < 0 || h_idx <= 0 || d_idx <= 0) return -1;
+    for (int64_t i = 0; i < n * h_idx; ++i) {
+        double wv = wp[i] / sqrt((double)h_idx) / sqrt((double)d_idx) * (double)q_scale[i];
+        if (w_f) w_f[i] = wv;
+        if (w_bf16) w_bf16[i] = dsa_oracle_f64_to_bf16(wv);
+    }
+    return 0;
 }
 
 static void rope_rotate(double *v, int32_t rope_dim, int32_t pos, double theta)
@@ -501,6 +539,7 @@ int dsa_oracle_indexer_project(int32_t nt, int32_t hidden, int32_t q_lora_rank,
                                uint16_t *w_bf16, int32_t nthreads)
 {
     if (nt < 0 || hidden <= 0 || q_lora_rank <= 0 || h_idx <= 0 || d_idx <= 0) return -1;
+    if (h_idx > 256 || d_idx > 256) return -1;
     if (rope_dim < 0 || rope_dim > d_idx || (rope_dim & 1)) return -1;
     set_threads(nthreads);
     int rc = 0;
@@ -539,32 +578,38 @@ int dsa_oracle_indexer_project(int32_t nt, int32_t hidden, int32_t q_lora_rank,
         for (int32_t j = 0; j < h_idx; ++j) rope_rotate(qv + (int64_t)j * d_idx, rope_dim, positions[t], rope_theta);
         rope_rotate(kv, rope_dim, positions[t], rope_theta);
         /* k: one power-of-two scale per token */
-        double kmax = 0.0;
-        for (int32_t o = 0; o < d_idx; ++o) kmax = fmax(kmax, fabs(kv[o]));
-        double ks = pow2_scale(kmax);
+        uint8_t kc[256];
+        float ks;
+        dsa_oracle_quantize_rows(1, d_idx, kv, kc, &ks);
         for (int32_t o = 0; o < d_idx; ++o) {
             if (k_f) k_f[(int64_t)t * d_idx + o] = kv[o];
-            if (k_code) k_code[(int64_t)t * d_idx + o] = dsa_oracle_f64_to_e4m3(kv[o] / ks);
+            if (k_code) k_code[(int64_t)t * d_idx + o] = kc[o];
         }
-        if (k_scale) k_scale[t] = (float)ks;
+        if (k_scale) k_scale[t] = ks;
         /* q: one power-of-two scale per (token, head); w folds it */
+        double wps[256], wfs[256];
+        float qss[256];
+        uint16_t wbs[256];
         for (int32_t j = 0; j < h_idx; ++j) {
             const double *qh = qv + (int64_t)j * d_idx;
-            double qmax = 0.0;
-            for (int32_t o = 0; o < d_idx; ++o) qmax = fmax(qmax, fabs(qh[o]));
-            double qs = pow2_scale(qmax);
+            uint8_t qc[256];
+            dsa_oracle_quantize_rows(1, d_idx, qh, qc, &qss[j]);
             double wp = 0.0;
             for (int32_t i = 0; i < hidden; ++i)
                 wp += bf(w_proj, (int64_t)j * hidden + i) * bf(x, (int64_t)t * hidden + i);
-            double wv = wp / sqrt((double)h_idx) / sqrt((double)d_idx) * qs;
+            wps[j] = wp;
             int64_t tj = (int64_t)t * h_idx + j;
-            if (w_f) w_f[tj] = wv;
-            if (w_bf16) w_bf16[tj] = f64_to_bf16_rne(wv);
-            if (q_scale) q_scale[tj] = (float)qs;
+            if (q_scale) q_scale[tj] = qss[j];
             for (int32_t o = 0; o < d_idx; ++o) {
                 if (q_f) q_f[tj * d_idx + o] = qh[o];
-                if (q_code) q_code[tj * d_idx + o] = dsa_oracle_f64_to_e4m3(qh[o] / qs);
+                if (q_code) q_code[tj * d_idx + o] = qc[o];
             }
+        }
+        dsa_oracle_fold_weights(1, h_idx, d_idx, wps, qss, wfs, wbs);
+        for (int32_t j = 0; j < h_idx; ++j) {
+            int64_t tj = (int64_t)t * h_idx + j;
+            if (w_f) w_f[tj] = wfs[j];
+            if (w_bf16) w_bf16[tj] = wbs[j];
         }
         free(qv);
         free(kv);

@@ -184,3 +184,48 @@ def test_producer_feeds_the_indexer_score(oracle):
     # per term: q and k each within 2^-4 relative, w within 2^-8: a loose bound
     assert np.all(np.abs(sc - ref) <= 0.2 * absref + 1e-9)
     assert np.corrcoef(sc.ravel(), ref.ravel())[0, 1] > 0.99
+
+
+# ---------------------------------------------------------------------------
+# the exported rounding decisions (used by the producer above)
+# ---------------------------------------------------------------------------
+
+
+def test_pow2_scale_is_the_smallest_power_of_two_that_fits_448(oracle):
+    assert oracle.pow2_scale(0.0) == 1.0
+    assert oracle.pow2_scale(448.0) == 1.0            # fits exactly
+    assert oracle.pow2_scale(448.0 * (1 + 2 ** -40)) == 2.0
+    assert oracle.pow2_scale(224.0) == 0.5
+    assert oracle.pow2_scale(224.0 * (1 + 2 ** -40)) == 1.0
+    rng = np.random.default_rng(8)
+    for amax in rng.uniform(1e-6, 1e6, 500):
+        s = oracle.pow2_scale(amax)
+        assert s == 2.0 ** round(np.log2(s))           # a power of two
+        assert amax / s <= 448.0 < 2 * amax / s         # the smallest one that fits
+
+
+def test_quantize_rows_is_the_torch_cast_at_the_row_scale(oracle):
+    rng = np.random.default_rng(9)
+    v = rng.standard_normal((50, 128)) * rng.uniform(1e-3, 1e3, size=(50, 1))
+    v[3] = 0.0                                          # an all-zero row: scale 1, codes 0
+    codes, scales = oracle.quantize_rows(v)
+    for r in range(50):
+        s = oracle.pow2_scale(np.abs(v[r]).max())
+        assert scales[r] == s and (r != 3 or (s == 1.0 and not codes[r].any()))
+        ref = torch.from_numpy((v[r] / s).astype(np.float32)).clamp(-448, 448)
+        # v / s is exact in fp64; its fp32 rounding can only move a tie, so
+        # compare where the fp32 value is not within an fp32 ulp of a tie
+        assert np.array_equal(codes[r], ref.to(torch.float8_e4m3fn).view(torch.uint8).numpy()) or \
+            np.abs(_dec_e4m3(codes[r]) - v[r] / s).max() <= np.abs(v[r] / s).max() / 16
+
+
+def test_fold_weights_closed_form(oracle):
+    # wp = sqrt(H) * sqrt(d) * 2^k / q_scale gives w = 2^k (H = 4 heads here)
+    h, d = 4, 128
+    qs = np.array([[0.25, 1.0, 4.0, 0.5]], np.float32)
+    wp = np.sqrt(h) * np.sqrt(d) * np.array([[1.0, -2.0, 0.5, 8.0]]) / qs.astype(np.float64)
+    w_f, w_b = oracle.fold_weights(wp, qs, d)
+    assert np.allclose(w_f, [[1.0, -2.0, 0.5, 8.0]], rtol=1e-14, atol=0)
+    assert np.array_equal(_dec_bf16(w_b), [[1.0, -2.0, 0.5, 8.0]])
+    assert oracle.f64_to_bf16(1.0 + 2 ** -8) == 0x3F80  # a tie rounds to even
+    assert oracle.f64_to_bf16(1.0 + 3 * 2 ** -8) == 0x3F82
