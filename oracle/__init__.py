@@ -74,6 +74,10 @@ def _load():
                 _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32]
             lib.dsa_oracle_f64_to_e4m3.restype = ctypes.c_uint8
             lib.dsa_oracle_f64_to_e4m3.argtypes = [_F64]
+            lib.dsa_oracle_index_kl.restype = ctypes.c_int
+            lib.dsa_oracle_index_kl.argtypes = [
+                _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _I64, _P,
+                _I32, _P, _P, _I32]
             lib.dsa_oracle_pow2_scale.restype = _F64
             lib.dsa_oracle_pow2_scale.argtypes = [_F64]
             lib.dsa_oracle_f64_to_bf16.restype = ctypes.c_uint16
@@ -299,3 +303,30 @@ def fold_weights(wp, q_scale, d_idx):
                                        _ptr(w_b)) != 0:
         raise RuntimeError("dsa_oracle_fold_weights failed")
     return w_f, w_b
+
+
+def index_kl(q, kv, q_seq, q_n, index_scores, *, scale, idx=None, seq_row0=None, page_table=None,
+             page_size=0, with_p=False, nthreads=0):
+    """Indexer distillation loss per query (fp64): KL(p || softmax(I)) over every
+    visible position (idx None: the dense stage) or over idx's valid entries
+    (the sparse stage); p = the heads' attention distributions summed over
+    heads and L1-normalised.  index_scores [nq, ld] fp64.  Returns kl [nq]
+    (and p [nq, ld] with with_p)."""
+    q = _c(q, np.uint16)
+    nq, h, d_qk = q.shape
+    kv = _c(kv, np.uint16)
+    index_scores = _c(index_scores, np.float64)
+    ld = index_scores.shape[1]
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    idx = _c(idx, np.int32)
+    k = idx.shape[1] if idx is not None else 0
+    kl = np.empty(nq, np.float64)
+    p = np.empty((nq, ld), np.float64) if with_p else None
+    rc = _load().dsa_oracle_index_kl(nq, h, d_qk, float(scale), _ptr(q), _ptr(kv), kv.shape[1],
+                                     _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table),
+                                     max_pages, page_size, _ptr(index_scores), ld, _ptr(idx), k,
+                                     _ptr(kl), _ptr(p), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_index_kl failed: %d" % rc)
+    return (kl, p) if with_p else kl

@@ -421,6 +421,102 @@ int dsa_oracle_forward(int32_t nq, int32_t h_idx, int32_t d_idx, int32_t h,
 }
 
 /* ------------------------------------------------------------------------- */
+/* The indexer's training signal, forward only                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Indexer distillation loss of each query t ([marsggbo] section 5.1 and 5.2):
+ * over a set of positions T_t (the dense stage: every visible s < q_n[t],
+ * when idx is NULL; the sparse stage: the valid entries of idx[t, :], a
+ * position listed twice counting twice),
+ *   A_h[s] = exp(S_h[s]) / sum_{s' in T_t} exp(S_h[s']),
+ *            S_h[s] = scale * q[t, h] . c[s]        (each head's attention)
+ *   p[s]   = sum_h A_h[s] / sum_{s' in T_t} sum_h A_h[s']
+ *            (the heads' scores summed over the head dimension, then L1-
+ *            normalised along the sequence)
+ *   r[s]   = exp(I[t, s]) / sum_{s' in T_t} exp(I[t, s'])   (softmax of the
+ *            index scores over the same set)
+ *   kl[t]  = sum_{s in T_t} p[s] * (ln p[s] - ln r[s])      (0 ln 0 = 0)
+ * Reading where the page is silent: in the sparse stage the main model
+ * attends to T_t only, so each head's distribution is normalised over T_t.
+ * index_scores [nq, ld] holds I[t, s] at column s (fp64); p_out, when not
+ * NULL, receives p[s] at column s ([nq, ld]; other columns 0).  A query with
+ * an empty set gets kl = 0. */
+int dsa_oracle_index_kl(int32_t nq, int32_t h, int32_t d_qk, double scale, const uint16_t *q,
+                        const uint16_t *kv, int64_t kv_row_stride, const int32_t *q_seq,
+                        const int32_t *q_n, const int64_t *seq_row0, const int32_t *page_table,
+                        int32_t max_pages, int32_t page_size, const double *index_scores,
+                        int64_t ld, const int32_t *idx, int32_t k, double *kl, double *p_out,
+                        int32_t nthreads)
+{
+    if (nq < 0 || h <= 0 || d_qk <= 0 || ld < 0 || (idx && k < 0)) return -1;
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        int64_t n = q_n[qi];
+        int64_t cap = idx ? k : n;
+        int64_t *pos = (int64_t *)malloc((size_t)(cap > 0 ? cap : 1) * sizeof(int64_t));
+        double *S = (double *)malloc((size_t)(cap > 0 ? cap : 1) * sizeof(double));
+        double *a = (double *)malloc((size_t)(cap > 0 ? cap : 1) * sizeof(double));
+        if (!pos || !S || !a) { bad |= 1; free(pos); free(S); free(a); continue; }
+        int64_t cnt = 0;
+        if (idx) {
+            for (int32_t i = 0; i < k; ++i) {
+                int32_t sv = idx[(int64_t)qi * k + i];
+                if (sv >= 0 && sv < n && sv < ld) pos[cnt++] = sv;
+            }
+        } else {
+            for (int64_t sv = 0; sv < n && sv < ld; ++sv) pos[cnt++] = sv;
+        }
+        if (p_out)
+            for (int64_t c = 0; c < ld; ++c) p_out[(int64_t)qi * ld + c] = 0.0;
+        if (cnt == 0) {
+            kl[qi] = 0.0;
+            free(pos); free(S); free(a);
+            continue;
+        }
+        for (int64_t i = 0; i < cnt; ++i) a[i] = 0.0;
+        /* each head's distribution over the set, summed over heads */
+        for (int32_t hh = 0; hh < h; ++hh) {
+            const uint16_t *qv = q + ((int64_t)qi * h + hh) * d_qk;
+            double m = -INFINITY;
+            for (int64_t i = 0; i < cnt; ++i) {
+                const uint16_t *c = kv + cache_row(q_seq[qi], pos[i], seq_row0, page_table,
+                                                   max_pages, page_size) * kv_row_stride;
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_qk; ++d)
+                    dot += dsa_oracle_bf16_to_f64(qv[d]) * dsa_oracle_bf16_to_f64(c[d]);
+                S[i] = scale * dot;
+                if (S[i] > m) m = S[i];
+            }
+            double z = 0.0;
+            for (int64_t i = 0; i < cnt; ++i) z += exp(S[i] - m);
+            for (int64_t i = 0; i < cnt; ++i) a[i] += exp(S[i] - m) / z;
+        }
+        /* L1 normalisation along the sequence */
+        double asum = 0.0;
+        for (int64_t i = 0; i < cnt; ++i) asum += a[i];
+        /* softmax of the index scores over the same set */
+        const double *I = index_scores + (int64_t)qi * ld;
+        double mi = -INFINITY;
+        for (int64_t i = 0; i < cnt; ++i)
+            if (I[pos[i]] > mi) mi = I[pos[i]];
+        double zi = 0.0;
+        for (int64_t i = 0; i < cnt; ++i) zi += exp(I[pos[i]] - mi);
+        const double lse_i = mi + log(zi);
+        double acc = 0.0;
+        for (int64_t i = 0; i < cnt; ++i) {
+            double p = a[i] / asum;
+            if (p_out) p_out[(int64_t)qi * ld + pos[i]] += p;
+            if (p > 0.0) acc += p * (log(p) - (I[pos[i]] - lse_i));
+        }
+        kl[qi] = acc;
+        free(pos); free(S); free(a);
+    }
+    return bad ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Next step on the path: the indexer's q^I / k^I / w producer                 */
 /* ------------------------------------------------------------------------- */
 
