@@ -182,8 +182,9 @@ int dsa_indexer_topk(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  * Arithmetic: bf16 tensor-core products with fp32 accumulation; softmax in
  * fp32; P enters the P.V product as a pair of bf16 tiles (P_hi + P_lo,
  * together exact to about 2^-16).  When a query's rows are split over
- * several CTAs, each split's normalised output is kept in ws as fp16 and
- * the splits are merged by their log-sum-exp. */
+ * several CTAs, each split's normalised output is kept in ws as fp16 times
+ * a power-of-two scale per 64 value columns (so any finite bf16 latent keeps
+ * fp16's 11-bit precision) and the splits are merged by their log-sum-exp. */
 int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q,
                           const void *kv_cache, int64_t kv_row_stride,
                           const int32_t *idx, void *out, float *lse, void *ws,
@@ -214,6 +215,67 @@ int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
                       const void *q, const void *kv_cache, int64_t kv_row_stride,
                       void *out, float *lse, int32_t *idx_out, void *ws,
                       size_t ws_bytes, void *stream);
+
+/* The indexer's own inputs, produced from the hidden state and the low-rank
+ * query ("DeepSeekV3.2之DSA" by yuyanqi, sections 4.1-4.3), with k^I
+ * appended to the index-K cache (the decode data flow of its section 5.1).
+ * For every token t:
+ *   q^I[t] = W_qb . q_lora[t] as [h_idx, d_idx]             (wq_b)
+ *   k^I[t] = LayerNorm(W_k . x[t]) * ln_gamma + ln_beta      (wk, k_norm;
+ *            biased variance, epsilon ln_eps)
+ *   RoPE on the first rope_dim dims of every q^I head and of k^I: the pair
+ *            (2i, 2i+1) rotated by positions[t] * rope_theta^(-2i / rope_dim)
+ *   q_scale[t, j] / k_scale = the smallest power of two s with amax / s <= 448
+ *            (the e8m0 k_s of section 4.3; per (token, head) for q, per
+ *            token for k), codes = e4m3(value / s) (ties to even, saturating)
+ *   w[t, j] = (W_proj . x[t])_j / sqrt(h_idx) / sqrt(d_idx) * q_scale[t, j],
+ *            rounded to bf16 (weights_proj with n_heads^-1/2, the softmax
+ *            scale d_I^-1/2 and the q scale folded in: the form the indexer
+ *            score takes, with no factor of its own)
+ * Shapes: nt tokens; hidden = width of x, q_lora_rank = width of q_lora (both
+ * multiples of 8); h_idx 1..64; d_idx 64 or 128; rope_dim even, <= d_idx. */
+typedef struct {
+    int32_t nt;
+    int32_t hidden;
+    int32_t q_lora_rank;
+    int32_t h_idx;
+    int32_t d_idx;
+    int32_t rope_dim;
+    float ln_eps;
+    float rope_theta;
+} dsa_project_params;
+
+/* Bytes of `ws` dsa_indexer_project needs (host only). */
+int dsa_project_workspace_size(const dsa_project_params *pp, size_t *bytes);
+
+/* Produce q^I, w and k^I of nt tokens and append k^I to the cache.
+ *   kv         where each token's k^I row goes: kv->q_seq [nt] is the token's
+ *              sequence and positions[t] its position; the row follows
+ *              kv->seq_row0 / kv->page_table as for the score (kv->q_n is not
+ *              read).  A row outside [0, cache_rows) flags DSA_ERR_DEVICE_CHECK
+ *              and is not written.
+ *   x          [nt, hidden] bf16;  q_lora [nt, q_lora_rank] bf16
+ *   w_qb       [h_idx * d_idx, q_lora_rank] bf16; w_k [d_idx, hidden] bf16;
+ *   w_proj     [h_idx, hidden] bf16  (all [out, in], 16-byte aligned)
+ *   ln_gamma, ln_beta [d_idx] fp32;  positions [nt] int32
+ *   q_idx      [nt, h_idx, d_idx] e4m3 output (the indexer's q_idx input)
+ *   q_scale    [nt, h_idx] fp32 output, or NULL
+ *   w          [nt, h_idx] bf16 output (the indexer's w input)
+ *   kidx_cache [cache_rows, d_idx] e4m3: row of token t overwritten
+ *   k_scale    [cache_rows] fp32: entry of token t's row overwritten (pass the
+ *              same array to the score as its k_scale)
+ *   q_f32, k_f32, w_f32: [nt, h_idx, d_idx], [nt, d_idx], [nt, h_idx] fp32
+ *              outputs of the values before rounding (after RoPE; w before
+ *              folding), or NULL
+ * Arithmetic: bf16 tensor-core products with fp32 accumulation (a split of
+ * the K dimension is summed in a fixed order); LayerNorm and the rounding
+ * decisions in fp32, RoPE angles and the weight folding in fp64. */
+int dsa_indexer_project(const dsa_project_params *pp, const dsa_kv *kv, const void *x,
+                        const void *q_lora, const void *w_qb, const void *w_k, const void *w_proj,
+                        const float *ln_gamma, const float *ln_beta, const int32_t *positions,
+                        void *q_idx, float *q_scale, void *w, void *kidx_cache, float *k_scale,
+                        float *q_f32, float *k_f32, float *w_f32, void *ws, size_t ws_bytes,
+                        void *stream);
 
 /* dsa_indexer_topk without a workspace, for callers that cannot allocate
  * device memory (their allocator owns the device, they run under a fixed

@@ -130,7 +130,7 @@ int check_kv(const dsa_params *p, const dsa_kv *kv) {
 
 // ----------------------------------------------------------------- planning
 struct IndexerPlan {
-    int hp, qg, gpb, n_groups, P, chunk, stages, acc_bufs;
+    int hp, qg, gpb, n_groups, P, n_big, chunk, stages, acc_bufs;
     bool parallel;  // fused, several chunks, every CTA resident: each chunk selects its own part
     uint32_t tmem_cols;
     size_t smem;
@@ -163,14 +163,26 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     if (P < p_min) P = p_min;
     if (P < 1) P = 1;
     pl.parallel = false;
+    pl.n_big = pl.n_groups;
+    int64_t p_cut = 0;  // chunk count the chunk size is planned for (0: P)
     if (mode != dsa::kModeScores) {
         // Parallel selection (fused, the grid resident at once) keeps no
-        // merge list in one CTA: up to kMaxChunks chunks.  Otherwise the
-        // last CTA's merge list (P * topk composites) must fit on chip.
+        // merge list in one CTA: up to kMaxChunks chunks, and the SMs left
+        // over give some groups one chunk more (every SM streams).
+        // Otherwise the last CTA's merge list (P * topk composites) must
+        // fit on chip.
         const int64_t p_par = P < dsa::kMaxChunks ? P : dsa::kMaxChunks;
+        const int64_t sms = num_sms();
         if (mode == dsa::kModeFused && p_par > 1 && p_par >= p_min &&
-            static_cast<int64_t>(pl.n_groups) * p_par <= num_sms()) {
-            P = p_par;
+            static_cast<int64_t>(pl.n_groups) * p_par <= sms) {
+            int64_t extra = 0;
+            if (DSA_K1_FILL_SMS && p_par < dsa::kMaxChunks && p_par < p_small) {
+                extra = sms - static_cast<int64_t>(pl.n_groups) * p_par;
+                if (extra > pl.n_groups) extra = pl.n_groups;
+            }
+            P = extra > 0 ? p_par + 1 : p_par;
+            pl.n_big = extra > 0 ? static_cast<int>(extra) : pl.n_groups;
+            p_cut = p_par;
             pl.parallel = true;
         } else {
             int64_t p_cap = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
@@ -181,10 +193,18 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
             }
         }
     }
-    int64_t chunk = (sp + P - 1) / P;
-    chunk = (chunk + 127) / 128 * 128;
+    // chunks are whole ring stages; each group cuts its own span the same
+    // way on the device (no larger than this)
+    const int64_t srows = 128 * DSA_K1_STAGE_TILES;
+    chunk_max = chunk_max / srows * srows;
+    const int64_t pc = p_cut > 0 ? p_cut : P;
+    int64_t chunk = (sp + pc - 1) / pc;
+    chunk = (chunk + srows - 1) / srows * srows;
     if (chunk > chunk_max) chunk = chunk_max;
-    P = (sp + chunk - 1) / chunk;
+    if (p_cut == 0) {
+        P = (sp + chunk - 1) / chunk;
+        pl.n_big = pl.n_groups;
+    }
     if (P <= 1) pl.parallel = false;
     pl.P = static_cast<int>(P);
     pl.chunk = static_cast<int>(chunk);
@@ -205,7 +225,7 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     // (the merge area reuses the ring once streaming is over)
     pl.stages = 0;
     if (mode != dsa::kModeTopk) {
-        int st = dsa::kK1MaxStages;
+        int st = dsa::kK1WantStages;
         while (st >= 2 &&
                dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st, !pl.parallel).total > 232448)
             --st;
@@ -242,7 +262,7 @@ MlaPlan plan_mla(const dsa_params *p) {
     if (m.splits == 1) {
         m.wave = p->nq;
     } else {
-        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv * 2 + 4 + 8);
+        const size_t per_q = static_cast<size_t>(m.splits) * 128 * (dsa::kDv * 2 + 4 + 4 * dsa::kMlaScaleBlocks);
         size_t w = kPartialBudget / per_q;
         if (w < 1) w = 1;
         m.wave = p->nq < static_cast<int>(w) ? p->nq : static_cast<int>(w);
@@ -289,7 +309,7 @@ size_t mla_ws(const dsa_params *p, const MlaPlan &m, size_t off, WsLayout &w) {
     w.part_lse = off;
     off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 4, 256);
     w.part_scale = off;
-    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * 2 * 4, 256);
+    off = up(off + static_cast<size_t>(m.wave) * m.splits * 128 * dsa::kMlaScaleBlocks * 4, 256);
     return off;
 }
 
@@ -372,6 +392,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.groups_per_block = pl.gpb;
     a.n_groups = pl.n_groups;
     a.P = pl.P;
+    a.n_big = pl.n_big;
     a.chunk = pl.chunk;
     a.stages = pl.stages;
     a.acc_bufs = pl.acc_bufs;
@@ -418,7 +439,8 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.page_size = kv->page_table ? kv->page_size : 0;
     a.cache_rows = kv->cache_rows;
     CUtensorMap kmap;
-    const uint32_t box_rows = kv->page_table ? static_cast<uint32_t>(kv->page_size) : 128u;
+    // one box per ring stage, or one per page
+    const uint32_t box_rows = kv->page_table ? static_cast<uint32_t>(kv->page_size) : 128u * DSA_K1_STAGE_TILES;
     int rc = make_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, kidx_cache, p->d_idx, kv->cache_rows,
                          p->d_idx, p->d_idx, box_rows,
                          p->d_idx == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
@@ -448,6 +470,7 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.page_size = kv->page_table ? kv->page_size : 0;
     a.cache_rows = kv->cache_rows;
     a.idx = idx;
+    a.q = static_cast<const uint16_t *>(q);
     a.kv = static_cast<const uint16_t *>(kv_cache);
     a.kv_row_stride = kv_row_stride;
     a.nq = p->nq;
@@ -495,6 +518,59 @@ int check_mla_inputs(const dsa_params *p, const void *q, const void *kv_cache, i
         return fail(DSA_ERR_INVALID_ARG, "q / kv_cache / out must be 16-byte aligned");
     if (stride < 576 || stride % 8 != 0) return fail(DSA_ERR_INVALID_ARG, "kv_row_stride must be >= 576 and a multiple of 8");
     return DSA_OK;
+}
+
+// ------------------------------------------------------- indexer producer
+struct ProjPlan {
+    int m_tiles, k_steps[2], n_cols[2], n_tiles[2], splits[2], ld[2];
+    size_t part_off[2], total;
+};
+
+int check_project(const dsa_project_params *pp) {
+    if (!pp) return fail(DSA_ERR_INVALID_ARG, "params is NULL");
+    if (pp->nt < 0) return fail(DSA_ERR_INVALID_ARG, "nt < 0");
+    if (pp->h_idx < 1 || pp->h_idx > 64) return fail(DSA_ERR_INVALID_ARG, "h_idx must be in [1, 64]");
+    if (pp->d_idx != 64 && pp->d_idx != 128) return fail(DSA_ERR_INVALID_ARG, "d_idx must be 64 or 128");
+    if (pp->rope_dim < 0 || pp->rope_dim > pp->d_idx || (pp->rope_dim & 1))
+        return fail(DSA_ERR_INVALID_ARG, "rope_dim must be even and in [0, d_idx]");
+    if (pp->hidden < 8 || pp->hidden % 8 || pp->q_lora_rank < 8 || pp->q_lora_rank % 8)
+        return fail(DSA_ERR_INVALID_ARG, "hidden and q_lora_rank must be positive multiples of 8");
+    if (!(pp->ln_eps >= 0.f) || !isfinite(pp->rope_theta) || !(pp->rope_theta > 0.f))
+        return fail(DSA_ERR_INVALID_ARG, "ln_eps must be >= 0 and rope_theta > 0");
+    return DSA_OK;
+}
+
+// K slices so that the grid fills the SMs when few token tiles exist, in
+// proportion to each problem's weight bytes (decode streams the weights).
+ProjPlan plan_project(const dsa_project_params *pp) {
+    ProjPlan pl;
+    pl.m_tiles = (pp->nt + 127) / 128;
+    pl.k_steps[0] = (pp->hidden + 63) / 64;
+    pl.k_steps[1] = (pp->q_lora_rank + 63) / 64;
+    pl.n_cols[0] = (pp->d_idx + pp->h_idx + 15) / 16 * 16;
+    pl.n_cols[1] = 128;
+    pl.n_tiles[0] = 1;
+    pl.n_tiles[1] = (pp->h_idx * pp->d_idx + 127) / 128;
+    pl.ld[0] = (pp->d_idx + pp->h_idx + 3) & ~3;
+    pl.ld[1] = pp->h_idx * pp->d_idx;
+    const double b0 = static_cast<double>(pp->d_idx + pp->h_idx) * pp->hidden;
+    const double b1 = static_cast<double>(pp->h_idx) * pp->d_idx * pp->q_lora_rank;
+    const int sms = num_sms();
+    const int base0 = pl.m_tiles, base1 = pl.m_tiles * pl.n_tiles[1];
+    int s0 = 1, s1 = 1;
+    if (pl.m_tiles > 0 && base0 + base1 < sms) {
+        s0 = static_cast<int>(sms * b0 / (b0 + b1) / base0);
+        s1 = static_cast<int>(sms * b1 / (b0 + b1) / base1);
+    }
+    pl.splits[0] = s0 < 1 ? 1 : (s0 > pl.k_steps[0] ? pl.k_steps[0] : s0);
+    pl.splits[1] = s1 < 1 ? 1 : (s1 > pl.k_steps[1] ? pl.k_steps[1] : s1);
+    size_t off = 256;  // status word
+    for (int q = 0; q < 2; ++q) {
+        pl.part_off[q] = off;
+        off = up(off + static_cast<size_t>(pl.splits[q]) * pp->nt * pl.ld[q] * 4, 256);
+    }
+    pl.total = off;
+    return pl;
 }
 
 }  // namespace
@@ -633,6 +709,106 @@ int dsa_forward_paged(const dsa_params *p, const dsa_kv *kv, const void *q_idx, 
     if (!kv || !kv->page_table) return fail(DSA_ERR_INVALID_ARG, "dsa_forward_paged needs kv->page_table");
     return dsa_forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, out, lse,
                        idx_out, ws, ws_bytes, stream);
+}
+
+int dsa_project_workspace_size(const dsa_project_params *pp, size_t *bytes) {
+    int rc = check_project(pp);
+    if (rc) return rc;
+    if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
+    *bytes = plan_project(pp).total;
+    return DSA_OK;
+}
+
+int dsa_indexer_project(const dsa_project_params *pp, const dsa_kv *kv, const void *x,
+                        const void *q_lora, const void *w_qb, const void *w_k, const void *w_proj,
+                        const float *ln_gamma, const float *ln_beta, const int32_t *positions,
+                        void *q_idx, float *q_scale, void *w, void *kidx_cache, float *k_scale,
+                        float *q_f32, float *k_f32, float *w_f32, void *ws, size_t ws_bytes,
+                        void *stream) {
+    int rc = check_project(pp);
+    if (rc) return rc;
+    if (!kv) return fail(DSA_ERR_INVALID_ARG, "kv is NULL");
+    if ((kv->seq_row0 == nullptr) == (kv->page_table == nullptr))
+        return fail(DSA_ERR_INVALID_ARG, "exactly one of seq_row0 and page_table must be set");
+    if (kv->page_table && kv->page_size != 64 && kv->page_size != 128)
+        return fail(DSA_ERR_UNSUPPORTED, "page_size must be 64 or 128");
+    if (kv->page_table && kv->max_pages < 1) return fail(DSA_ERR_INVALID_ARG, "max_pages < 1");
+    if (kv->cache_rows < 1 || kv->cache_rows >= (int64_t(1) << 31))
+        return fail(DSA_ERR_INVALID_ARG, "cache_rows must be in [1, 2^31)");
+    const ProjPlan pl = plan_project(pp);
+    if (!ws) return fail(DSA_ERR_WORKSPACE, "ws is NULL");
+    if (!aligned(ws, 256)) return fail(DSA_ERR_WORKSPACE, "ws must be 256-byte aligned");
+    if (ws_bytes < pl.total) return fail(DSA_ERR_WORKSPACE, "ws_bytes %zu < required %zu", ws_bytes, pl.total);
+    if (pp->nt == 0) return DSA_OK;
+    if (!x || !q_lora || !w_qb || !w_k || !w_proj || !ln_gamma || !ln_beta || !positions || !q_idx || !w ||
+        !kidx_cache || !k_scale || !kv->q_seq)
+        return fail(DSA_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned(x, 16) || !aligned(q_lora, 16) || !aligned(w_qb, 16) || !aligned(w_k, 16) ||
+        !aligned(w_proj, 16) || !aligned(q_idx, 4) || !aligned(kidx_cache, 4))
+        return fail(DSA_ERR_INVALID_ARG, "x, q_lora and the weights must be 16-byte aligned, q_idx and "
+                                         "kidx_cache 4-byte aligned");
+    CUtensorMap xm, qm, km, pm, wm;
+    const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    rc = make_map_2d(&xm, bf, x, pp->hidden, pp->nt, pp->hidden * 2ull, 64, 128, sw);
+    if (!rc) rc = make_map_2d(&qm, bf, q_lora, pp->q_lora_rank, pp->nt, pp->q_lora_rank * 2ull, 64, 128, sw);
+    if (!rc) rc = make_map_2d(&km, bf, w_k, pp->hidden, pp->d_idx, pp->hidden * 2ull, 64, pp->d_idx, sw);
+    if (!rc) rc = make_map_2d(&pm, bf, w_proj, pp->hidden, pp->h_idx, pp->hidden * 2ull, 64, pp->h_idx, sw);
+    if (!rc) rc = make_map_2d(&wm, bf, w_qb, pp->q_lora_rank, static_cast<uint64_t>(pp->h_idx) * pp->d_idx,
+                              pp->q_lora_rank * 2ull, 64, 128, sw);
+    if (rc) return rc;
+    dsa::ProjGemmParams g;
+    memset(&g, 0, sizeof g);
+    g.nt = pp->nt;
+    g.m_tiles = pl.m_tiles;
+    for (int q = 0; q < 2; ++q) {
+        g.k_steps[q] = pl.k_steps[q];
+        g.n_cols[q] = pl.n_cols[q];
+        g.n_tiles[q] = pl.n_tiles[q];
+        g.splits[q] = pl.splits[q];
+        g.part[q] = at<float>(ws, pl.part_off[q]);
+        g.ld[q] = pl.ld[q];
+    }
+    g.items0 = pl.m_tiles * pl.n_tiles[0] * pl.splits[0];
+    g.d_idx = pp->d_idx;
+    g.h_idx = pp->h_idx;
+    g.status = at<int>(ws, 0);
+    g.wait_budget = dsa::kWaitBudgetCycles;
+    dsa::ProjEpiParams e;
+    memset(&e, 0, sizeof e);
+    e.part0 = g.part[0];
+    e.part1 = g.part[1];
+    e.splits0 = pl.splits[0];
+    e.splits1 = pl.splits[1];
+    e.ld0 = pl.ld[0];
+    e.ld1 = pl.ld[1];
+    e.nt = pp->nt;
+    e.d_idx = pp->d_idx;
+    e.h_idx = pp->h_idx;
+    e.rope_dim = pp->rope_dim;
+    e.ln_eps = pp->ln_eps;
+    e.rope_theta = pp->rope_theta;
+    e.ln_gamma = ln_gamma;
+    e.ln_beta = ln_beta;
+    e.positions = positions;
+    e.q_seq = kv->q_seq;
+    e.seq_row0 = kv->seq_row0;
+    e.page_table = kv->page_table;
+    e.max_pages = kv->max_pages;
+    e.page_size = kv->page_table ? kv->page_size : 1;
+    e.cache_rows = kv->cache_rows;
+    e.kidx_cache = static_cast<uint8_t *>(kidx_cache);
+    e.k_scale = k_scale;
+    e.q_idx = static_cast<uint8_t *>(q_idx);
+    e.q_scale = q_scale;
+    e.w = static_cast<uint16_t *>(w);
+    e.q_f32 = q_f32;
+    e.k_f32 = k_f32;
+    e.w_f32 = w_f32;
+    e.status = g.status;
+    cudaError_t err = dsa::launch_project(xm, qm, km, pm, wm, g, e, static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_fail(err, "indexer producer launch");
+    return DSA_OK;
 }
 
 int dsa_check_status(void *ws, void *stream) {

@@ -52,7 +52,9 @@ namespace dsa {
 
 namespace {
 
-constexpr int kTileRows = 128;
+constexpr int kTileRows = 128;            // positions per MMA (M) and per epilogue tile
+constexpr int kStageTiles = DSA_K1_STAGE_TILES;  // tiles per TMA ring stage (one box)
+constexpr int kStageRows = kStageTiles * kTileRows;
 
 struct K1Smem {
     uint64_t full[kK1MaxStages];
@@ -72,6 +74,7 @@ struct K1Smem {
     int32_t cand_above[kMaxChunks];      // parallel: keys of each chunk above the threshold bin
     int32_t sel_cnt[kMaxChunks];         // parallel: positions each chunk selects
     int32_t sel_ok;                      // parallel: the bounded waits succeeded
+    int32_t chunk_c, chunk_P;            // this CTA's chunk and its group's chunk count
     unsigned long long t_exact;          // parallel: the need-th largest listed composite
     uint64_t merge_bar;                  // merge: bulk copies of the candidate lists
     uint32_t merge_phase;
@@ -171,52 +174,108 @@ __device__ uint32_t hist_sum_from(const uint32_t *hist, uint32_t lo, SelectScrat
     return r;
 }
 
+// The chunk's candidates: 16-bit offsets into its keys (position - start), in
+// position order, read as composites four at a time (the list is padded with
+// offset 0 to the next multiple of 4).
+struct CandSrc {
+    const uint16_t *off;
+    const uint32_t *keys;
+    int base;
+    __device__ void load4(int i, uint64_t (&v)[4]) const {
+        const uint2 o = *reinterpret_cast<const uint2 *>(off + i);
+        const uint32_t o0 = o.x & 0xFFFFu, o1 = o.x >> 16, o2 = o.y & 0xFFFFu, o3 = o.y >> 16;
+        v[0] = make_composite(keys[o0], static_cast<uint32_t>(base) + o0);
+        v[1] = make_composite(keys[o1], static_cast<uint32_t>(base) + o1);
+        v[2] = make_composite(keys[o2], static_cast<uint32_t>(base) + o2);
+        v[3] = make_composite(keys[o3], static_cast<uint32_t>(base) + o3);
+    }
+};
+
+constexpr int kSlotLog2 = 9;  // parallel selection: staged entries per chunk list, at most 2^9
+
+// The chunks' lists staged in slots of 2^slot_log2 entries (slot c holds
+// chunk c's first n[c] entries; the rest of a slot reads as zero composites).
+struct SlotSrc {
+    const uint64_t *list;
+    const int32_t *n;
+    int slot_log2;
+    __device__ void load4(int i, uint64_t (&v)[4]) const {
+        const uint4 a = *reinterpret_cast<const uint4 *>(list + i);
+        const uint4 b = *reinterpret_cast<const uint4 *>(list + i + 2);
+        const int m = n[i >> slot_log2];
+        const int j = i & ((1 << slot_log2) - 1);
+        v[0] = j < m ? (static_cast<uint64_t>(a.y) << 32) | a.x : 0ull;
+        v[1] = j + 1 < m ? (static_cast<uint64_t>(a.w) << 32) | a.z : 0ull;
+        v[2] = j + 2 < m ? (static_cast<uint64_t>(b.y) << 32) | b.x : 0ull;
+        v[3] = j + 3 < m ? (static_cast<uint64_t>(b.w) << 32) | b.z : 0ull;
+    }
+};
+
 // Parallel exact selection of query q by chunk c = blockIdx.x % P, once the
 // snapshot of G taken in chunk_select is final (every chunk's histogram in
 // it): d* is the threshold bin, `above` the query's keys in higher bins,
 // need = K - above the keys to take from bin d*.
-//   1. publish this chunk's keys of bin d* (its `need` largest at most: a
-//      key beaten by `need` keys of the bin in its own chunk never wins) and
-//      its count of keys above d*; bump the query's `published` counter;
-//   2. wait (bounded) until every chunk has published, read all the lists
-//      (staged into the free streaming area when they fit, else in place)
-//      and find the exact threshold T: the need-th largest composite among
-//      them;
-//   3. every chunk's selected count is its keys above d* plus its listed
-//      keys >= T; the chunks before this one give its offset, and it writes
-//      its own keys >= T there, in ascending position order.
+//   1. one pass over the chunk's keys lists its candidates C (keys of bin d*
+//      or above) in position order;
+//   2. publish C's keys of bin d* (its `need` largest at most: a key beaten
+//      by `need` keys of the bin in its own chunk never wins) and the
+//      chunk's count of keys above d*; bump the query's `published` counter;
+//   3. wait (bounded) until every chunk has published; one round trip
+//      brings every chunk's list (its first 2^kSlotLog2 entries) and counts on
+//      chip; the exact threshold Te is the need-th largest listed composite
+//      (read in place from L2 when a list is longer than that);
+//   4. every chunk's selected count is its keys above d* plus its listed
+//      keys >= Te; the chunks before this one give its offset, and it writes
+//      its candidates >= Te there, in ascending position order.
 // `list` / `list_cap`: shared memory below the chunk's keys (the TMA ring and
-// the q tile, free once streaming is over), in composites.
+// the q tile, free once streaming is over), in composites: the staged lists
+// at its start, C (16-bit) at its end.
 __device__ void parallel_select(const K1Params &a, K1Smem &sm, int q, int qi, const uint32_t *keys,
                                 int start, int len, const uint32_t *lhist, uint32_t *scratch,
                                 uint64_t *list, int list_cap) {
-    const int K = a.topk, P = a.P, c = blockIdx.x % P;
+    const int K = a.topk, P = sm.chunk_P, c = sm.chunk_c;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
-    LocalSrc src{keys, start};
     const bool complete = sm.sel_ok && sm.g_complete[qi];
     const uint32_t d = sm.g_digit[qi];
     const uint32_t need = static_cast<uint32_t>(K) - sm.g_above[qi];
-    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * P + c) * a.cand_stride;
-    int32_t m = 0;
-    int32_t above_c = 0;
+    uint64_t *cand = a.cand + (static_cast<int64_t>(q) * a.P + c) * a.cand_stride;
+    const int c_cap = (len + 4 + 7) & ~7;  // 16-bit entries, room for the padding
+    uint16_t *cands = reinterpret_cast<uint16_t *>(reinterpret_cast<uint8_t *>(list) +
+                                                   static_cast<size_t>(list_cap) * 8 - static_cast<size_t>(c_cap) * 2);
+    // slots of a power of two entries (at most 2^kSlotLog2, and the cand stride)
+    int slot_log2 = kSlotLog2;
+    while (slot_log2 >= 2 && ((1 << slot_log2) * P > list_cap - c_cap / 4 || (1 << slot_log2) > a.cand_stride))
+        --slot_log2;
+    const int stage_cap = slot_log2 >= 2 ? (1 << slot_log2) : 0;  // 0: no room, the lists are read in place
+    CandSrc csrc{cands, keys, start};
+    int32_t m = 0, above_c = 0;
+    uint32_t nC = 0;
     if (complete) {
         above_c = static_cast<int32_t>(hist_sum_from(lhist, d + 1, sm.sel));
         const uint32_t bucket_c = lhist[d];
+        nC = compact_ordered(
+            LocalSrc{keys, start}, len, [d](uint64_t v) { return static_cast<uint32_t>(v >> 53) >= d; },
+            [cands, start](uint32_t slot, uint64_t v) {
+                cands[slot] = static_cast<uint16_t>(composite_pos(v) - static_cast<uint32_t>(start));
+            },
+            0u, sm.sel.wsum);
+        if (tid < 4) cands[nC + tid] = 0;
+        __syncthreads();
         uint64_t thr = static_cast<uint64_t>(d) << 53;
-        if (bucket_c > need) thr = radix_refine(src, len, d, 1, need, scratch, sm.sel);
-        m = static_cast<int32_t>(emit_ordered(
-            src, len, [thr, d](uint64_t v) { return (v >> 53) == d && v >= thr; },
+        if (bucket_c > need) thr = radix_refine(csrc, static_cast<int>(nC), d, 1, need, scratch, sm.sel);
+        m = static_cast<int32_t>(compact_ordered(
+            csrc, static_cast<int>(nC), [thr, d](uint64_t v) { return (v >> 53) == d && v >= thr; },
             [cand, K](uint32_t slot, uint64_t v) {
                 if (slot < static_cast<uint32_t>(K)) cand[slot] = v;
             },
-            0u, sm.sel.wsum, reinterpret_cast<uint4 *>(scratch)));
+            0u, sm.sel.wsum));
         if (m > K) m = K;  // cannot happen: at most `need` <= K keys pass
     }
     // zero composites pad the list to a multiple of 4 (below every key)
     if (tid < 4 && m + tid < ((m + 3) & ~3)) cand[m + tid] = 0ull;
     if (tid == 0) {
-        a.cand_cnt[static_cast<int64_t>(q) * P + c] = m;
-        a.cand_above[static_cast<int64_t>(q) * P + c] = above_c;
+        a.cand_cnt[static_cast<int64_t>(q) * a.P + c] = m;
+        a.cand_above[static_cast<int64_t>(q) * a.P + c] = above_c;
     }
     __threadfence();
     __syncthreads();
@@ -227,47 +286,43 @@ __device__ void parallel_select(const K1Params &a, K1Smem &sm, int q, int qi, co
     }
     __syncthreads();
     if (!sm.sel_ok) return;
-    // every chunk's list length (padded to 4) and above-count; offsets
-    const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * P;
-    const int32_t *abv = a.cand_above + static_cast<int64_t>(q) * P;
-    if (warp == 0) {
+    // one round trip: each chunk's list into its slot of stage_cap entries,
+    // the counts and above-counts alongside
+    const uint64_t *cand_q = a.cand + static_cast<int64_t>(q) * a.P * a.cand_stride;
+    if (tid == 0) mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(P * stage_cap) * 8u);
+    if (tid < P && stage_cap > 0) {
+        fence_proxy_async_global();
+        bulk_load(list + tid * stage_cap, cand_q + static_cast<int64_t>(tid) * a.cand_stride,
+                  static_cast<uint32_t>(stage_cap) * 8u, &sm.merge_bar);
+    }
+    if (warp == 1) {
+        const int32_t *cnt = a.cand_cnt + static_cast<int64_t>(q) * a.P;
+        const int32_t *abv = a.cand_above + static_cast<int64_t>(q) * a.P;
         const int m_l = lane < P ? min(__ldcg(&cnt[lane]), K) : 0;
         const int padded = (m_l + 3) & ~3;
         const int incl = static_cast<int>(warp_incl_scan(static_cast<uint32_t>(padded)));
         if (lane < P) {
-            sm.cand_off[lane] = incl - padded;
+            sm.cand_off[lane] = incl - padded;  // virtual offsets of the lists read in place
             sm.cand_n[lane] = m_l;
             sm.cand_above[lane] = __ldcg(&abv[lane]);
         }
         const int tot = __shfl_sync(0xffffffffu, incl, 31);
-        const int true_tot = static_cast<int>(warp_sum(static_cast<uint32_t>(m_l)));
+        const uint32_t listed = warp_sum(static_cast<uint32_t>(m_l));
+        const bool fits = stage_cap > 0 && __all_sync(0xffffffffu, m_l <= stage_cap);
         if (lane == 0) {
             sm.cand_off[P] = tot;
-            sm.sel.res[3] = static_cast<uint32_t>(true_tot);
-            if (tot <= list_cap) {
-                fence_proxy_async_global();
-                mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(tot) * 8u);
-            }
+            sm.sel.res[3] = listed;
+            sm.sel.res[2] = fits ? 1u : 0u;
         }
     }
-    __syncthreads();
-    const int total = sm.cand_off[P];
+    const bool landed = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase, a.wait_budget));
+    if (tid == 0) sm.merge_phase ^= 1u;
+    if (!landed) {
+        if (tid == 0) record_status(a.status, DSA_ERR_TIMEOUT);
+        return;
+    }
+    const bool staged = sm.sel.res[2] != 0;
     const uint32_t listed = sm.sel.res[3];
-    const bool staged = total <= list_cap;
-    if (staged) {
-        if (tid < P && sm.cand_n[tid] > 0) {
-            fence_proxy_async_global();
-            bulk_load(list + sm.cand_off[tid], a.cand + (static_cast<int64_t>(q) * P + tid) * a.cand_stride,
-                      static_cast<uint32_t>((sm.cand_n[tid] + 3) & ~3) * 8u, &sm.merge_bar);
-        }
-        const bool ok = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase, a.wait_budget));
-        if (tid == 0) sm.merge_phase ^= 1u;
-        __syncthreads();
-        if (!ok) {
-            if (tid == 0) record_status(a.status, DSA_ERR_TIMEOUT);
-            return;
-        }
-    }
     // the threshold: the need-th largest listed composite (listed >= need:
     // a chunk whose bin-d* keys exceed `need` lists `need` of them, else all).
     // radix_refine gives a bound T with exactly `need` listed composites >= T;
@@ -276,18 +331,16 @@ __device__ void parallel_select(const K1Params &a, K1Smem &sm, int q, int qi, co
     // smallest listed one, which is <= Te, but may lie above T.
     uint64_t T = static_cast<uint64_t>(d) << 53;
     if (listed != need) {
-        if (staged) T = radix_refine(ListSrc{list}, total, d, 1, need, scratch, sm.sel);
-        else T = radix_refine(GlobalSegSrc{a.cand + static_cast<int64_t>(q) * P * a.cand_stride,
-                                           a.cand_stride, P, sm.cand_off},
-                              total, d, 1, need, scratch, sm.sel);
+        if (staged) T = radix_refine(SlotSrc{list, sm.cand_n, slot_log2}, P * stage_cap, d, 1, need, scratch, sm.sel);
+        else T = radix_refine(GlobalSegSrc{cand_q, a.cand_stride, P, sm.cand_off}, sm.cand_off[P], d, 1, need,
+                              scratch, sm.sel);
     }
     if (tid == 0) sm.t_exact = ~0ull;
     __syncthreads();
     // selected count of every chunk: keys above d* + listed keys >= T
     for (int cc = warp; cc < P; cc += nwarps) {
         const int mm = sm.cand_n[cc];
-        const uint64_t *seg = staged ? list + sm.cand_off[cc]
-                                     : a.cand + (static_cast<int64_t>(q) * P + cc) * a.cand_stride;
+        const uint64_t *seg = staged ? list + cc * stage_cap : cand_q + static_cast<int64_t>(cc) * a.cand_stride;
         uint32_t k = 0;
         unsigned long long lo = ~0ull;
         for (int j = lane; j < mm; j += 32) {
@@ -316,12 +369,12 @@ __device__ void parallel_select(const K1Params &a, K1Smem &sm, int q, int qi, co
         all += sm.sel_cnt[cc];
     }
     int32_t *out = a.idx + static_cast<int64_t>(q) * K;
-    const uint32_t got = emit_ordered(
-        src, len, [Te](uint64_t v) { return v >= Te; },
+    const uint32_t got = compact_ordered(
+        csrc, static_cast<int>(nC), [Te](uint64_t v) { return v >= Te; },
         [out, K](uint32_t slot, uint64_t v) {
             if (slot < static_cast<uint32_t>(K)) out[slot] = static_cast<int32_t>(composite_pos(v));
         },
-        static_cast<uint32_t>(off), sm.sel.wsum, reinterpret_cast<uint4 *>(scratch));
+        static_cast<uint32_t>(off), sm.sel.wsum);
     if (tid == 0) {
         if (got != static_cast<uint32_t>(off + sm.sel_cnt[c]) || all != K)
             record_status(a.status, DSA_ERR_DEVICE_CHECK);
@@ -341,7 +394,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
                              uint32_t *scratch, uint64_t *list, int list_cap) {
     const int K = a.topk;
     LocalSrc src{keys, start};
-    if (a.P == 1) {
+    if (sm.chunk_P == 1) {
         // the whole history is here: len == n > K
         find_digit(lhist, kSelBins, static_cast<uint32_t>(K), sm.sel);
         const uint32_t d = sm.sel.res[0], above = sm.sel.res[1], bucket = sm.sel.res[2];
@@ -366,7 +419,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
 
     // ---- several chunks: publish this chunk's histogram, then read G back
     uint32_t *G = a.ghist + static_cast<int64_t>(q) * kSelBins;
-    const int c = blockIdx.x % a.P;
+    const int c = sm.chunk_c;
     for (int b = threadIdx.x; b < kSelBins; b += blockDim.x)
         if (lhist[b]) atomicAdd(&G[b], lhist[b]);
     __threadfence();
@@ -556,10 +609,26 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     K1Smem &sm = *reinterpret_cast<K1Smem *>(base + L.misc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = blockIdx.x / a.P, c = blockIdx.x % a.P;
+    // group and chunk of this CTA: groups [0, n_big) have P chunks, the rest
+    // P - 1 (a batch then fills every SM); each group cuts its own span
+    int g, c, Pg;
+    {
+        const int b = blockIdx.x, big = a.n_big * a.P;
+        if (b < big) {
+            g = b / a.P;
+            c = b % a.P;
+            Pg = a.P;
+        } else {
+            const int r = b - big;
+            g = a.n_big + r / (a.P - 1);
+            c = r % (a.P - 1);
+            Pg = a.P - 1;
+        }
+    }
     int q0, nqg;
     group_queries(a, g, q0, nqg);
     constexpr int kTileBytes = kTileRows * DI;
+    constexpr int kStageBytes = kStageRows * DI;
     const int N = a.qg * HP;  // MMA N (columns per accumulator buffer)
 
     // ---- set-up
@@ -572,34 +641,38 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     }
     const int seq = nqg > 0 ? a.q_seq[q0] : 0;
     const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
-    const int start = c * a.chunk;
-    const int end = min(start + a.chunk, span);
+    const int chunk = min(a.chunk, ((span + Pg - 1) / Pg + kStageRows - 1) / kStageRows * kStageRows);
+    const int start = c * chunk;
+    const int end = min(start + chunk, span);
     const int len = max(end - start, 0);
     const int ntiles = (len + kTileRows - 1) / kTileRows;
+    const int nst = (ntiles + kStageTiles - 1) / kStageTiles;  // ring stages of 256 rows
 
     // The producer (thread 0) fills the TMA ring as soon as its barriers
     // exist, so the first tiles are in flight during the rest of the set-up.
     const int64_t row0 = (a.page_table == nullptr && nqg > 0) ? a.seq_row0[seq] : 0;
-    // tests only: the first CTA never loads its first tile, so the MMA
+    // tests only: the first CTA never loads its first stage, so the MMA
     // issuer's wait for it runs out
     const bool skip_first = a.inject != 0 && blockIdx.x == 0;
-    auto issue_tile = [&](int t, int s) {
-        if (skip_first && t == 0) return;
-        const int p0 = start + t * kTileRows;
-        uint8_t *dst = stages + s * kTileBytes;
+    // stage u holds tiles 2u and 2u + 1: one 256-row box (contiguous cache;
+    // a box past the end of the cache reads zeros), or one box per page
+    auto issue_stage = [&](int u, int s) {
+        if (skip_first && u == 0) return;
+        const int p0 = start + u * kStageRows;
+        uint8_t *dst = stages + s * kStageBytes;
         if (a.page_table == nullptr) {
-            mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
+            mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
             tma_load_2d(dst, &kmap, &sm.full[s], 0, static_cast<int32_t>(row0 + p0));
         } else {
             const int box = a.page_size;
             const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages + p0 / box;
             int n_box = 0;
-            for (int h = 0; h < kTileRows / box; ++h) n_box += (p0 + h * box < nmax);
+            for (int h = 0; h < kStageRows / box; ++h) n_box += (p0 + h * box < nmax);
             mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
             for (int h = 0; h < n_box; ++h, dst += box * DI) tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[h] * box);
         }
     };
-    const int n_pro = min(ntiles, a.stages);  // tiles issued before the set-up barrier
+    const int n_pro = min(nst, a.stages);  // stages issued before the set-up barrier
 
     if (tid == 0) {
         sm.abort = 0;
@@ -617,7 +690,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b % 2
         }
         fence_mbar_init();
-        for (int t = 0; t < n_pro; ++t) issue_tile(t, t);
+        for (int u = 0; u < n_pro; ++u) issue_stage(u, u);
+        sm.chunk_c = c;
+        sm.chunk_P = Pg;
     }
     if (tid < kMaxGroupQueries) sm.n_q[tid] = tid < nqg ? a.q_n[q0 + tid] : 0;
     // q^I tile (B operand, K-major, swizzled like the TMA tiles) and weights
@@ -657,27 +732,27 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (ntiles > 0) {
         if (warp == 0) {
             if (lane == 0) {
-                // ring position (s, ph) advances by one per tile: no divisions
+                // ring position (s, ph) advances by one per stage: no divisions
                 // in this single-thread loop, which paces the whole stream
                 int s = n_pro == a.stages ? 0 : n_pro;
                 uint32_t ph = n_pro == a.stages ? 1u : 0u;
-                int t_end = n_pro;  // tiles issued (or skipped) so far
-                for (int t = n_pro; t < ntiles; ++t) {
+                int u_end = n_pro;  // stages issued (or skipped) so far
+                for (int u = n_pro; u < nst; ++u) {
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
                     }
-                    issue_tile(t, s);
-                    t_end = t + 1;
+                    issue_stage(u, s);
+                    u_end = u + 1;
                     if (++s == a.stages) { s = 0; ph ^= 1; }
                 }
-                // before the CTA may exit, every tile load issued must have
-                // landed: wait (bounded) for the newest phase of each stage
-                // (a no-op when the MMA consumed them all)
-                for (int t = max(t_end - a.stages, 0); t < t_end; ++t)
-                    if (!(skip_first && t == 0) &&
-                        !mbar_wait(&sm.full[t % a.stages], static_cast<uint32_t>(t / a.stages) & 1u, a.wait_budget))
+                // before the CTA may exit, every load issued must have landed:
+                // wait (bounded) for the newest phase of each stage (a no-op
+                // when the MMA consumed them all)
+                for (int u = max(u_end - a.stages, 0); u < u_end; ++u)
+                    if (!(skip_first && u == 0) &&
+                        !mbar_wait(&sm.full[u % a.stages], static_cast<uint32_t>(u / a.stages) & 1u, a.wait_budget))
                         record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else if (warp == 1) {
@@ -691,22 +766,33 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 const uint64_t bd0 = make_sdesc(smem_u32(qtile), 16, kSbo, kLayout);
                 int s = 0, b = 0;
                 uint32_t ph = 0, aph = 0;
-                for (int t = 0; t < ntiles; ++t) {
-                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
-                        !mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
-                        record_status(a.status, DSA_ERR_TIMEOUT);
-                        sm.abort = 1;
+                bool failed = false;
+                for (int u = 0; u < nst && !failed; ++u) {
+                    if (!mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
+                        failed = true;
                         break;
                     }
-                    tc_fence_after();
-                    const uint64_t ad = ad0 + static_cast<uint64_t>(s * (kTileBytes >> 4));
+                    for (int sub = 0; sub < kStageTiles && kStageTiles * u + sub < ntiles; ++sub) {
+                        if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) || sm.abort) {
+                            failed = true;
+                            break;
+                        }
+                        tc_fence_after();
+                        const uint64_t ad =
+                            ad0 + static_cast<uint64_t>((s * kStageBytes + sub * kTileBytes) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < DI / 32; ++kk)
-                        mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < DI / 32; ++kk)
+                            mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                        tc_commit(&sm.acc_full[b]);
+                        if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
+                    }
+                    if (failed) break;
                     tc_commit(&sm.empty[s]);
-                    tc_commit(&sm.acc_full[b]);
                     if (++s == a.stages) { s = 0; ph ^= 1; }
-                    if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
+                }
+                if (failed) {
+                    record_status(a.status, DSA_ERR_TIMEOUT);
+                    sm.abort = 1;
                 }
                 // every MMA issued must complete before TMEM is freed
                 tc_commit(&sm.mma_done);
@@ -846,6 +932,8 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
     if (threadIdx.x == 0) {
         sm.abort = 0;
         sm.is_last = 0;
+        sm.chunk_c = c;
+        sm.chunk_P = a.P;
         sm.n_q[0] = a.q_n[q];
         sm.g_complete[0] = 0;
         mbar_init(&sm.merge_bar, 1);
@@ -893,7 +981,7 @@ static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaS
     auto kern = k1_indexer<MODE, HP, DI>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const int grid = a.n_groups * a.P;
+    const int grid = a.n_big * a.P + (a.n_groups - a.n_big) * (a.P - 1);
     if (grid == 0) return cudaSuccess;
     kern<<<grid, kK1Threads, smem, st>>>(kmap, a);
     return cudaGetLastError();

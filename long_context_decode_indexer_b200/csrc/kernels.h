@@ -18,7 +18,17 @@ constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
 constexpr int kModeScores = 1;  // scores written to HBM
 constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 
-constexpr int kK1MaxStages = 12;     // TMA ring depth limit (128-row k^I tiles)
+// Indexer stream tuning: 128-row tiles per TMA ring stage (one box of
+// 128 * DSA_K1_STAGE_TILES rows), ring depth, and whether the SMs a batch of
+// equal chunk counts leaves idle give some groups one more chunk.
+#ifndef DSA_K1_STAGE_TILES
+#define DSA_K1_STAGE_TILES 2
+#endif
+#ifndef DSA_K1_FILL_SMS
+#define DSA_K1_FILL_SMS 1
+#endif
+constexpr int kK1MaxStages = 12;     // TMA ring barriers
+constexpr int kK1WantStages = 8 / DSA_K1_STAGE_TILES;  // ring depth used when shared memory allows
 constexpr int kK1MaxAcc = 4;         // TMEM accumulator buffers (even: one parity per epilogue group)
 constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
@@ -50,9 +60,10 @@ struct K1Params {
     int32_t nq, h_idx, d_idx, topk;
     // work split
     int32_t q_per_seq, qg, groups_per_block, n_groups;
-    int32_t P;      // chunks per group
+    int32_t P;      // chunks per group: groups [0, n_big) have P, the others P - 1
+    int32_t n_big;
     int32_t chunk;  // positions per chunk (multiple of 128)
-    int32_t stages; // TMA ring depth
+    int32_t stages; // TMA ring depth (stages of 256 rows)
     int32_t acc_bufs;  // TMEM accumulator buffers of qg*hp columns (2 or 4)
     uint32_t tmem_cols;
     // outputs
@@ -91,7 +102,7 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
     K1Layout L;
     uint32_t off = 0;
     L.stages = off;
-    if (mode != kModeTopk) off += static_cast<uint32_t>(stages) * 128u * static_cast<uint32_t>(di);
+    if (mode != kModeTopk) off += static_cast<uint32_t>(stages) * 128u * DSA_K1_STAGE_TILES * static_cast<uint32_t>(di);
     L.qtile = off;
     if (mode != kModeTopk) off += align_up(static_cast<uint32_t>(qg * hp * di), 1024);
     L.keys = off;
@@ -132,12 +143,12 @@ cudaError_t launch_topk(const K1Params &a, cudaStream_t st);
 constexpr int kDqk = 576;           // key width (512 latent + 64 rope)
 constexpr int kDv = 512;            // value width
 constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
-constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
-constexpr int kMlaStages = 4;       // pass-1 ring depth (Q chunk + K chunk)
-constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
-constexpr int kMlaVStages = 3;      // pass-2 ring depth
+constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit: S takes <= 256 TMEM columns)
+constexpr int kMlaBlockRows = 32;   // pass 1: rows per ring block (MMA N)
+constexpr int kMlaRing = 4;         // pass 1: ring depth (blocks of 32 whole rows)
 constexpr int kMlaMaxSplits = 32;   // splits per query (the combine kernel's warp reads one LSE per lane)
-constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers (0-3 help in pass 1)
+constexpr int kMlaThreads = 448;    // warps 0-3 group A, 4-7 group B, 8-11 group C, 12 MMA, 13 rope-Q TMA
+constexpr int kMlaScaleBlocks = 8;  // power-of-two scales per partial row (one per 64 value columns)
 
 struct MlaParams {
     const int32_t *q_seq;
@@ -147,6 +158,7 @@ struct MlaParams {
     int32_t max_pages, page_size;
     int64_t cache_rows;
     const int32_t *idx;  // [nq, topk]
+    const uint16_t *q;   // [nq, h, 576] bf16 bits
     const uint16_t *kv;  // latent cache (bf16 bits)
     int64_t kv_row_stride;  // elements between cache rows
     int32_t nq, h, topk;
@@ -160,37 +172,76 @@ struct MlaParams {
     float *lse;          // [nq, h]
     uint16_t *part_o;    // [wave_q, splits, 128, d_v] normalised partial outputs / part_scale (fp16 bits)
     float *part_lse;     // [wave_q, splits, 128]
-    float *part_scale;   // [wave_q, splits, 128, 2] power of two of each half row of part_o
+    float *part_scale;   // [wave_q, splits, 128, 8] power of two of each 64-column block of part_o
     int *status;
     long long wait_budget;  // bounded waits, SM cycles
     int32_t inject;         // tests only: the first CTA's gathers skip one arrival
 };
 
 struct MlaLayout {
-    uint32_t ring, p_tile, p_lo, v_ring, misc, total;
+    uint32_t ring, vq, rope, misc, total;
 };
 
 __host__ __device__ inline MlaLayout mla_layout() {
     MlaLayout L;
-    // pass 1: kMlaStages x (Q chunk 128x64 bf16 = 16 KB + K chunk 256x64 bf16 = 32 KB)
-    const uint32_t stage = 128u * 128u + kMlaMaxRows * 128u;
-    const uint32_t pass1 = kMlaStages * stage;
-    // pass 2: P as a hi + lo pair of bf16 tiles (128 x 256 each, 64 KB each)
-    // + kMlaVStages V tiles (32 rows x 512 bf16 = 32 KB each)
-    const uint32_t ptile = 128u * kMlaMaxRows * 2u;
-    const uint32_t vtile = kMlaVRows * kDv * 2u;
+    const uint32_t block = kMlaBlockRows * kDqk * 2u;  // 36 KB: 9 chunks of [32 rows x 64 cols]
+    const uint32_t pass1 = kMlaRing * block;
+    const uint32_t vq = kMlaMaxRows * 256u;            // a value quarter (128 cols) of 256 rows: 64 KB
     L.ring = 0;
-    L.p_tile = 0;
-    L.p_lo = ptile;
-    L.v_ring = 2 * ptile;
-    const uint32_t pass2 = 2 * ptile + kMlaVStages * vtile;
-    uint32_t end = pass1 > pass2 ? pass1 : pass2;
-    L.misc = align_up(end, 128);
-    L.total = L.misc + 2048 + 1024;  // barriers and row table, alignment slack
+    L.vq = 0;                                          // pass 2 reuses the ring: two quarter buffers
+    const uint32_t end = pass1 > 2 * vq ? pass1 : 2 * vq;
+    L.rope = align_up(end, 1024);                      // Q columns 512..575, 128 heads x 128 B
+    L.misc = L.rope + 128u * 128u;
+    L.total = L.misc + 4096 + 1024;                    // barriers, row table, exchanges; alignment slack
     return L;
 }
 
 cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st);
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st);
+
+// ------------------------------------------------ indexer producer (q^I, k^I, w)
+constexpr int kProjStages = 4;  // TMA ring depth of the projection GEMM
+
+// Split-K GEMM of both projections: problem 0 = x . [W_k; W_proj]^T
+// (N = d_I + H_I), problem 1 = q_lora . W_qb^T (N tiles of 128 rows).
+struct ProjGemmParams {
+    int32_t nt;              // tokens
+    int32_t m_tiles;         // 128-token tiles
+    int32_t k_steps[2];      // 64-wide K steps per problem
+    int32_t n_cols[2];       // MMA N of a tile (a multiple of 16)
+    int32_t n_tiles[2];      // tiles along N (1 for problem 0)
+    int32_t splits[2];       // K slices per problem
+    int32_t items0;          // work items of problem 0 (they come first in the grid)
+    int32_t d_idx, h_idx;
+    float *part[2];          // [splits, nt, ld] fp32 partial sums per K slice
+    int32_t ld[2];           // row lengths of part
+    int *status;
+    long long wait_budget;
+};
+
+struct ProjEpiParams {
+    const float *part0, *part1;
+    int32_t splits0, splits1, ld0, ld1;
+    int32_t nt, d_idx, h_idx, rope_dim;
+    float ln_eps, rope_theta;
+    const float *ln_gamma, *ln_beta;  // [d_idx]
+    const int32_t *positions;         // [nt]
+    const int32_t *q_seq;             // [nt]
+    const int64_t *seq_row0;
+    const int32_t *page_table;
+    int32_t max_pages, page_size;
+    int64_t cache_rows;
+    uint8_t *kidx_cache;              // [cache_rows, d_idx] e4m3
+    float *k_scale;                   // [cache_rows]
+    uint8_t *q_idx;                   // [nt, h_idx, d_idx] e4m3
+    float *q_scale;                   // [nt, h_idx] or null
+    uint16_t *w;                      // [nt, h_idx] bf16
+    float *q_f32, *k_f32, *w_f32;     // values before rounding, or null
+    int *status;
+};
+
+cudaError_t launch_project(const CUtensorMap &x_map, const CUtensorMap &ql_map, const CUtensorMap &wk_map,
+                           const CUtensorMap &wp_map, const CUtensorMap &wq_map, const ProjGemmParams &g,
+                           const ProjEpiParams &e, cudaStream_t st);
 
 }  // namespace dsa

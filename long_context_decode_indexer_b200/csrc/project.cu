@@ -1,0 +1,354 @@
+// project.cu -- the lightning indexer's own projections on sm_100a: the step
+// that produces q^I, k^I and the head weights the indexer score consumes
+// ("DeepSeekV3.2之DSA" by yuyanqi, sections 4.1-4.3), with k^I appended to
+// the index-K cache (its decode data flow, section 5.1):
+//   q^I[t] = W_qb . q_lora[t]                 -> [H_I, d_I], RoPE, FP8 + scale
+//   k^I[t] = LayerNorm(W_k . x[t])            -> RoPE, FP8 + scale -> cache row
+//   w[t]   = (W_proj . x[t]) * H_I^-1/2 * d_I^-1/2 * q_scale[t]   -> bf16
+// RoPE rotates the pairs (2i, 2i+1) of the first rope_dim dims by
+// pos * theta^(-2i / rope_dim); the FP8 scales are powers of two (the e8m0
+// k_s of section 4.3; the same for q, so folding it into w is exact).
+//
+// k5_proj_gemm: both contractions in one launch, on the tensor cores.  A work
+// item is (problem, 128-token tile, N tile, K slice); a TMA ring feeds
+// tcgen05.mma kind::f16 (M = 128 tokens, N = d_I + H_I for the x problem, 128
+// for the q_lora problem, K = 64 per stage) into TMEM, and the epilogue warps
+// write the fp32 partial sums of the slice.  Few tokens (decode) leave most
+// SMs without a token tile, so K is split into slices until the grid fills
+// the SMs, in proportion to each problem's weight bytes.
+// k6_proj_epilogue: one CTA per token sums the slices in a fixed order and
+// applies LayerNorm, RoPE, the quantisation, the weight folding and the
+// cache append.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kPBm = 128;                 // tokens per tile (MMA M)
+constexpr int kPBk = 64;                  // K per stage (128 bytes of bf16: one swizzle span)
+constexpr int kPABytes = kPBm * kPBk * 2; // 16 KB
+constexpr int kPBMaxRows = 256;           // B rows per tile (MMA N <= 256)
+constexpr int kPStageBytes = kPABytes + kPBMaxRows * kPBk * 2;
+
+struct ProjSmem {
+    uint64_t full[kProjStages];
+    uint64_t empty[kProjStages];
+    uint64_t acc_full;
+    uint32_t tmem_base;
+    volatile int32_t abort;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ float warp_sum_f(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+__device__ __forceinline__ float warp_max_f(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+// The smallest power of two 2^e with amax / 2^e <= 448 (the E4M3 maximum);
+// 1 when amax is 0.  frexp makes the test exact: amax / 448 = f * 2^e with f
+// in [0.5, 1) is at most 2^e, and equals 2^(e-1) when f = 0.5.
+__device__ __forceinline__ float pow2_scale(float amax) {
+    if (!(amax > 0.f)) return 1.f;
+    int e;
+    const double f = frexp(static_cast<double>(amax) / 448.0, &e);
+    return static_cast<float>(ldexp(1.0, f == 0.5 ? e - 1 : e));
+}
+
+__device__ __forceinline__ uint32_t e4m3(float x) {
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
+}
+
+// RoPE of the pair (v0, v1) at dims (2i, 2i+1): angle pos * theta^(-2i/rope_dim)
+// in double (positions reach 2^27; an fp32 angle would lose the fraction).
+__device__ __forceinline__ void rope_pair(float &v0, float &v1, int i, int rope_dim, int pos, float theta) {
+    const double inv = pow(static_cast<double>(theta), -2.0 * static_cast<double>(i) / static_cast<double>(rope_dim));
+    double s, c;
+    sincos(static_cast<double>(pos) * inv, &s, &c);
+    const double x0 = v0, x1 = v1;
+    v0 = static_cast<float>(x0 * c - x1 * s);
+    v1 = static_cast<float>(x0 * s + x1 * c);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// k5: split-K tcgen05 GEMM of both projections.  192 threads: warp 0 TMA,
+// warp 1 MMA, warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(192, 1)
+    k5_proj_gemm(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap ql_map,
+                 const __grid_constant__ CUtensorMap wk_map, const __grid_constant__ CUtensorMap wp_map,
+                 const __grid_constant__ CUtensorMap wq_map, const ProjGemmParams a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    ProjSmem &sm = *reinterpret_cast<ProjSmem *>(base + kProjStages * kPStageBytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int prob = static_cast<int>(blockIdx.x) < a.items0 ? 0 : 1;
+    const int it = prob ? static_cast<int>(blockIdx.x) - a.items0 : static_cast<int>(blockIdx.x);
+    const int split = it % a.splits[prob];
+    const int rest = it / a.splits[prob];
+    const int n_tile = rest % a.n_tiles[prob];
+    const int m_tile = rest / a.n_tiles[prob];
+    const int k_begin = static_cast<int>(static_cast<int64_t>(split) * a.k_steps[prob] / a.splits[prob]);
+    const int k_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.k_steps[prob] / a.splits[prob]);
+    const int nk = k_end - k_begin;
+    const int N = a.n_cols[prob];
+    const uint32_t b_bytes = prob == 0 ? static_cast<uint32_t>(a.d_idx + a.h_idx) * kPBk * 2u
+                                       : static_cast<uint32_t>(kPBm) * kPBk * 2u;
+    const uint32_t tmem_cols = N <= 128 ? 128u : 256u;
+
+    if (tid == 0) {
+        sm.abort = 0;
+        for (int s = 0; s < kProjStages; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, tmem_cols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int t_end = 0;
+            for (int t = 0; t < nk; ++t) {
+                if (!mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) || sm.abort) {
+                    record_status(a.status, DSA_ERR_TIMEOUT);
+                    sm.abort = 1;
+                    break;
+                }
+                uint8_t *st = base + s * kPStageBytes;
+                const int k0 = (k_begin + t) * kPBk;
+                mbar_arrive_expect_tx(&sm.full[s], kPABytes + b_bytes);
+                if (prob == 0) {
+                    tma_load_2d(st, &x_map, &sm.full[s], k0, m_tile * kPBm);
+                    tma_load_2d(st + kPABytes, &wk_map, &sm.full[s], k0, 0);
+                    tma_load_2d(st + kPABytes + a.d_idx * kPBk * 2, &wp_map, &sm.full[s], k0, 0);
+                } else {
+                    tma_load_2d(st, &ql_map, &sm.full[s], k0, m_tile * kPBm);
+                    tma_load_2d(st + kPABytes, &wq_map, &sm.full[s], k0, n_tile * kPBm);
+                }
+                t_end = t + 1;
+                if (++s == kProjStages) { s = 0; ph ^= 1; }
+            }
+            // every load issued lands before the CTA may exit
+            for (int t = max(t_end - kProjStages, 0); t < t_end; ++t)
+                mbar_wait(&sm.full[t % kProjStages], static_cast<uint32_t>(t / kProjStages) & 1u, a.wait_budget);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = make_idesc(1, 1, 0, 0, kPBm, static_cast<uint32_t>(N));
+            int s = 0;
+            uint32_t ph = 0;
+            for (int t = 0; t < nk; ++t) {
+                if (!mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
+                    record_status(a.status, DSA_ERR_TIMEOUT);
+                    sm.abort = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t aa = smem_u32(base + s * kPStageBytes);
+                const uint32_t ba = aa + kPABytes;
+#pragma unroll
+                for (int kk = 0; kk < kPBk / 16; ++kk) {
+                    const uint64_t ad = make_sdesc(aa + kk * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t bd = make_sdesc(ba + kk * 32, 16, 1024, kSwizzle128B);
+                    mma_bf16_ss(tmem, ad, bd, idesc, (t > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc_commit(&sm.empty[s]);
+                if (++s == kProjStages) { s = 0; ph ^= 1; }
+            }
+            // completes once every MMA issued above has (also when none was)
+            tc_commit(&sm.acc_full);
+        }
+    } else {
+        // epilogue: TMEM lane = token row of the tile
+        const int quarter = warp & 3;
+        const int m = m_tile * kPBm + quarter * 32 + lane;
+        const bool ok = warp_wait(&sm.acc_full, 0, &sm.abort, a.wait_budget);
+        if (ok) {
+            tc_fence_after();
+            // valid columns of this tile
+            const int ncol = prob == 0 ? a.d_idx + a.h_idx : min(kPBm, a.ld[1] - n_tile * kPBm);
+            float *row = a.part[prob] + (static_cast<int64_t>(split) * a.nt + m) * a.ld[prob] +
+                         static_cast<int64_t>(n_tile) * kPBm;
+            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            for (int c0 = 0; c0 < N; c0 += 32) {
+                uint32_t v[32];
+                tmem_ld32(lane_addr + c0, v);
+                tmem_wait_ld();
+                if (m < a.nt) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        if (c0 + j + 3 < ncol)
+                            *reinterpret_cast<float4 *>(row + c0 + j) =
+                                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                            __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                        else
+                            for (int e = 0; e < 4; ++e)
+                                if (c0 + j + e < ncol) row[c0 + j + e] = __uint_as_float(v[j + e]);
+                }
+            }
+        } else if (lane == 0) {
+            record_status(a.status, DSA_ERR_TIMEOUT);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, tmem_cols);
+}
+
+// ---------------------------------------------------------------------------
+// k6: per token, sum the K slices (in slice order) and finish the producer.
+// 256 threads; lane l of a warp holds dims [l * per, (l + 1) * per) of a
+// d_I-wide vector (per = d_I / 32: 4 or 2), so every RoPE pair is in-lane.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
+    __shared__ float wraw[64];
+    const int t = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int d = a.d_idx, H = a.h_idx, per = a.d_idx / 32;
+    const int pos = a.positions[t];
+
+    if (warp == 0) {
+        // ---- k^I: LayerNorm, RoPE, FP8 with a power-of-two scale, cache append
+        float v[4];
+        for (int i = 0; i < per; ++i) {
+            const int o = lane * per + i;
+            float acc = 0.f;
+            for (int s = 0; s < a.splits0; ++s) acc += a.part0[(static_cast<int64_t>(s) * a.nt + t) * a.ld0 + o];
+            v[i] = acc;
+        }
+        float sum = 0.f;
+        for (int i = 0; i < per; ++i) sum += v[i];
+        const float mean = warp_sum_f(sum) / static_cast<float>(d);
+        float sq = 0.f;
+        for (int i = 0; i < per; ++i) sq += (v[i] - mean) * (v[i] - mean);
+        const float var = warp_sum_f(sq) / static_cast<float>(d);
+        const float inv_std = 1.f / sqrtf(var + a.ln_eps);
+        for (int i = 0; i < per; ++i) {
+            const int o = lane * per + i;
+            v[i] = (v[i] - mean) * inv_std * a.ln_gamma[o] + a.ln_beta[o];
+        }
+        for (int i = 0; i < per; i += 2) {
+            const int o = lane * per + i;
+            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], o / 2, a.rope_dim, pos, a.rope_theta);
+        }
+        float amax = 0.f;
+        for (int i = 0; i < per; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const float scale = pow2_scale(warp_max_f(amax));
+        const float inv = 1.f / scale;  // exact: a power of two
+        // cache row of (sequence, position)
+        const int seq = a.q_seq[t];
+        int64_t row;
+        if (a.page_table)
+            row = static_cast<int64_t>(a.page_table[static_cast<int64_t>(seq) * a.max_pages + pos / a.page_size]) *
+                      a.page_size + pos % a.page_size;
+        else
+            row = a.seq_row0[seq] + pos;
+        const bool in_range = pos >= 0 && row >= 0 && row < a.cache_rows &&
+                              (a.page_table == nullptr || static_cast<int64_t>(pos) / a.page_size < a.max_pages);
+        if (!in_range) {
+            if (lane == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
+        } else {
+            uint32_t packed = 0;
+            for (int i = 0; i < per; ++i) packed |= e4m3(v[i] * inv) << (8 * i);
+            uint8_t *dst = a.kidx_cache + row * d + lane * per;
+            if (per == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+            else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
+            if (lane == 0) a.k_scale[row] = scale;
+        }
+        if (a.k_f32)
+            for (int i = 0; i < per; ++i) a.k_f32[static_cast<int64_t>(t) * d + lane * per + i] = v[i];
+    } else if (warp == 1) {
+        // ---- the raw head weights W_proj . x
+        for (int j = lane; j < H; j += 32) {
+            float acc = 0.f;
+            for (int s = 0; s < a.splits0; ++s) acc += a.part0[(static_cast<int64_t>(s) * a.nt + t) * a.ld0 + d + j];
+            wraw[j] = acc;
+            if (a.w_f32) a.w_f32[static_cast<int64_t>(t) * H + j] = acc;
+        }
+    }
+    __syncthreads();
+    // ---- q^I heads: RoPE, FP8 with a power-of-two scale; w folds the scale
+    for (int h = warp; h < H; h += 8) {
+        float v[4];
+        const int64_t col0 = static_cast<int64_t>(h) * d + lane * per;
+        for (int i = 0; i < per; ++i) {
+            float acc = 0.f;
+            for (int s = 0; s < a.splits1; ++s) acc += a.part1[(static_cast<int64_t>(s) * a.nt + t) * a.ld1 + col0 + i];
+            v[i] = acc;
+        }
+        for (int i = 0; i < per; i += 2) {
+            const int o = lane * per + i;
+            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], o / 2, a.rope_dim, pos, a.rope_theta);
+        }
+        float amax = 0.f;
+        for (int i = 0; i < per; ++i) amax = fmaxf(amax, fabsf(v[i]));
+        const float scale = pow2_scale(warp_max_f(amax));
+        const float inv = 1.f / scale;
+        uint32_t packed = 0;
+        for (int i = 0; i < per; ++i) packed |= e4m3(v[i] * inv) << (8 * i);
+        uint8_t *dst = a.q_idx + (static_cast<int64_t>(t) * H + h) * d + lane * per;
+        if (per == 4) *reinterpret_cast<uint32_t *>(dst) = packed;
+        else *reinterpret_cast<uint16_t *>(dst) = static_cast<uint16_t>(packed);
+        if (a.q_f32)
+            for (int i = 0; i < per; ++i) a.q_f32[(static_cast<int64_t>(t) * H + h) * d + lane * per + i] = v[i];
+        if (lane == 0) {
+            const int64_t th = static_cast<int64_t>(t) * H + h;
+            if (a.q_scale) a.q_scale[th] = scale;
+            // the same operations, in the same order, as the definition:
+            // w / sqrt(H_I) / sqrt(d_I) * q_scale, then bf16 (ties to even)
+            const double wv = static_cast<double>(wraw[h]) / sqrt(static_cast<double>(H)) /
+                              sqrt(static_cast<double>(d)) * static_cast<double>(scale);
+            a.w[th] = __bfloat16_as_ushort(__double2bfloat16(wv));
+        }
+    }
+}
+
+cudaError_t launch_project(const CUtensorMap &x_map, const CUtensorMap &ql_map, const CUtensorMap &wk_map,
+                           const CUtensorMap &wp_map, const CUtensorMap &wq_map, const ProjGemmParams &g,
+                           const ProjEpiParams &e, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(kProjStages) * kPStageBytes + sizeof(ProjSmem) + 1024;
+    cudaError_t err = cudaFuncSetAttribute(k5_proj_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    const int grid = g.items0 + g.m_tiles * g.n_tiles[1] * g.splits[1];
+    if (grid == 0 || g.nt == 0) return cudaSuccess;
+    k5_proj_gemm<<<grid, 192, smem, st>>>(x_map, ql_map, wk_map, wp_map, wq_map, g);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    k6_proj_epilogue<<<g.nt, 256, 0, st>>>(e);
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

@@ -282,4 +282,50 @@ __device__ uint32_t emit_ordered(const Src &src, int n, const Pred &pred, const 
     return base + total;
 }
 
+// Ordered block-wide compaction for large n with few matches: thread t owns
+// the contiguous elements [t * seg, (t + 1) * seg), counts its matches, one
+// block-wide scan gives each thread its first slot, and a second pass over
+// its own elements writes them.  `seg` is a multiple of 4 whose quarter is
+// odd, so the 16-byte loads of a warp start in eight different bank groups.
+// Elements i with pred(v) true go to out(slot, v), slots base, base + 1, ...
+// in increasing i.  `src.load4(i, v)` as for emit_ordered (readable up to the
+// next multiple of 4 past n).  `wsum`: 32 shared words.  Returns the next
+// free slot; ends with __syncthreads().
+template <class Src, class Pred, class Out>
+__device__ uint32_t compact_ordered(const Src &src, int n, const Pred &pred, const Out &out, uint32_t base,
+                                    uint32_t *wsum) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    int seg = ((n + static_cast<int>(blockDim.x) - 1) / static_cast<int>(blockDim.x) + 3) & ~3;
+    if (((seg >> 2) & 1) == 0) seg += 4;
+    const int lo = min(tid * seg, n), hi = min(lo + seg, n);
+    uint32_t cnt = 0;
+    for (int i = lo; i < hi; i += 4) {
+        uint64_t v[4];
+        src.load4(i, v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) cnt += (i + e < hi && pred(v[e])) ? 1u : 0u;
+    }
+    const uint32_t incl = warp_incl_scan(cnt);
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+        const uint32_t c = wsum[w];
+        before += (w < warp) ? c : 0u;
+        total += c;
+    }
+    uint32_t slot = base + before + incl - cnt;
+    if (cnt) {
+        for (int i = lo; i < hi; i += 4) {
+            uint64_t v[4];
+            src.load4(i, v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (i + e < hi && pred(v[e])) out(slot++, v[e]);
+        }
+    }
+    __syncthreads();
+    return base + total;
+}
+
 }  // namespace dsa

@@ -34,7 +34,8 @@ OP_FORWARD = 5
 ENTRY_POINTS = (
     "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk",
     "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill", "dsa_forward", "dsa_forward_paged",
-    "dsa_indexer_topk_static", "dsa_check_status", "dsa_last_error",
+    "dsa_indexer_topk_static", "dsa_project_workspace_size", "dsa_indexer_project",
+    "dsa_check_status", "dsa_last_error",
 )
 
 
@@ -49,6 +50,12 @@ class Params(ctypes.Structure):
                 ("h", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("max_n", ctypes.c_int32),
                 ("q_per_seq", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class ProjectParams(ctypes.Structure):
+    _fields_ = [("nt", ctypes.c_int32), ("hidden", ctypes.c_int32), ("q_lora_rank", ctypes.c_int32),
+                ("h_idx", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("rope_dim", ctypes.c_int32),
+                ("ln_eps", ctypes.c_float), ("rope_theta", ctypes.c_float)]
 
 
 class KV(ctypes.Structure):
@@ -85,6 +92,9 @@ def lib() -> ctypes.CDLL:
                 getattr(L, name).argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P,
                                              _P, _P, _P, ctypes.c_size_t, _P]
             L.dsa_indexer_topk_static.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, _P]
+            jp = ctypes.POINTER(ProjectParams)
+            L.dsa_project_workspace_size.argtypes = [jp, ctypes.POINTER(ctypes.c_size_t)]
+            L.dsa_indexer_project.argtypes = [jp, kp] + [_P] * 16 + [ctypes.c_size_t, _P]
             L.dsa_check_status.argtypes = [_P, _P]
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ENTRY_POINTS[:-1]:
@@ -184,6 +194,29 @@ def forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, ou
               _ptr(k_scale), _ptr(q), _ptr(kv_cache), int(kv_row_stride), _ptr(out), _ptr(lse),
               _ptr(idx_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "dsa_forward_paged" if paged else "dsa_forward")
+
+
+def make_project_params(*, nt, hidden, q_lora_rank, h_idx, d_idx, rope_dim=64, ln_eps=1e-6,
+                        rope_theta=10000.0) -> ProjectParams:
+    return ProjectParams(int(nt), int(hidden), int(q_lora_rank), int(h_idx), int(d_idx),
+                         int(rope_dim), float(ln_eps), float(rope_theta))
+
+
+def project_workspace_size(pp: ProjectParams) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().dsa_project_workspace_size(ctypes.byref(pp), ctypes.byref(out)),
+           "dsa_project_workspace_size")
+    return int(out.value)
+
+
+def indexer_project(pp, kv, x, q_lora, w_qb, w_k, w_proj, ln_gamma, ln_beta, positions, q_idx,
+                    q_scale, w, kidx_cache, k_scale, ws, q_f32=None, k_f32=None, w_f32=None,
+                    stream=None):
+    _check(lib().dsa_indexer_project(
+        ctypes.byref(pp), ctypes.byref(kv), _ptr(x), _ptr(q_lora), _ptr(w_qb), _ptr(w_k),
+        _ptr(w_proj), _ptr(ln_gamma), _ptr(ln_beta), _ptr(positions), _ptr(q_idx), _ptr(q_scale),
+        _ptr(w), _ptr(kidx_cache), _ptr(k_scale), _ptr(q_f32), _ptr(k_f32), _ptr(w_f32), _ptr(ws),
+        ws.numel() * ws.element_size(), _stream(stream)), "dsa_indexer_project")
 
 
 def check_status(ws, stream=None) -> int:

@@ -9,7 +9,9 @@ sides never have to agree on a quantisation step.
 Every tensor comes from its own PCG64 stream seeded by
 ``SeedSequence([1000 + config_id + seed_offset, stream])`` with these streams:
   0 context lengths, 1 page permutation, 2 q^I, 3 w, 4 k^I, 5 heavy-tail rows,
-  6 q (attention query), 7 latent KV, 8 per-row key scales.
+  6 q (attention query), 7 latent KV, 8 per-row key scales; and for the
+  indexer producer (make_project_inputs): 9 x, 10 q_lora, 11 W_qb, 12 W_k,
+  13 W_proj, 14 LayerNorm gamma / beta.
 Encodings: e4m3 via torch's float8_e4m3fn cast after clamping to +-448 (round
 to nearest even, saturating); bf16 via torch's round-to-nearest-even cast.
 """
@@ -282,3 +284,50 @@ def to_paged(inp: Inputs, *, config_id: Optional[int] = None, seed_offset: int =
             ks[phys] = inp.k_scale[src]
     return dataclasses.replace(inp, kidx=kidx, kv=kv, k_scale=ks, seq_row0=None,
                                page_table=pt, page_size=page_size)
+
+
+@dataclasses.dataclass
+class ProjectInputs:
+    """Inputs of the indexer producer for nt tokens (host, storage formats)."""
+    x: np.ndarray            # [nt, hidden] bf16 bits
+    q_lora: np.ndarray       # [nt, q_lora_rank] bf16 bits
+    w_qb: np.ndarray         # [h_idx * d_idx, q_lora_rank] bf16 bits
+    w_k: np.ndarray          # [d_idx, hidden] bf16 bits
+    w_proj: np.ndarray       # [h_idx, hidden] bf16 bits
+    ln_gamma: np.ndarray     # [d_idx] float32
+    ln_beta: np.ndarray      # [d_idx] float32
+    positions: np.ndarray    # [nt] int32
+    q_seq: np.ndarray        # [nt] int32 sequence of each token
+    h_idx: int
+    d_idx: int
+    rope_dim: int
+
+    @property
+    def nt(self) -> int:
+        return int(self.positions.shape[0])
+
+
+def make_project_inputs(positions, q_seq=None, *, hidden: int = 7168, q_lora_rank: int = 1536,
+                        h_idx: int = 64, d_idx: int = 128, rope_dim: int = 64,
+                        seed_offset: int = 0) -> ProjectInputs:
+    """Producer inputs at DeepSeek-V3.2 widths: x and q_lora ~ N(0,1); the
+    weights ~ N(0, 1/fan_in) ([out, in]); LayerNorm gamma ~ 1 + N(0, 0.1^2),
+    beta ~ N(0, 0.1^2); one token per entry of `positions` (its sequence in
+    q_seq, default 0)."""
+    positions = np.asarray(positions, np.int32)
+    nt = len(positions)
+    q_seq = np.zeros(nt, np.int32) if q_seq is None else np.asarray(q_seq, np.int32)
+    cid = 3
+    r = lambda stream: _rng(cid, seed_offset, stream)
+    x = _normal_bf16(r(9), (nt, hidden))
+    q_lora = _normal_bf16(r(10), (nt, q_lora_rank))
+    w_qb = encode_bf16(r(11).standard_normal((h_idx * d_idx, q_lora_rank), dtype=np.float32)
+                       * np.float32(q_lora_rank ** -0.5))
+    w_k = encode_bf16(r(12).standard_normal((d_idx, hidden), dtype=np.float32) * np.float32(hidden ** -0.5))
+    w_proj = encode_bf16(r(13).standard_normal((h_idx, hidden), dtype=np.float32) * np.float32(hidden ** -0.5))
+    g = r(14)
+    ln_gamma = (1.0 + 0.1 * g.standard_normal(d_idx)).astype(np.float32)
+    ln_beta = (0.1 * g.standard_normal(d_idx)).astype(np.float32)
+    return ProjectInputs(x=x, q_lora=q_lora, w_qb=w_qb, w_k=w_k, w_proj=w_proj, ln_gamma=ln_gamma,
+                         ln_beta=ln_beta, positions=positions, q_seq=q_seq, h_idx=h_idx, d_idx=d_idx,
+                         rope_dim=rope_dim)
