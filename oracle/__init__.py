@@ -74,6 +74,9 @@ def _load():
                 _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P, _P, _I32]
             lib.dsa_oracle_f64_to_e4m3.restype = ctypes.c_uint8
             lib.dsa_oracle_f64_to_e4m3.argtypes = [_F64]
+            lib.dsa_oracle_masked_mha.restype = ctypes.c_int
+            lib.dsa_oracle_masked_mha.argtypes = [
+                _I32, _I32, _I32, _I32, _F64, _P, _P, _P, _P, _P, _P, _P, _I32, _P, _P, _I32]
             lib.dsa_oracle_index_kl.restype = ctypes.c_int
             lib.dsa_oracle_index_kl.argtypes = [
                 _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _I64, _P,
@@ -303,6 +306,32 @@ def fold_weights(wp, q_scale, d_idx):
                                        _ptr(w_b)) != 0:
         raise RuntimeError("dsa_oracle_fold_weights failed")
     return w_f, w_b
+
+
+def masked_mha(q, k, v, q_seq, q_n, seq_row0, *, scale, idx=None, nthreads=0):
+    """Dense MHA attention over every visible position under the index set's
+    mask (idx None: no mask beyond s < q_n).  q [nq, H, d_qk], k [rows, H, d_qk],
+    v [rows, H, d_v] uint16 (bf16 bits).  Returns out [nq, H, d_v], lse [nq, H]
+    (fp64)."""
+    q = _c(q, np.uint16)
+    nq, h, d_qk = q.shape
+    k = _c(k, np.uint16)
+    v = _c(v, np.uint16)
+    d_v = v.shape[2]
+    assert k.shape[1] == h and v.shape[1] == h and k.shape[2] == d_qk and k.shape[0] == v.shape[0]
+    q_seq = _c(q_seq, np.int32)
+    q_n = _c(q_n, np.int32)
+    seq_row0 = _c(seq_row0, np.int64)
+    idx = _c(idx, np.int32)
+    topk = idx.shape[1] if idx is not None else 0
+    out = np.empty((nq, h, d_v), np.float64)
+    lse = np.empty((nq, h), np.float64)
+    rc = _load().dsa_oracle_masked_mha(nq, h, d_qk, d_v, float(scale), _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(idx), topk,
+                                       _ptr(out), _ptr(lse), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_masked_mha failed: %d" % rc)
+    return out, lse
 
 
 def index_kl(q, kv, q_seq, q_n, index_scores, *, scale, idx=None, seq_row0=None, page_table=None,

@@ -16,13 +16,17 @@
  *   [marsggbo]  "arXiv'25 | DSA lets DeepSeek-V3.2's long-context attention read
  *               less KV" (marsggbo.github.io), section 2 (toy example),
  *               section 3 (index score, TopK and attention equations),
- *               section 4 (MQA mode).
+ *               section 4 (MQA and MHA modes of MLA), sections 5.1 and 5.2
+ *               (the indexer's distillation loss), section 6 (masked MHA
+ *               for short prefill).
  *   [yuyanqi]   "DeepSeekV3.2之DSA" (yuyanqi.com), section 3.1 (symbol table),
  *               section 3.3 (TopK and the short-history rule), section 4.3
  *               (FP8 kernel comment: fp8 q.k -> relu * weights -> head sum ->
  *               * k_s), section 4.4 (topk(min(topk, end_pos)) returns indices),
  *               section 4.5 (skip scoring when the history fits in k),
  *               section 5.1 (softmax(q.[c_kv; k_pe]^T).c_kv).
+ *   [aicoding]  "从稠密到稀疏：DeepSeek-V3.2的DSA机制如何重塑Transformer效率边界"
+ *               (aicoding.csdn.net), section 4.3 (masked MHA below 8K tokens).
  *
  * Where the pages leave a step open, the reading taken is stated at the
  * function.  Parity is pinned by the tests under tests/ (toy example, brute
@@ -512,6 +516,83 @@ int dsa_oracle_index_kl(int32_t nq, int32_t h, int32_t d_qk, double scale, const
         }
         kl[qi] = acc;
         free(pos); free(S); free(a);
+    }
+    return bad ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Short prefill: the selection applied as a mask to dense MHA attention       */
+/* ------------------------------------------------------------------------- */
+
+/* For short prompts the DSA prefill runs as multi-head attention (each head
+ * with its own key and value: the MHA form of MLA used for prefill,
+ * [marsggbo] section 4) over every visible position, with a mask that keeps
+ * only what the indexer selected ([marsggbo] section 6: masked MHA emulates
+ * DSA for short-sequence prefill; [aicoding] section 4.3: masked MHA below
+ * 8K tokens).  For query t and head h:
+ *   keep[s] = s < q_n[t] and s is listed in idx[t, :]   (idx NULL: s < q_n[t])
+ *   S[s]    = scale * sum_{d < d_qk} q[t,h,d] * k[s,h,d]
+ *   out     = sum_{s kept} exp(S[s] - m) v[s,h,:] / sum_{s kept} exp(S[s] - m)
+ *   lse     = m + ln sum_{s kept} exp(S[s] - m),   m = max_{s kept} S[s]
+ * A mask holds membership, so a position listed twice is kept once; entries
+ * < 0 or >= q_n[t] are ignored.  Nothing kept: out = 0, lse = -inf.
+ * k [rows, h, d_qk] and v [rows, h, d_v] bf16; position s of sequence b is
+ * row seq_row0[b] + s. */
+int dsa_oracle_masked_mha(int32_t nq, int32_t h, int32_t d_qk, int32_t d_v, double scale,
+                          const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                          const int32_t *q_seq, const int32_t *q_n, const int64_t *seq_row0,
+                          const int32_t *idx, int32_t topk, double *out, double *lse,
+                          int32_t nthreads)
+{
+    if (nq < 0 || h <= 0 || d_qk <= 0 || d_v <= 0 || (idx && topk < 0)) return -1;
+    set_threads(nthreads);
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int32_t t = 0; t < nq; ++t) {
+        const int64_t n = q_n[t];
+        unsigned char *keep = (unsigned char *)calloc((size_t)(n > 0 ? n : 1), 1);
+        double *S = (double *)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+        if (!keep || !S) { bad |= 1; free(keep); free(S); continue; }
+        if (idx) {
+            for (int32_t i = 0; i < topk; ++i) {
+                const int32_t sv = idx[(int64_t)t * topk + i];
+                if (sv >= 0 && sv < n) keep[sv] = 1;
+            }
+        } else {
+            for (int64_t sv = 0; sv < n; ++sv) keep[sv] = 1;
+        }
+        const int64_t row0 = seq_row0[q_seq[t]];
+        for (int32_t hh = 0; hh < h; ++hh) {
+            const uint16_t *qv = q + ((int64_t)t * h + hh) * d_qk;
+            double m = -INFINITY;
+            for (int64_t sv = 0; sv < n; ++sv) {
+                if (!keep[sv]) continue;
+                const uint16_t *kr = k + ((row0 + sv) * h + hh) * d_qk;
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_qk; ++d)
+                    dot += dsa_oracle_bf16_to_f64(qv[d]) * dsa_oracle_bf16_to_f64(kr[d]);
+                S[sv] = scale * dot;
+                if (S[sv] > m) m = S[sv];
+            }
+            double *o = out + ((int64_t)t * h + hh) * d_v;
+            for (int32_t d = 0; d < d_v; ++d) o[d] = 0.0;
+            if (m == -INFINITY) {
+                lse[(int64_t)t * h + hh] = -INFINITY;
+                continue;
+            }
+            double z = 0.0;
+            for (int64_t sv = 0; sv < n; ++sv) {
+                if (!keep[sv]) continue;
+                const double e = exp(S[sv] - m);
+                const uint16_t *vr = v + ((row0 + sv) * h + hh) * d_v;
+                z += e;
+                for (int32_t d = 0; d < d_v; ++d) o[d] += e * dsa_oracle_bf16_to_f64(vr[d]);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] /= z;
+            lse[(int64_t)t * h + hh] = m + log(z);
+        }
+        free(keep);
+        free(S);
     }
     return bad ? -2 : 0;
 }
