@@ -113,7 +113,9 @@ typedef enum {
     DSA_OP_INDEXER_TOPK = 2,
     DSA_OP_SPARSE_MLA_DECODE = 3,
     DSA_OP_SPARSE_MLA_PREFILL = 4,
-    DSA_OP_FORWARD = 5
+    DSA_OP_FORWARD = 5,
+    DSA_OP_INDEX_KL_SPARSE = 6, /* dsa_index_kl with idx (topk entries per query) */
+    DSA_OP_INDEX_KL_DENSE = 7   /* dsa_index_kl without idx (every visible position) */
 } dsa_op;
 
 /* Bytes of scratch `ws` the given operation needs for this shape (host only,
@@ -183,8 +185,10 @@ int dsa_indexer_topk(const dsa_params *p, const dsa_kv *kv, const void *q_idx,
  * fp32; P enters the P.V product as a pair of bf16 tiles (P_hi + P_lo,
  * together exact to about 2^-16).  When a query's rows are split over
  * several CTAs, each split's normalised output is kept in ws as fp16 times
- * a power-of-two scale per 64 value columns (so any finite bf16 latent keeps
- * fp16's 11-bit precision) and the splits are merged by their log-sum-exp. */
+ * a power-of-two scale per 256 value columns (so a finite bf16 latent of any
+ * magnitude neither overflows fp16 nor falls under its normal range relative
+ * to its half row's largest value) and the splits are merged by their
+ * log-sum-exp. */
 int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q,
                           const void *kv_cache, int64_t kv_row_stride,
                           const int32_t *idx, void *out, float *lse, void *ws,
@@ -197,6 +201,39 @@ int dsa_sparse_mla_prefill(const dsa_params *p, const dsa_kv *kv, const void *q,
                            const void *kv_cache, int64_t kv_row_stride,
                            const int32_t *idx, void *out, float *lse, void *ws,
                            size_t ws_bytes, void *stream);
+
+/* The indexer's training signal, forward only: the distillation loss of each
+ * query t (DSA blog by marsggbo, section 5.1 for the dense warm-up, 5.2 for
+ * the sparse stage).  Over the set T_t (idx == NULL: every visible position
+ * s < q_n[t]; else the valid entries of idx[t, :], a position listed twice
+ * counting twice):
+ *   A_h[s] = softmax over T_t of scale * q[t, h] . c[s]   (each head's
+ *            attention distribution, MQA form as in dsa_sparse_mla_decode)
+ *   p[s]   = sum_h A_h[s] / sum_{s' in T_t} sum_h A_h[s']  (summed over
+ *            heads, L1-normalised along the sequence)
+ *   kl[t]  = sum_{s in T_t} p[s] * (ln p[s] - ln softmax_{T_t}(I[t, .])[s])
+ * A query whose set is empty gets kl = 0.  In the sparse stage each head is
+ * normalised over T_t, the set the main model attends to (the page does not
+ * say; this is the plain reading).
+ *   q, kv_cache, kv_row_stride, kv  as for dsa_sparse_mla_decode
+ *   index_scores [nq, ld_scores] fp32 (e.g. dsa_indexer_scores' output);
+ *                max_n <= ld_scores <= 2^27
+ *   idx          [nq, topk] int32 or NULL (the dense stage); entries < 0 are
+ *                skipped, entries >= q_n[t] flag DSA_ERR_DEVICE_CHECK
+ *   kl           [nq] fp32 output
+ *   p_out        [nq, ld_scores] fp32 output or NULL: p[s] at column s,
+ *                0 elsewhere (every column of the query's row is written)
+ *   ws           dsa_workspace_size(DSA_OP_INDEX_KL_SPARSE, or _DENSE when
+ *                idx is NULL)
+ * Arithmetic: the attention scores as in dsa_sparse_mla_decode (bf16
+ * products, fp32 accumulation, exp in fp32); each head's log-sum-exp is
+ * merged over the splits of the set, then the scores are recomputed and
+ * exp(S - lse) summed over heads in fp32; the normalisation, the index
+ * scores' softmax and the KL sum in fp64. */
+int dsa_index_kl(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
+                 int64_t kv_row_stride, const float *index_scores, int64_t ld_scores,
+                 const int32_t *idx, float *kl, float *p_out, void *ws, size_t ws_bytes,
+                 void *stream);
 
 /* Steps 1-3 in one call: fused indexer + TopK, then sparse attention, as in
  * the decode data flow of yuyanqi section 5.1.  idx_out [nq, topk] receives

@@ -173,7 +173,15 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
         // fit on chip.
         const int64_t p_par = P < dsa::kMaxChunks ? P : dsa::kMaxChunks;
         const int64_t sms = num_sms();
-        if (mode == dsa::kModeFused && p_par > 1 && p_par >= p_min &&
+        int64_t p_cap_merge = (200 * 1024) / (8 * static_cast<int64_t>(p->topk));
+        if (p_cap_merge > dsa::kMaxChunks) p_cap_merge = dsa::kMaxChunks;
+        const int64_t p_merge = P < p_cap_merge ? P : p_cap_merge;
+        // the merge (one CTA per group finishes the selection, the others
+        // exit) measured faster whenever it keeps nine tenths of the SMs
+        // streaming; the parallel selection serves the batches it cannot
+        // fill (a few long queries: it allows more chunks)
+        const bool merge_fills = p_merge >= p_min && 10 * static_cast<int64_t>(pl.n_groups) * p_merge >= 9 * sms;
+        if (mode == dsa::kModeFused && !merge_fills && p_par > 1 && p_par >= p_min &&
             static_cast<int64_t>(pl.n_groups) * p_par <= sms) {
             int64_t extra = 0;
             if (DSA_K1_FILL_SMS && p_par < dsa::kMaxChunks && p_par < p_small) {
@@ -270,10 +278,37 @@ MlaPlan plan_mla(const dsa_params *p) {
     return m;
 }
 
+// The distillation loss's set per query: topk entries of idx (sparse), or
+// every visible position (dense, up to max_n).  Splits of at most 256 rows,
+// as many as fill the SMs; no cap on their number (no output combine).
+MlaPlan plan_kl(const dsa_params *p, bool dense) {
+    MlaPlan m;
+    const int k = dense ? p->max_n : p->topk;
+    if (k <= 0) {
+        m.splits = 1;
+        m.rows_per_split = 16;
+        m.wave = p->nq;
+        return m;
+    }
+    const int s_min = (k + dsa::kMlaMaxRows - 1) / dsa::kMlaMaxRows;
+    const int s_fill = p->nq > 0 ? num_sms() / p->nq : 1;
+    const int s_small = (k + 63) / 64;
+    int s = s_fill < s_small ? s_fill : s_small;
+    if (s < s_min) s = s_min;
+    if (s < 1) s = 1;
+    int rps = (k + s - 1) / s;
+    rps = (rps + 15) / 16 * 16;
+    if (rps > dsa::kMlaMaxRows) rps = dsa::kMlaMaxRows;
+    m.rows_per_split = rps;
+    m.splits = (k + rps - 1) / rps;
+    m.wave = p->nq;
+    return m;
+}
+
 // -------------------------------------------------------------- workspace
 struct WsLayout {
     size_t status, ghist, gtot, published, cand, cand_cnt, cand_above, done, idx, part_o, part_lse,
-        part_scale, total;
+        part_scale, kl_lse, kl_a, total;
     size_t zero_begin, zero_end;  // cleared at the start of every call
 };
 
@@ -342,6 +377,21 @@ int layout_for(const dsa_params *p, int op, WsLayout &w, IndexerPlan *ipl, MlaPl
         m = plan_mla(p);
         off = mla_ws(p, m, off, w);
         break;
+    case DSA_OP_INDEX_KL_SPARSE:
+    case DSA_OP_INDEX_KL_DENSE: {
+        const bool dense = op == DSA_OP_INDEX_KL_DENSE;
+        const MlaPlan k = plan_kl(p, dense);
+        const int64_t entries = dense ? p->max_n : p->topk;
+        w.part_lse = off;
+        off = up(off + static_cast<size_t>(p->nq) * k.splits * 128 * 4, 256);
+        w.kl_lse = off;
+        off = up(off + static_cast<size_t>(p->nq) * 128 * 4, 256);
+        w.kl_a = off;
+        off = up(off + static_cast<size_t>(p->nq) * static_cast<size_t>(entries) * 4, 256);
+        w.total = off;
+        if (mpl) *mpl = k;
+        return DSA_OK;
+    }
     case DSA_OP_FORWARD:
         rc = plan_indexer(p, dsa::kModeFused, p->max_n, pl);
         if (rc) return rc;
@@ -415,6 +465,8 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
         // every CTA of the launch is resident at once (at most one per SM
         // is needed): each chunk selects its own part of the output
         a.parallel = pl.parallel ? 1 : 0;
+        const int64_t grid = static_cast<int64_t>(pl.n_big) * pl.P + static_cast<int64_t>(pl.n_groups - pl.n_big) * (pl.P - 1);
+        a.wait_hist = (!pl.parallel && grid <= num_sms()) ? 1 : 0;
         a.cand = at<uint64_t>(ws, wl.cand);
         a.cand_stride = cand_stride(p);
         a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
@@ -470,7 +522,6 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.page_size = kv->page_table ? kv->page_size : 0;
     a.cache_rows = kv->cache_rows;
     a.idx = idx;
-    a.q = static_cast<const uint16_t *>(q);
     a.kv = static_cast<const uint16_t *>(kv_cache);
     a.kv_row_stride = kv_row_stride;
     a.nq = p->nq;
@@ -677,6 +728,70 @@ int dsa_sparse_mla_prefill(const dsa_params *p, const dsa_kv *kv, const void *q,
                            size_t ws_bytes, void *stream) {
     return mla_common(DSA_OP_SPARSE_MLA_PREFILL, p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws,
                       ws_bytes, stream);
+}
+
+int dsa_index_kl(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
+                 int64_t kv_row_stride, const float *index_scores, int64_t ld_scores, const int32_t *idx,
+                 float *kl, float *p_out, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (rc) return rc;
+    if (p->nq > 0) {
+        if (!q || !kv_cache || !index_scores || !kl)
+            return fail(DSA_ERR_INVALID_ARG, "q / kv_cache / index_scores / kl is NULL");
+        if (!aligned(q, 16) || !aligned(kv_cache, 16)) return fail(DSA_ERR_INVALID_ARG, "q / kv_cache must be 16-byte aligned");
+        if (kv_row_stride < 576 || kv_row_stride % 8 != 0)
+            return fail(DSA_ERR_INVALID_ARG, "kv_row_stride must be >= 576 and a multiple of 8");
+    }
+    if (ld_scores < p->max_n || ld_scores > (int64_t(1) << 27)) return fail(DSA_ERR_INVALID_ARG, "ld_scores must be in [max_n, 2^27]");
+    const bool dense = idx == nullptr;
+    WsLayout wl;
+    MlaPlan m;
+    rc = layout_for(p, dense ? DSA_OP_INDEX_KL_DENSE : DSA_OP_INDEX_KL_SPARSE, wl, nullptr, &m, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    if (p->nq == 0) return DSA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    CUtensorMap qmap;
+    const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
+    rc = make_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dsa::kDqk, static_cast<uint64_t>(p->nq) * p->h,
+                     dsa::kDqk * 2, 64, hbox, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    dsa::MlaParams a;
+    memset(&a, 0, sizeof a);
+    a.q_seq = kv->q_seq;
+    a.q_n = kv->q_n;
+    a.seq_row0 = kv->seq_row0;
+    a.page_table = kv->page_table;
+    a.max_pages = kv->max_pages;
+    a.page_size = kv->page_table ? kv->page_size : 0;
+    a.cache_rows = kv->cache_rows;
+    a.idx = idx;
+    a.dense = dense ? 1 : 0;
+    a.kv = static_cast<const uint16_t *>(kv_cache);
+    a.kv_row_stride = kv_row_stride;
+    a.nq = p->nq;
+    a.h = p->h;
+    a.topk = dense ? p->max_n : p->topk;
+    a.splits = m.splits;
+    a.rows_per_split = m.rows_per_split;
+    a.scale = p->scale;
+    a.scale_log2 = p->scale * 1.4426950408889634f;
+    a.part_lse = at<float>(ws, wl.part_lse);
+    a.kl_lse = at<float>(ws, wl.kl_lse);
+    a.kl_a = at<float>(ws, wl.kl_a);
+    a.iscores = index_scores;
+    a.ld = ld_scores;
+    a.kl = kl;
+    a.p_out = p_out;
+    a.status = at<int>(ws, wl.status);
+    a.wait_budget = dsa::kWaitBudgetCycles;
+    cudaError_t e = dsa::launch_kl_pass(dsa::kMlaKlStats, qmap, a, st);
+    if (e == cudaSuccess) e = dsa::launch_kl_lse(a, st);
+    if (e == cudaSuccess) e = dsa::launch_kl_pass(dsa::kMlaKlSum, qmap, a, st);
+    if (e == cudaSuccess) e = dsa::launch_kl_reduce(a, st);
+    if (e != cudaSuccess) return cuda_fail(e, "distillation loss launch");
+    return DSA_OK;
 }
 
 int dsa_forward(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,

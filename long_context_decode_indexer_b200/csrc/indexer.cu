@@ -426,13 +426,21 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
     __syncthreads();
     if (threadIdx.x == 0) {
         atomicAdd(&a.gtot[q], static_cast<uint32_t>(len));
-        // Parallel mode: every chunk runs at the same time, so wait (bounded)
-        // until all of them have added their histograms.  Read the count
-        // BEFORE the snapshot: every chunk adds its histogram to G before its
-        // count to gtot, so a count that covers all n positions here proves
-        // the snapshot below complete.  (Read after the snapshot, it could
-        // cover chunks the snapshot missed.)
-        sm.sel_ok = a.parallel ? wait_count(&a.gtot[q], static_cast<uint32_t>(n), a.wait_budget) : 1;
+        // When every chunk runs at the same time, wait (bounded) until all of
+        // them have added their histograms: parallel selection needs the
+        // final threshold bin; the merge only gets a tighter candidate bound
+        // (any earlier snapshot is a valid, weaker one), so its wait is short
+        // and running out of it is no error.  Read the count BEFORE the
+        // snapshot: every chunk adds its histogram to G before its count to
+        // gtot, so a count that covers all n positions here proves the
+        // snapshot below complete.  (Read after the snapshot, it could cover
+        // chunks the snapshot missed.)
+        if (a.parallel) {
+            sm.sel_ok = wait_count(&a.gtot[q], static_cast<uint32_t>(n), a.wait_budget);
+        } else {
+            sm.sel_ok = 1;
+            if (a.wait_hist) wait_count(&a.gtot[q], static_cast<uint32_t>(n), kHistWaitCycles);
+        }
         sm.g_seen = ld_acquire_u32(&a.gtot[q]);
     }
     __syncthreads();

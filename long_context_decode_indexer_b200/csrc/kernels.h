@@ -12,6 +12,9 @@ namespace dsa {
 // A wait that runs out records DSA_ERR_TIMEOUT and abandons the work instead
 // of hanging the GPU.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
+// A merge-mode chunk waits at most this long (about 50 us) for the other
+// chunks' histograms; a shorter wait only weakens its candidate bound.
+constexpr long long kHistWaitCycles = 100000;
 
 // ---------------------------------------------------------------- indexer
 constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
@@ -22,13 +25,13 @@ constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 // 128 * DSA_K1_STAGE_TILES rows), ring depth, and whether the SMs a batch of
 // equal chunk counts leaves idle give some groups one more chunk.
 #ifndef DSA_K1_STAGE_TILES
-#define DSA_K1_STAGE_TILES 2
+#define DSA_K1_STAGE_TILES 1
 #endif
 #ifndef DSA_K1_FILL_SMS
 #define DSA_K1_FILL_SMS 1
 #endif
 constexpr int kK1MaxStages = 12;     // TMA ring barriers
-constexpr int kK1WantStages = 8 / DSA_K1_STAGE_TILES;  // ring depth used when shared memory allows
+constexpr int kK1WantStages = kK1MaxStages / DSA_K1_STAGE_TILES;  // ring depth used when shared memory allows
 constexpr int kK1MaxAcc = 4;         // TMEM accumulator buffers (even: one parity per epilogue group)
 constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
@@ -75,6 +78,7 @@ struct K1Params {
     uint32_t *ghist;      // [nq, 2048] global top-digit histograms
     uint32_t *gtot;       // [nq] positions counted into ghist so far
     int32_t parallel;     // every CTA is co-resident: each chunk selects its own part exactly
+    int32_t wait_hist;    // merge selection with every CTA co-resident: wait (briefly) for the full histogram
     uint64_t *cand;       // [nq, P, cand_stride] candidate composites
     int32_t cand_stride;  // topk rounded up to a multiple of 4 (32-byte aligned chunk lists)
     int32_t *cand_cnt;    // [nq, P]
@@ -143,12 +147,13 @@ cudaError_t launch_topk(const K1Params &a, cudaStream_t st);
 constexpr int kDqk = 576;           // key width (512 latent + 64 rope)
 constexpr int kDv = 512;            // value width
 constexpr int kMlaHeads = 128;      // MMA M: heads per CTA (zero-padded)
-constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit: S takes <= 256 TMEM columns)
-constexpr int kMlaBlockRows = 32;   // pass 1: rows per ring block (MMA N)
-constexpr int kMlaRing = 4;         // pass 1: ring depth (blocks of 32 whole rows)
+constexpr int kMlaMaxRows = 256;    // KV rows per CTA (split size limit)
+constexpr int kMlaStages = 4;       // pass-1 ring depth (Q chunk + K chunk)
+constexpr int kMlaVRows = 32;       // rows per pass-2 V tile
+constexpr int kMlaVStages = 3;      // pass-2 ring depth
 constexpr int kMlaMaxSplits = 32;   // splits per query (the combine kernel's warp reads one LSE per lane)
-constexpr int kMlaThreads = 448;    // warps 0-3 group A, 4-7 group B, 8-11 group C, 12 MMA, 13 rope-Q TMA
-constexpr int kMlaScaleBlocks = 8;  // power-of-two scales per partial row (one per 64 value columns)
+constexpr int kMlaScaleBlocks = 2;  // power-of-two scales per partial row (one per 256 value columns)
+constexpr int kMlaThreads = 320;    // warps 0-3 softmax/epilogue, 4 Q TMA, 5 MMA, 6-9 row gathers (0-3 help in pass 1)
 
 struct MlaParams {
     const int32_t *q_seq;
@@ -158,7 +163,6 @@ struct MlaParams {
     int32_t max_pages, page_size;
     int64_t cache_rows;
     const int32_t *idx;  // [nq, topk]
-    const uint16_t *q;   // [nq, h, 576] bf16 bits
     const uint16_t *kv;  // latent cache (bf16 bits)
     int64_t kv_row_stride;  // elements between cache rows
     int32_t nq, h, topk;
@@ -172,32 +176,55 @@ struct MlaParams {
     float *lse;          // [nq, h]
     uint16_t *part_o;    // [wave_q, splits, 128, d_v] normalised partial outputs / part_scale (fp16 bits)
     float *part_lse;     // [wave_q, splits, 128]
-    float *part_scale;   // [wave_q, splits, 128, 8] power of two of each 64-column block of part_o
+    float *part_scale;   // [wave_q, splits, 128, 2] power of two of each half row of part_o
     int *status;
     long long wait_budget;  // bounded waits, SM cycles
     int32_t inject;         // tests only: the first CTA's gathers skip one arrival
+    // indexer distillation loss (the attention's first pass reused)
+    int32_t dense;          // entries are positions e (every visible one) instead of idx[q, e]
+    int64_t ld;             // columns of iscores / p_out
+    float *kl_lse;          // [nq, 128] each head's log-sum-exp over the whole set
+    float *kl_a;            // [nq, topk] head-summed attention probability of each entry
+    const float *iscores;   // [nq, ld] index scores
+    float *kl;              // [nq] the loss
+    float *p_out;           // [nq, ld] the target distribution, or null
 };
 
+// What the attention kernel computes: the attention itself, or one of the
+// two passes of the indexer distillation loss over the same rows.
+constexpr int kMlaAttn = 0;
+constexpr int kMlaKlStats = 1;  // each (split, head)'s log-sum-exp of the scaled scores
+constexpr int kMlaKlSum = 2;    // each entry's attention probability summed over heads
+
 struct MlaLayout {
-    uint32_t ring, vq, rope, misc, total;
+    uint32_t ring, p_tile, p_lo, v_ring, misc, total;
 };
 
 __host__ __device__ inline MlaLayout mla_layout() {
     MlaLayout L;
-    const uint32_t block = kMlaBlockRows * kDqk * 2u;  // 36 KB: 9 chunks of [32 rows x 64 cols]
-    const uint32_t pass1 = kMlaRing * block;
-    const uint32_t vq = kMlaMaxRows * 256u;            // a value quarter (128 cols) of 256 rows: 64 KB
+    // pass 1: kMlaStages x (Q chunk 128x64 bf16 = 16 KB + K chunk 256x64 bf16 = 32 KB)
+    const uint32_t stage = 128u * 128u + kMlaMaxRows * 128u;
+    const uint32_t pass1 = kMlaStages * stage;
+    // pass 2: P as a hi + lo pair of bf16 tiles (128 x 256 each, 64 KB each)
+    // + kMlaVStages V tiles (32 rows x 512 bf16 = 32 KB each)
+    const uint32_t ptile = 128u * kMlaMaxRows * 2u;
+    const uint32_t vtile = kMlaVRows * kDv * 2u;
     L.ring = 0;
-    L.vq = 0;                                          // pass 2 reuses the ring: two quarter buffers
-    const uint32_t end = pass1 > 2 * vq ? pass1 : 2 * vq;
-    L.rope = align_up(end, 1024);                      // Q columns 512..575, 128 heads x 128 B
-    L.misc = L.rope + 128u * 128u;
-    L.total = L.misc + 4096 + 1024;                    // barriers, row table, exchanges; alignment slack
+    L.p_tile = 0;
+    L.p_lo = ptile;
+    L.v_ring = 2 * ptile;
+    const uint32_t pass2 = 2 * ptile + kMlaVStages * vtile;
+    uint32_t end = pass1 > pass2 ? pass1 : pass2;
+    L.misc = align_up(end, 128);
+    L.total = L.misc + 2048 + 1024;  // barriers and row table, alignment slack
     return L;
 }
 
 cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st);
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st);
+cudaError_t launch_kl_pass(int mode, const CUtensorMap &qmap, const MlaParams &a, cudaStream_t st);
+cudaError_t launch_kl_lse(const MlaParams &a, cudaStream_t st);
+cudaError_t launch_kl_reduce(const MlaParams &a, cudaStream_t st);
 
 // ------------------------------------------------ indexer producer (q^I, k^I, w)
 constexpr int kProjStages = 4;  // TMA ring depth of the projection GEMM

@@ -29,13 +29,15 @@ OP_INDEXER_TOPK = 2
 OP_SPARSE_MLA_DECODE = 3
 OP_SPARSE_MLA_PREFILL = 4
 OP_FORWARD = 5
+OP_INDEX_KL_SPARSE = 6
+OP_INDEX_KL_DENSE = 7
 
 # Entry points declared in include/dsa.h.
 ENTRY_POINTS = (
     "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk",
     "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill", "dsa_forward", "dsa_forward_paged",
     "dsa_indexer_topk_static", "dsa_project_workspace_size", "dsa_indexer_project",
-    "dsa_check_status", "dsa_last_error",
+    "dsa_index_kl", "dsa_check_status", "dsa_last_error",
 )
 
 
@@ -95,6 +97,8 @@ def lib() -> ctypes.CDLL:
             jp = ctypes.POINTER(ProjectParams)
             L.dsa_project_workspace_size.argtypes = [jp, ctypes.POINTER(ctypes.c_size_t)]
             L.dsa_indexer_project.argtypes = [jp, kp] + [_P] * 16 + [ctypes.c_size_t, _P]
+            L.dsa_index_kl.argtypes = [pp, kp, _P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _P, _P,
+                                       _P, ctypes.c_size_t, _P]
             L.dsa_check_status.argtypes = [_P, _P]
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ENTRY_POINTS[:-1]:
@@ -185,6 +189,17 @@ def sparse_mla_prefill(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, str
                                         int(kv_row_stride), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
                                         ws.numel() * ws.element_size(), _stream(stream)),
            "dsa_sparse_mla_prefill")
+
+
+def index_kl(p, kv, q, kv_cache, kv_row_stride, index_scores, ld_scores, idx, kl, p_out, ws,
+             stream=None):
+    """Indexer distillation loss per query; idx None selects the dense stage
+    (every visible position), else the sparse stage over idx's entries."""
+    _check(lib().dsa_index_kl(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(kv_cache),
+                              int(kv_row_stride), _ptr(index_scores), int(ld_scores), _ptr(idx),
+                              _ptr(kl), _ptr(p_out), _ptr(ws), ws.numel() * ws.element_size(),
+                              _stream(stream)),
+           "dsa_index_kl")
 
 
 def forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, out, lse, idx_out,
