@@ -11,7 +11,9 @@ Every tensor comes from its own PCG64 stream seeded by
   0 context lengths, 1 page permutation, 2 q^I, 3 w, 4 k^I, 5 heavy-tail rows,
   6 q (attention query), 7 latent KV, 8 per-row key scales; and for the
   indexer producer (make_project_inputs): 9 x, 10 q_lora, 11 W_qb, 12 W_k,
-  13 W_proj, 14 LayerNorm gamma / beta.
+  13 W_proj, 14 LayerNorm gamma / beta; and for the masked-MHA short prefill
+  (make_mha_inputs): 15 q, 16 k, 17 v; and for the FP8 latent cache
+  (make_fp8_latent): 18 codes, 19 row exponents.
 Encodings: e4m3 via torch's float8_e4m3fn cast after clamping to +-448 (round
 to nearest even, saturating); bf16 via torch's round-to-nearest-even cast.
 """
@@ -331,3 +333,45 @@ def make_project_inputs(positions, q_seq=None, *, hidden: int = 7168, q_lora_ran
     return ProjectInputs(x=x, q_lora=q_lora, w_qb=w_qb, w_k=w_k, w_proj=w_proj, ln_gamma=ln_gamma,
                          ln_beta=ln_beta, positions=positions, q_seq=q_seq, h_idx=h_idx, d_idx=d_idx,
                          rope_dim=rope_dim)
+
+
+@dataclasses.dataclass
+class MhaInputs:
+    """Per-head MHA q / k / v of one prefill sequence (bf16 bits)."""
+    q: np.ndarray          # [L, h, d_qk]
+    k: np.ndarray          # [L, h, d_qk]
+    v: np.ndarray          # [L, h, d_v]
+    q_seq: np.ndarray      # [L] int32 (all 0)
+    q_n: np.ndarray        # [L] int32: token t sees s < t
+    seq_row0: np.ndarray   # [1] int64
+    scale: float
+
+
+def make_mha_inputs(L: int, *, h: int = 128, d_qk: int = 192, d_v: int = 128,
+                    seed_offset: int = 0) -> MhaInputs:
+    """MHA-form prefill activations for one sequence of L tokens (the short
+    prefill's masked MHA): q, k, v ~ N(0, 1) bf16, token t visible positions
+    s < t (as the causal prefill workload), softmax scale d_qk^-1/2.  Drawn
+    from the causal-prefill workload's seed."""
+    cid = 4
+    r = lambda stream: _rng(cid, seed_offset, stream)
+    q = _normal_bf16(r(15), (L, h, d_qk))
+    k = _normal_bf16(r(16), (L, h, d_qk))
+    v = _normal_bf16(r(17), (L, h, d_v))
+    return MhaInputs(q=q, k=k, v=v, q_seq=np.zeros(L, np.int32), q_n=np.arange(L, dtype=np.int32),
+                     seq_row0=np.zeros(1, np.int64), scale=float(d_qk) ** -0.5)
+
+
+def make_fp8_latent(rows: int, *, d_qk: int = D_QK, config_id: int = 3, seed_offset: int = 0):
+    """An FP8 latent cache of `rows` rows: e4m3 codes of N(0,1) draws
+    ([rows, d_qk] uint8) and one power-of-two scale per row, 2^U{-3..3}
+    ([rows] fp32).  A row stands for code * scale."""
+    r = lambda stream: _rng(config_id, seed_offset, stream)
+    codes = np.empty((rows, d_qk), np.uint8)
+    g = r(18)
+    step = max(1, (1 << 24) // d_qk)
+    for i in range(0, rows, step):
+        j = min(rows, i + step)
+        codes[i:j] = encode_e4m3(g.standard_normal((j - i, d_qk), dtype=np.float32))
+    scale = np.ldexp(np.float32(1.0), r(19).integers(-3, 4, size=rows)).astype(np.float32)
+    return codes, scale

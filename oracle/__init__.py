@@ -64,6 +64,10 @@ def _load():
             lib.dsa_oracle_sparse_mla.argtypes = [
                 _I32, _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P,
                 _I32, _I32, _P, _I32, _P, _P, _I32]
+            lib.dsa_oracle_sparse_mla_fp8.restype = ctypes.c_int
+            lib.dsa_oracle_sparse_mla_fp8.argtypes = [
+                _I32, _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P, _P,
+                _I32, _I32, _P, _I32, _P, _P, _I32]
             lib.dsa_oracle_dense_mla.restype = ctypes.c_int
             lib.dsa_oracle_dense_mla.argtypes = [
                 _I32, _I32, _I32, _I32, _F64, _P, _P, _I64, _P, _P, _P, _P,
@@ -188,6 +192,30 @@ def sparse_mla(q, kv, idx, q_seq, q_n, *, scale, d_v=512, seq_row0=None,
         page_size, _ptr(idx), k, _ptr(out), _ptr(lse), nthreads)
     if rc != 0:
         raise RuntimeError("dsa_oracle_sparse_mla failed: %d" % rc)
+    return out, lse
+
+
+def sparse_mla_fp8(q, kv8, kv_scale, idx, q_seq, q_n, *, scale, d_v=512, seq_row0=None,
+                   page_table=None, page_size=0, nthreads=0):
+    """Sparse attention over an FP8 latent cache: kv8 [rows, row_bytes] uint8
+    e4m3 codes (the first d_qk used), kv_scale [rows] fp32.  Returns out
+    [nq, H, d_v], lse [nq, H] (fp64)."""
+    q = _c(q, np.uint16)
+    nq, h, d_qk = q.shape
+    kv8 = _c(kv8, np.uint8)
+    kv_scale = _c(kv_scale, np.float32)
+    idx = _c(idx, np.int32)
+    k = idx.shape[1] if idx.ndim == 2 else 0
+    q_seq, q_n, seq_row0, page_table, max_pages, page_size = _kv_args(
+        q_seq, q_n, seq_row0, page_table, page_size)
+    out = np.empty((nq, h, d_v), np.float64)
+    lse = np.empty((nq, h), np.float64)
+    rc = _load().dsa_oracle_sparse_mla_fp8(
+        nq, h, d_qk, d_v, float(scale), _ptr(q), _ptr(kv8), kv8.shape[1], _ptr(kv_scale),
+        _ptr(q_seq), _ptr(q_n), _ptr(seq_row0), _ptr(page_table), max_pages,
+        page_size, _ptr(idx), k, _ptr(out), _ptr(lse), nthreads)
+    if rc != 0:
+        raise RuntimeError("dsa_oracle_sparse_mla_fp8 failed: %d" % rc)
     return out, lse
 
 

@@ -330,6 +330,74 @@ int dsa_oracle_sparse_mla(int32_t nq, int32_t h, int32_t d_qk, int32_t d_v,
     return bad ? -2 : 0;
 }
 
+/* The same attention over an FP8 latent cache.  Reading (the pages give FP8
+ * only for the indexer's keys, [marsggbo] section 3 and [yuyanqi] section
+ * 4.3): each latent row is stored in that same format, d_qk e4m3 codes and
+ * one power-of-two scale per row (the pages' e8m0 k_s), and stands for
+ *   c[s, d] = e4m3(code[s, d]) * kv_scale[row of s]
+ * Everything else is dsa_oracle_sparse_mla's definition.  kv8 row r starts
+ * at kv8 + r * kv8_row_bytes. */
+int dsa_oracle_sparse_mla_fp8(int32_t nq, int32_t h, int32_t d_qk, int32_t d_v,
+                              double scale, const uint16_t *q, const uint8_t *kv8,
+                              int64_t kv8_row_bytes, const float *kv_scale,
+                              const int32_t *q_seq, const int32_t *q_n,
+                              const int64_t *seq_row0, const int32_t *page_table,
+                              int32_t max_pages, int32_t page_size, const int32_t *idx,
+                              int32_t k, double *out, double *lse, int32_t nthreads)
+{
+    if (nq < 0 || h <= 0 || d_qk <= 0 || d_v <= 0 || d_v > d_qk || k < 0)
+        return -1;
+    set_threads(nthreads);
+    int bad = 0;
+
+#pragma omp parallel for collapse(2) schedule(dynamic, 1) reduction(| : bad)
+    for (int32_t qi = 0; qi < nq; ++qi) {
+        for (int32_t hh = 0; hh < h; ++hh) {
+            const uint16_t *qv = q + ((int64_t)qi * h + hh) * d_qk;
+            double *o = out + ((int64_t)qi * h + hh) * d_v;
+            double *S = (double *)malloc((size_t)(k > 0 ? k : 1) * sizeof(double));
+            int64_t *rows = (int64_t *)malloc((size_t)(k > 0 ? k : 1) * sizeof(int64_t));
+            if (!S || !rows) { bad |= 1; free(S); free(rows); continue; }
+            int32_t cnt = 0;
+            for (int32_t i = 0; i < k; ++i) {
+                int32_t s = idx[(int64_t)qi * k + i];
+                if (s < 0 || s >= q_n[qi]) continue;
+                rows[cnt++] = cache_row(q_seq[qi], s, seq_row0, page_table,
+                                        max_pages, page_size);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] = 0.0;
+            if (cnt == 0) {
+                lse[(int64_t)qi * h + hh] = -INFINITY;
+                free(S); free(rows);
+                continue;
+            }
+            double m = -INFINITY;
+            for (int32_t i = 0; i < cnt; ++i) {
+                const uint8_t *c = kv8 + rows[i] * kv8_row_bytes;
+                const double sc = (double)kv_scale[rows[i]];
+                double dot = 0.0;
+                for (int32_t d = 0; d < d_qk; ++d)
+                    dot += dsa_oracle_bf16_to_f64(qv[d]) * (dsa_oracle_e4m3_to_f64(c[d]) * sc);
+                S[i] = scale * dot;
+                if (S[i] > m) m = S[i];
+            }
+            double denom = 0.0;
+            for (int32_t i = 0; i < cnt; ++i) {
+                double p = exp(S[i] - m);
+                const uint8_t *c = kv8 + rows[i] * kv8_row_bytes;
+                const double sc = (double)kv_scale[rows[i]];
+                denom += p;
+                for (int32_t d = 0; d < d_v; ++d) o[d] += p * (dsa_oracle_e4m3_to_f64(c[d]) * sc);
+            }
+            for (int32_t d = 0; d < d_v; ++d) o[d] /= denom;
+            lse[(int64_t)qi * h + hh] = m + log(denom);
+            free(S);
+            free(rows);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
 /* Dense attention over the whole visible history 0..q_n-1, with no index
  * list: the textbook MQA softmax attention.  When the history has at most k
  * positions DSA keeps all of them ([yuyanqi] section 3.3), so the sparse path
