@@ -115,7 +115,8 @@ typedef enum {
     DSA_OP_SPARSE_MLA_PREFILL = 4,
     DSA_OP_FORWARD = 5,
     DSA_OP_INDEX_KL_SPARSE = 6, /* dsa_index_kl with idx (topk entries per query) */
-    DSA_OP_INDEX_KL_DENSE = 7   /* dsa_index_kl without idx (every visible position) */
+    DSA_OP_INDEX_KL_DENSE = 7,  /* dsa_index_kl without idx (every visible position) */
+    DSA_OP_MASKED_MHA = 8       /* dsa_masked_mha_prefill */
 } dsa_op;
 
 /* Bytes of scratch `ws` the given operation needs for this shape (host only,
@@ -194,12 +195,59 @@ int dsa_sparse_mla_decode(const dsa_params *p, const dsa_kv *kv, const void *q,
                           const int32_t *idx, void *out, float *lse, void *ws,
                           size_t ws_bytes, void *stream);
 
+/* Step 3 over an FP8 latent cache (half the bytes of every gathered row).
+ * The pages give FP8 only for the indexer's keys (e4m3 with a per-row e8m0
+ * scale, yuyanqi section 4.3); the latent cache here uses that same format,
+ * a reading of ours: row r holds d_qk e4m3 codes and stands for
+ *   c[r, d] = e4m3(kv8_cache[r * kv8_row_bytes + d]) * kv_scale[r]
+ * with kv_scale[r] a power of two (then every c is exact in bf16 and the
+ * result is that of dsa_sparse_mla_decode on the bf16 cache of those values).
+ *   kv8_cache     [cache_rows, kv8_row_bytes] e4m3 codes, 16-byte aligned;
+ *                 kv8_row_bytes >= 576 and a multiple of 16
+ *   kv_scale      [cache_rows] fp32
+ * Everything else (arguments, ws, errors, arithmetic) as for
+ * dsa_sparse_mla_decode. */
+int dsa_sparse_mla_decode_fp8(const dsa_params *p, const dsa_kv *kv, const void *q,
+                              const void *kv8_cache, int64_t kv8_row_bytes,
+                              const float *kv_scale, const int32_t *idx, void *out,
+                              float *lse, void *ws, size_t ws_bytes, void *stream);
+
 /* Step 3 scheduled for many queries of one sequence (causal prefill, where
  * token t sees n = t positions).  Same arguments and results as
  * dsa_sparse_mla_decode. */
 int dsa_sparse_mla_prefill(const dsa_params *p, const dsa_kv *kv, const void *q,
                            const void *kv_cache, int64_t kv_row_stride,
                            const int32_t *idx, void *out, float *lse, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/* Short prefill as masked MHA: dense multi-head attention over every visible
+ * position with the index set applied as a mask, the form the pages give
+ * DSA for short prompts (DSA blog by marsggbo, section 6; aicoding.csdn.net
+ * DSA article, section 4.3: below 8K tokens).  MHA form of MLA (marsggbo,
+ * section 4): every head has its own key and value rows.  For query t, head h:
+ *   keep[s] = s < q_n[t] and s listed in idx[t, :]  (idx NULL: every s < q_n[t])
+ *   out[t,h] = sum_{s kept} softmax(scale * q[t,h] . k[s,h]) v[s,h]
+ *   lse[t,h] = ln sum_{s kept} exp(scale * q[t,h] . k[s,h])
+ * A position listed twice is kept once (a mask holds membership); nothing
+ * kept gives out = 0 and lse = -inf.
+ *   p      d_qk = per-head q/k width (64, 128 or 192), d_v = per-head v width
+ *          (64 or 128), h heads, topk = idx columns, max_n >= every q_n
+ *          (<= 2^20), q_per_seq: queries come in blocks of q_per_seq
+ *          consecutive queries of one sequence (a prefill of L tokens: L);
+ *          h_idx / d_idx are not read
+ *   kv     q_seq, q_n, seq_row0 (contiguous layout only); cache_rows = rows
+ *          of k and v; position s of sequence b is row seq_row0[b] + s (rows
+ *          past cache_rows read as zero)
+ *   q      [nq, h, d_qk] bf16;  k [cache_rows, h, d_qk] bf16;
+ *   v      [cache_rows, h, d_v] bf16 (all 16-byte aligned)
+ *   idx    [nq, topk] int32 (e.g. dsa_indexer_topk's output) or NULL;
+ *          entries < 0 are skipped, entries >= q_n[t] flag DSA_ERR_DEVICE_CHECK
+ *   out    [nq, h, d_v] bf16;  lse [nq, h] fp32
+ *   ws     dsa_workspace_size(DSA_OP_MASKED_MHA): the membership bitmap
+ * Arithmetic as in dsa_sparse_mla_decode: bf16 products, fp32 accumulation,
+ * softmax in fp32 with P as a bf16 pair (P_hi + P_lo). */
+int dsa_masked_mha_prefill(const dsa_params *p, const dsa_kv *kv, const void *q, const void *k,
+                           const void *v, const int32_t *idx, void *out, float *lse, void *ws,
                            size_t ws_bytes, void *stream);
 
 /* The indexer's training signal, forward only: the distillation loss of each

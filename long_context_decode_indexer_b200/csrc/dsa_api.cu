@@ -84,6 +84,20 @@ int make_map_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, uint64_
     return DSA_OK;
 }
 
+int make_map_3d(CUtensorMap *m, CUtensorMapDataType dt, const void *ptr, const uint64_t (&dims)[3],
+                const uint64_t (&stride_bytes)[2], const uint32_t (&box)[3], CUtensorMapSwizzle swz) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+    cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t st[2] = {stride_bytes[0], stride_bytes[1]};
+    cuuint32_t bx[3] = {box[0], box[1], box[2]};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, dt, 3, const_cast<void *>(ptr), d, st, bx, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return DSA_OK;
+}
+
 int num_sms() {
     static int sms = 0;
     static std::once_flag once;
@@ -111,6 +125,23 @@ int check_params(const dsa_params *p) {
     if (!isfinite(p->scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite");
     return DSA_OK;
 }
+
+// The masked-MHA prefill reads d_qk / d_v as the per-head MHA widths.
+int check_params_mha(const dsa_params *p) {
+    if (!p) return fail(DSA_ERR_INVALID_ARG, "params is NULL");
+    if (p->nq < 0) return fail(DSA_ERR_INVALID_ARG, "nq < 0");
+    if (p->h < 1 || p->h > (1 << 16)) return fail(DSA_ERR_INVALID_ARG, "h must be in [1, 65536]");
+    if (p->d_qk != 64 && p->d_qk != 128 && p->d_qk != 192)
+        return fail(DSA_ERR_UNSUPPORTED, "masked MHA: d_qk must be 64, 128 or 192");
+    if (p->d_v != 64 && p->d_v != 128) return fail(DSA_ERR_UNSUPPORTED, "masked MHA: d_v must be 64 or 128");
+    if (p->topk < 1 || p->topk > 2048) return fail(DSA_ERR_INVALID_ARG, "topk must be in [1, 2048]");
+    if (p->max_n < 0 || p->max_n > (1 << 20)) return fail(DSA_ERR_INVALID_ARG, "masked MHA: max_n must be in [0, 2^20]");
+    if (p->q_per_seq < 1) return fail(DSA_ERR_INVALID_ARG, "q_per_seq must be >= 1");
+    if (!isfinite(p->scale)) return fail(DSA_ERR_INVALID_ARG, "scale must be finite");
+    return DSA_OK;
+}
+
+int mha_mask_words(const dsa_params *p) { return 4 * ((p->max_n + dsa::kMhaTile - 1) / dsa::kMhaTile); }
 
 int check_kv(const dsa_params *p, const dsa_kv *kv) {
     if (!kv) return fail(DSA_ERR_INVALID_ARG, "kv is NULL");
@@ -392,6 +423,11 @@ int layout_for(const dsa_params *p, int op, WsLayout &w, IndexerPlan *ipl, MlaPl
         if (mpl) *mpl = k;
         return DSA_OK;
     }
+    case DSA_OP_MASKED_MHA:
+        w.idx = off;  // the membership bitmap
+        off = up(off + static_cast<size_t>(p->nq) * mha_mask_words(p) * 4, 256);
+        w.total = off;
+        return DSA_OK;
     case DSA_OP_FORWARD:
         rc = plan_indexer(p, dsa::kModeFused, p->max_n, pl);
         if (rc) return rc;
@@ -504,7 +540,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
 
 int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv_cache,
             int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
-            const WsLayout &wl, const MlaPlan &m, cudaStream_t st) {
+            const WsLayout &wl, const MlaPlan &m, cudaStream_t st, const float *kv_scale = nullptr) {
     if (p->nq == 0) return DSA_OK;
     CUtensorMap qmap;
     const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
@@ -522,8 +558,16 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     a.page_size = kv->page_table ? kv->page_size : 0;
     a.cache_rows = kv->cache_rows;
     a.idx = idx;
-    a.kv = static_cast<const uint16_t *>(kv_cache);
-    a.kv_row_stride = kv_row_stride;
+    // an FP8 cache (kv_scale set): kv_cache holds e4m3 codes, kv_row_stride bytes apart
+    const bool kv8 = kv_scale != nullptr;
+    if (kv8) {
+        a.kv8 = static_cast<const uint8_t *>(kv_cache);
+        a.kv8_row_bytes = kv_row_stride;
+        a.kv_scale = kv_scale;
+    } else {
+        a.kv = static_cast<const uint16_t *>(kv_cache);
+        a.kv_row_stride = kv_row_stride;
+    }
     a.nq = p->nq;
     a.h = p->h;
     a.topk = p->topk;
@@ -545,7 +589,7 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
     for (int q0 = 0; q0 < p->nq; q0 += m.wave) {
         const int nw = (p->nq - q0) < m.wave ? (p->nq - q0) : m.wave;
         a.q0 = q0;
-        cudaError_t e = dsa::launch_sparse_mla(qmap, a, nw, st);
+        cudaError_t e = dsa::launch_sparse_mla(qmap, a, nw, st, kv8);
         if (e != cudaSuccess) return cuda_fail(e, "sparse MLA launch");
         e = dsa::launch_mla_combine(a, nw, st);
         if (e != cudaSuccess) return cuda_fail(e, "split combine launch");
@@ -629,7 +673,7 @@ ProjPlan plan_project(const dsa_project_params *pp) {
 extern "C" {
 
 int dsa_workspace_size(const dsa_params *p, const dsa_kv *kv, int op, size_t *bytes) {
-    int rc = check_params(p);
+    int rc = op == DSA_OP_MASKED_MHA ? check_params_mha(p) : check_params(p);
     if (rc) return rc;
     if (!bytes) return fail(DSA_ERR_INVALID_ARG, "bytes is NULL");
     if (op != DSA_OP_TOPK) {
@@ -792,6 +836,97 @@ int dsa_index_kl(const dsa_params *p, const dsa_kv *kv, const void *q, const voi
     if (e == cudaSuccess) e = dsa::launch_kl_reduce(a, st);
     if (e != cudaSuccess) return cuda_fail(e, "distillation loss launch");
     return DSA_OK;
+}
+
+int dsa_masked_mha_prefill(const dsa_params *p, const dsa_kv *kv, const void *q, const void *k, const void *v,
+                           const int32_t *idx, void *out, float *lse, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params_mha(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (rc) return rc;
+    if (kv->page_table) return fail(DSA_ERR_UNSUPPORTED, "masked MHA: k / v are contiguous (seq_row0), not paged");
+    if (p->nq > 0) {
+        if (!q || !k || !v || !out || !lse) return fail(DSA_ERR_INVALID_ARG, "q / k / v / out / lse is NULL");
+        if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+            return fail(DSA_ERR_INVALID_ARG, "q / k / v / out must be 16-byte aligned");
+        if (static_cast<int64_t>(p->nq) + dsa::kMhaTile >= (int64_t(1) << 31))
+            return fail(DSA_ERR_INVALID_ARG, "nq too large");
+    }
+    WsLayout wl;
+    rc = layout_for(p, DSA_OP_MASKED_MHA, wl, nullptr, nullptr, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    if (p->nq == 0) return DSA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const uint64_t H = static_cast<uint64_t>(p->h);
+    CUtensorMap qmap, kmap, vmap;
+    rc = make_map_3d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, {static_cast<uint64_t>(p->d_qk), H, static_cast<uint64_t>(p->nq)},
+                     {static_cast<uint64_t>(p->d_qk) * 2, H * p->d_qk * 2}, {64, 1, dsa::kMhaTile},
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!rc)
+        rc = make_map_3d(&kmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k,
+                         {static_cast<uint64_t>(p->d_qk), H, static_cast<uint64_t>(kv->cache_rows)},
+                         {static_cast<uint64_t>(p->d_qk) * 2, H * p->d_qk * 2}, {64, 1, dsa::kMhaTile},
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!rc)
+        rc = make_map_3d(&vmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v,
+                         {static_cast<uint64_t>(p->d_v), H, static_cast<uint64_t>(kv->cache_rows)},
+                         {static_cast<uint64_t>(p->d_v) * 2, H * p->d_v * 2}, {64, 1, dsa::kMhaTile},
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    dsa::MhaParams a;
+    memset(&a, 0, sizeof a);
+    a.q_seq = kv->q_seq;
+    a.q_n = kv->q_n;
+    a.seq_row0 = kv->seq_row0;
+    a.mask_words = mha_mask_words(p);
+    uint32_t *mask = idx ? at<uint32_t>(ws, wl.idx) : nullptr;
+    a.mask = mask;
+    a.nq = p->nq;
+    a.h = p->h;
+    a.d_qk = p->d_qk;
+    a.d_v = p->d_v;
+    a.max_n = p->max_n;
+    a.q_per_seq = p->q_per_seq;
+    a.tiles_per_block = (p->q_per_seq + dsa::kMhaTile - 1) / dsa::kMhaTile;
+    a.scale_log2 = p->scale * 1.4426950408889634f;
+    a.out = static_cast<uint16_t *>(out);
+    a.lse = lse;
+    a.status = at<int>(ws, wl.status);
+    a.wait_budget = dsa::kWaitBudgetCycles;
+    int stages = dsa::kMhaMaxStages;
+    while (stages > 1 && dsa::mha_layout(p->d_qk, p->d_v, stages).total > 232448) --stages;
+    a.stages = stages;
+    const int64_t blocks = (static_cast<int64_t>(p->nq) + p->q_per_seq - 1) / p->q_per_seq;
+    const int64_t grid = blocks * a.tiles_per_block * p->h;
+    if (grid >= (int64_t(1) << 31)) return fail(DSA_ERR_UNSUPPORTED, "masked MHA: grid too large");
+    cudaError_t e = cudaSuccess;
+    if (idx) e = dsa::launch_mha_mask(idx, p->topk, kv->q_n, mask, a.mask_words, p->nq, a.status, st);
+    if (e == cudaSuccess) e = dsa::launch_masked_mha(qmap, kmap, vmap, a, static_cast<int>(grid), st);
+    if (e != cudaSuccess) return cuda_fail(e, "masked MHA launch");
+    return DSA_OK;
+}
+
+int dsa_sparse_mla_decode_fp8(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv8_cache,
+                              int64_t kv8_row_bytes, const float *kv_scale, const int32_t *idx, void *out,
+                              float *lse, void *ws, size_t ws_bytes, void *stream) {
+    int rc = check_params(p);
+    if (!rc) rc = check_kv(p, kv);
+    if (rc) return rc;
+    if (p->nq > 0) {
+        if (!q || !kv8_cache || !kv_scale || !idx || !out || !lse)
+            return fail(DSA_ERR_INVALID_ARG, "q / kv8_cache / kv_scale / idx / out / lse is NULL");
+        if (!aligned(q, 16) || !aligned(kv8_cache, 16) || !aligned(out, 16))
+            return fail(DSA_ERR_INVALID_ARG, "q / kv8_cache / out must be 16-byte aligned");
+        if (kv8_row_bytes < 576 || kv8_row_bytes % 16 != 0)
+            return fail(DSA_ERR_INVALID_ARG, "kv8_row_bytes must be >= 576 and a multiple of 16");
+    }
+    WsLayout wl;
+    MlaPlan m;
+    rc = layout_for(p, DSA_OP_SPARSE_MLA_DECODE, wl, nullptr, &m, p->max_n);
+    if (!rc) rc = check_ws(ws, ws_bytes, wl);
+    if (rc) return rc;
+    return run_mla(p, kv, q, kv8_cache, kv8_row_bytes, idx, out, lse, ws, wl, m, static_cast<cudaStream_t>(stream),
+                   kv_scale);
 }
 
 int dsa_forward(const dsa_params *p, const dsa_kv *kv, const void *q_idx, const void *w,

@@ -776,12 +776,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 uint32_t ph = 0, aph = 0;
                 bool failed = false;
                 for (int u = 0; u < nst && !failed; ++u) {
-                    if (!mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
-                        failed = true;
-                        break;
-                    }
-                    for (int sub = 0; sub < kStageTiles && kStageTiles * u + sub < ntiles; ++sub) {
-                        if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) || sm.abort) {
+                    const int nsub = min(kStageTiles, ntiles - kStageTiles * u);
+                    for (int sub = 0; sub < nsub; ++sub) {
+                        if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
+                            (sub == 0 && !mbar_wait(&sm.full[s], ph, a.wait_budget)) || sm.abort) {
                             failed = true;
                             break;
                         }
@@ -791,11 +789,13 @@ __global__ void __launch_bounds__(kK1Threads, 1)
 #pragma unroll
                         for (int kk = 0; kk < DI / 32; ++kk)
                             mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                        // release the ring slot first (its refill paces the
+                        // stream), then hand the accumulator over
+                        if (sub == nsub - 1) tc_commit(&sm.empty[s]);
                         tc_commit(&sm.acc_full[b]);
                         if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
                     }
                     if (failed) break;
-                    tc_commit(&sm.empty[s]);
                     if (++s == a.stages) { s = 0; ph ^= 1; }
                 }
                 if (failed) {

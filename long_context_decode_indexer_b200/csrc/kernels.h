@@ -165,6 +165,9 @@ struct MlaParams {
     const int32_t *idx;  // [nq, topk]
     const uint16_t *kv;  // latent cache (bf16 bits)
     int64_t kv_row_stride;  // elements between cache rows
+    const uint8_t *kv8;     // FP8 latent cache (e4m3 codes), when the cache is stored in FP8
+    const float *kv_scale;  // [cache_rows] power-of-two scale of each FP8 row
+    int64_t kv8_row_bytes;  // bytes between FP8 cache rows
     int32_t nq, h, topk;
     int32_t splits;      // CTAs per query along the index list
     int32_t rows_per_split;
@@ -220,11 +223,62 @@ __host__ __device__ inline MlaLayout mla_layout() {
     return L;
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st);
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st,
+                              bool kv8 = false);
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st);
 cudaError_t launch_kl_pass(int mode, const CUtensorMap &qmap, const MlaParams &a, cudaStream_t st);
 cudaError_t launch_kl_lse(const MlaParams &a, cudaStream_t st);
 cudaError_t launch_kl_reduce(const MlaParams &a, cudaStream_t st);
+
+// --------------------------------------------- masked MHA (short prefill)
+// Dense multi-head attention of 128-query tiles over 128-key tiles, the
+// index set applied as a membership mask.  One CTA per (query tile, head).
+constexpr int kMhaTile = 128;      // queries per CTA (MMA M) and keys per tile (MMA N)
+constexpr int kMhaThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax + epilogue
+constexpr int kMhaMaxStages = 3;   // K ring depth limit (the V ring has 2 slots)
+constexpr int kMhaVStages = 2;
+
+struct MhaParams {
+    const int32_t *q_seq;
+    const int32_t *q_n;
+    const int64_t *seq_row0;
+    const uint32_t *mask;   // [nq, mask_words] bit s of row t: s is in t's index set; null: every s < q_n
+    int32_t mask_words;     // 4 * ceil(max_n / 128)
+    int32_t nq, h, d_qk, d_v;
+    int32_t max_n;          // q_n above this flags DSA_ERR_DEVICE_CHECK and is clamped
+    int32_t q_per_seq;      // queries are in blocks of q_per_seq of one sequence; a tile stays in its block
+    int32_t tiles_per_block;
+    float scale_log2;
+    uint16_t *out;          // [nq, h, d_v] bf16
+    float *lse;             // [nq, h]
+    int *status;
+    long long wait_budget;
+    int32_t stages;         // K ring depth
+};
+
+// Q, then a K ring (released as soon as S(j) is computed) and a V ring
+// (released after P(j) . V(j)), in 128-row x 64-column swizzled chunks.
+struct MhaLayout {
+    uint32_t q, k_ring, k_stage, v_ring, v_stage, misc, total;
+};
+
+__host__ __device__ inline MhaLayout mha_layout(int d_qk, int d_v, int stages) {
+    MhaLayout L;
+    const uint32_t chunk = kMhaTile * 128u;  // 128 rows x 64 bf16 columns, 128B-swizzled
+    L.q = 0;
+    L.k_stage = static_cast<uint32_t>(d_qk / 64) * chunk;
+    L.v_stage = static_cast<uint32_t>(d_v / 64) * chunk;
+    L.k_ring = L.k_stage;
+    L.v_ring = L.k_ring + static_cast<uint32_t>(stages) * L.k_stage;
+    L.misc = L.v_ring + kMhaVStages * L.v_stage;
+    L.total = L.misc + 1024 + 1024;  // barriers, alignment slack
+    return L;
+}
+
+cudaError_t launch_mha_mask(const int32_t *idx, int topk, const int32_t *q_n, uint32_t *mask, int words, int nq,
+                            int *status, cudaStream_t st);
+cudaError_t launch_masked_mha(const CUtensorMap &qmap, const CUtensorMap &kmap, const CUtensorMap &vmap,
+                              const MhaParams &a, int grid, cudaStream_t st);
 
 // ------------------------------------------------ indexer producer (q^I, k^I, w)
 constexpr int kProjStages = 4;  // TMA ring depth of the projection GEMM

@@ -50,6 +50,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -123,6 +124,75 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const uint32_t a = __bfloat16_as_ushort(__float2bfloat16_rn(lo));
     const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(hi));
     return a | (b << 16);
+}
+
+// Eight e4m3 codes (one 8-byte load) times a power-of-two row scale as eight
+// bf16 values (a 16-byte shared-memory piece).  e4m3 -> f16 is exact, the
+// power-of-two product is exact in fp32 and a value with 4 significant bits
+// is exact in bf16: the piece equals the cache's value, with no rounding.
+__device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 codes, float sc) {
+    const uint32_t w[2] = {codes.x, codes.y};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
+        const __half2 h = __half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3));
+        const float2 f = __half22float2(h);
+        o[i] = pack_bf16x2(f.x * sc, f.y * sc);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ uint2 ldg_u2(const uint8_t *p) {
+    return __ldg(reinterpret_cast<const uint2 *>(p));
+}
+
+// Pass-1 gathers from an FP8 cache: the same piece ownership as the bf16
+// gather below, with the 8 codes of a piece loaded into registers two
+// chunks ahead, converted, and stored into the swizzled stage; a chunk is
+// published once this thread's stores of it are done.
+__device__ bool gather_pass1_fp8(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int gt, int Rp) {
+    const int j = gt & 7, r0 = gt >> 3, lane = threadIdx.x & 31;
+    const uint8_t *src[kPass1Rows];
+    uint32_t dst[kPass1Rows];
+    float sc[kPass1Rows];
+#pragma unroll
+    for (int k = 0; k < kPass1Rows; ++k) {
+        const int r = r0 + 32 * k;
+        src[k] = a.kv8 + static_cast<int64_t>(sm.rows[r]) * a.kv8_row_bytes + j * 8;
+        dst[k] = static_cast<uint32_t>(r * 128 + ((j ^ (r & 7)) << 4));
+        sc[k] = sm.valid[r] ? a.kv_scale[sm.rows[r]] : 0.f;
+    }
+    constexpr int kAhead = 2;
+    uint2 buf[kAhead + 1][kPass1Rows];
+    auto load = [&](int c, uint2 (&b)[kPass1Rows]) {
+#pragma unroll
+        for (int k = 0; k < kPass1Rows; ++k)
+            b[k] = (r0 + 32 * k < Rp) ? ldg_u2(src[k] + c * 64) : make_uint2(0u, 0u);
+    };
+#pragma unroll
+    for (int c = 0; c < kAhead; ++c) load(c, buf[c]);
+    bool ok = true;
+#pragma unroll
+    for (int c = 0; c < kNumKChunks; ++c) {
+        if (c + kAhead < kNumKChunks) load(c + kAhead, buf[(c + kAhead) % (kAhead + 1)]);
+        const int s = c % kMlaStages;
+        const uint32_t ph = (c / kMlaStages) & 1;
+        ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) && !sm.abort);
+        if (ok) {
+            uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
+#pragma unroll
+            for (int k = 0; k < kPass1Rows; ++k)
+                if (r0 + 32 * k < Rp)
+                    *reinterpret_cast<uint4 *>(kst + dst[k]) = fp8x8_to_bf16x8(buf[c % (kAhead + 1)][k], sc[k]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        // tests only: the first CTA never publishes chunk 0
+        const bool skip = a.inject != 0 && blockIdx.x == 0 && c == 0;
+        if (lane == 0 && !skip) mbar_arrive(&sm.full[s]);
+    }
+    return ok;
 }
 
 // Pass-1 row gathers by one of the kPass1Threads gather threads (gt): it
@@ -252,7 +322,7 @@ __device__ __forceinline__ float warp_column_sum(float (&v)[32]) {
 
 }  // namespace
 
-template <int MODE>
+template <int MODE, bool KV8>
 __global__ void __launch_bounds__(kMlaThreads, 1)
     k3_sparse_mla(const __grid_constant__ CUtensorMap qmap, const MlaParams a) {
     extern __shared__ uint8_t smem_raw[];
@@ -370,9 +440,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             // ------------------------------------------ row gathers (cp.async)
             const int gt = tid - kGatherWarp0 * 32;  // 0..127
             for (int i = gt; i < R; i += kGatherThreads)
-                if (sm.valid[i])
-                    prefetch_l2_bulk(a.kv + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
-            bool ok = gather_pass1(a, sm, ring, kPass1Threads / 2 + gt, Rp);
+                if (sm.valid[i]) {
+                    if constexpr (KV8)
+                        prefetch_l2_bulk(a.kv8 + static_cast<int64_t>(sm.rows[i]) * a.kv8_row_bytes, kDqk);
+                    else
+                        prefetch_l2_bulk(a.kv + static_cast<int64_t>(sm.rows[i]) * a.kv_row_stride, kDqk * 2);
+                }
+            bool ok = KV8 ? gather_pass1_fp8(a, sm, ring, kPass1Threads / 2 + gt, Rp)
+                          : gather_pass1(a, sm, ring, kPass1Threads / 2 + gt, Rp);
             if constexpr (MODE != kMlaAttn) {
                 if (!ok && lane == 0) {
                     record_status(a.status, DSA_ERR_TIMEOUT);
@@ -385,29 +460,66 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.s_full, 0, a.wait_budget) && !sm.abort);
                 const int vr = gt >> 2, vu = gt & 3;
                 const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
-                for (int vt = 0; vt < nvt + kVLag; ++vt) {
-                    if (vt < nvt) {
+                if constexpr (KV8) {
+                    // FP8 rows: this thread's 16 pieces of row vr of a tile,
+                    // loaded into registers one tile ahead and converted
+                    uint2 cur[16], nxt[16];
+                    float csc = 0.f, nsc = 0.f;
+                    auto vload = [&](int vt, uint2 (&b)[16], float &sc) {
+                        const int rr = vt * kMlaVRows + vr;
+                        const uint8_t *vsrc = a.kv8 + static_cast<int64_t>(sm.rows[rr]) * a.kv8_row_bytes;
+                        sc = sm.valid[rr] ? a.kv_scale[sm.rows[rr]] : 0.f;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) b[m] = ldg_u2(vsrc + (vu + 4 * m) * 8);
+                    };
+                    if (nvt > 0) vload(0, cur, csc);
+                    for (int vt = 0; vt < nvt; ++vt) {
+                        if (vt + 1 < nvt) vload(vt + 1, nxt, nsc);
                         const int v = vt % kMlaVStages;
                         const uint32_t ph = (vt / kMlaVStages) & 1;
                         ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1, a.wait_budget) && !sm.abort);
                         if (ok) {
                             uint8_t *vdst = vring + v * kVTileBytes + vr * 128;
-                            const uint16_t *vsrc = a.kv + static_cast<int64_t>(sm.rows[vt * kMlaVRows + vr]) * a.kv_row_stride;
 #pragma unroll
                             for (int m = 0; m < 16; ++m) {
-                                const int pc = vu + 4 * m;  // 16-byte piece of the 512 value columns
+                                const int pc = vu + 4 * m;
                                 const int blk = pc >> 3, j = pc & 7;
-                                cp_async16(vdst + blk * kVBlockBytes + ((j ^ (vr & 7)) << 4), vsrc + pc * 8);
+                                *reinterpret_cast<uint4 *>(vdst + blk * kVBlockBytes + ((j ^ (vr & 7)) << 4)) =
+                                    fp8x8_to_bf16x8(cur[m], csc);
                             }
                         }
-                        cp_async_commit();
-                    }
-                    if (vt >= kVLag && vt - kVLag < nvt) {
-                        if (vt < nvt) cp_async_wait<kVLag>();
-                        else cp_async_wait<0>();
                         fence_proxy_async_smem();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(&sm.v_full[(vt - kVLag) % kMlaVStages]);
+                        if (lane == 0) mbar_arrive(&sm.v_full[v]);
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) cur[m] = nxt[m];
+                        csc = nsc;
+                    }
+                } else {
+                    for (int vt = 0; vt < nvt + kVLag; ++vt) {
+                        if (vt < nvt) {
+                            const int v = vt % kMlaVStages;
+                            const uint32_t ph = (vt / kMlaVStages) & 1;
+                            ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.v_empty[v], ph ^ 1, a.wait_budget) && !sm.abort);
+                            if (ok) {
+                                uint8_t *vdst = vring + v * kVTileBytes + vr * 128;
+                                const uint16_t *vsrc = a.kv + static_cast<int64_t>(sm.rows[vt * kMlaVRows + vr]) * a.kv_row_stride;
+#pragma unroll
+                                for (int m = 0; m < 16; ++m) {
+                                    const int pc = vu + 4 * m;  // 16-byte piece of the 512 value columns
+                                    const int blk = pc >> 3, j = pc & 7;
+                                    cp_async16(vdst + blk * kVBlockBytes + ((j ^ (vr & 7)) << 4), vsrc + pc * 8);
+                                }
+                            }
+                            cp_async_commit();
+                        }
+                        if (vt >= kVLag && vt - kVLag < nvt) {
+                            if (vt < nvt) cp_async_wait<kVLag>();
+                            else cp_async_wait<0>();
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&sm.v_full[(vt - kVLag) % kMlaVStages]);
+                        }
                     }
                 }
                 if (!ok && lane == 0) {
@@ -505,7 +617,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
             }
         } else if (warp < 4) {
             // ------------------- pass-1 gathers, softmax, then epilogue
-            bool ok = gather_pass1(a, sm, ring, tid, Rp);
+            bool ok = KV8 ? gather_pass1_fp8(a, sm, ring, tid, Rp) : gather_pass1(a, sm, ring, tid, Rp);
             const int hrow = warp * 32 + lane;  // head = TMEM lane
             const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
             ok = __all_sync(0xffffffffu, ok && mbar_wait(&sm.s_full, 0, a.wait_budget) && !sm.abort);
@@ -841,15 +953,16 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, size_
     return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st) {
+cudaError_t launch_sparse_mla(const CUtensorMap &qmap, const MlaParams &a, int nq_wave, cudaStream_t st,
+                              bool kv8) {
     const MlaLayout L = mla_layout();
     const size_t smem = smem_for_tmem(L.total, 512);
-    cudaError_t e = cudaFuncSetAttribute(k3_sparse_mla<kMlaAttn>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    auto kern = kv8 ? k3_sparse_mla<kMlaAttn, true> : k3_sparse_mla<kMlaAttn, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int grid = nq_wave * a.splits;
     if (grid == 0) return cudaSuccess;
-    return launch_pdl(k3_sparse_mla<kMlaAttn>, grid, kMlaThreads, smem, st, qmap, a);
+    return launch_pdl(kern, grid, kMlaThreads, smem, st, qmap, a);
 }
 
 cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st) {
@@ -861,7 +974,7 @@ cudaError_t launch_mla_combine(const MlaParams &a, int nq_wave, cudaStream_t st)
 cudaError_t launch_kl_pass(int mode, const CUtensorMap &qmap, const MlaParams &a, cudaStream_t st) {
     const MlaLayout L = mla_layout();
     const size_t smem = smem_for_tmem(L.total, 512);
-    auto kern = mode == kMlaKlStats ? k3_sparse_mla<kMlaKlStats> : k3_sparse_mla<kMlaKlSum>;
+    auto kern = mode == kMlaKlStats ? k3_sparse_mla<kMlaKlStats, false> : k3_sparse_mla<kMlaKlSum, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int64_t grid = static_cast<int64_t>(a.nq) * a.splits;

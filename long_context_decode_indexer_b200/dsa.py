@@ -31,13 +31,15 @@ OP_SPARSE_MLA_PREFILL = 4
 OP_FORWARD = 5
 OP_INDEX_KL_SPARSE = 6
 OP_INDEX_KL_DENSE = 7
+OP_MASKED_MHA = 8
 
 # Entry points declared in include/dsa.h.
 ENTRY_POINTS = (
     "dsa_workspace_size", "dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk",
     "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill", "dsa_forward", "dsa_forward_paged",
     "dsa_indexer_topk_static", "dsa_project_workspace_size", "dsa_indexer_project",
-    "dsa_index_kl", "dsa_check_status", "dsa_last_error",
+    "dsa_index_kl", "dsa_masked_mha_prefill", "dsa_sparse_mla_decode_fp8",
+    "dsa_check_status", "dsa_last_error",
 )
 
 
@@ -99,6 +101,9 @@ def lib() -> ctypes.CDLL:
             L.dsa_indexer_project.argtypes = [jp, kp] + [_P] * 16 + [ctypes.c_size_t, _P]
             L.dsa_index_kl.argtypes = [pp, kp, _P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _P, _P,
                                        _P, ctypes.c_size_t, _P]
+            L.dsa_masked_mha_prefill.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
+            L.dsa_sparse_mla_decode_fp8.argtypes = [pp, kp, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P,
+                                                    ctypes.c_size_t, _P]
             L.dsa_check_status.argtypes = [_P, _P]
             L.dsa_last_error.restype = ctypes.c_char_p
             for name in ENTRY_POINTS[:-1]:
@@ -184,6 +189,15 @@ def sparse_mla_decode(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, stre
            "dsa_sparse_mla_decode")
 
 
+def sparse_mla_decode_fp8(p, kv, q, kv8_cache, kv8_row_bytes, kv_scale, idx, out, lse, ws, stream=None):
+    """Sparse attention over an FP8 latent cache (e4m3 codes, power-of-two row scales)."""
+    _check(lib().dsa_sparse_mla_decode_fp8(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(kv8_cache),
+                                           int(kv8_row_bytes), _ptr(kv_scale), _ptr(idx), _ptr(out),
+                                           _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                                           _stream(stream)),
+           "dsa_sparse_mla_decode_fp8")
+
+
 def sparse_mla_prefill(p, kv, q, kv_cache, kv_row_stride, idx, out, lse, ws, stream=None):
     _check(lib().dsa_sparse_mla_prefill(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(kv_cache),
                                         int(kv_row_stride), _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
@@ -200,6 +214,14 @@ def index_kl(p, kv, q, kv_cache, kv_row_stride, index_scores, ld_scores, idx, kl
                               _ptr(kl), _ptr(p_out), _ptr(ws), ws.numel() * ws.element_size(),
                               _stream(stream)),
            "dsa_index_kl")
+
+
+def masked_mha_prefill(p, kv, q, k, v, idx, out, lse, ws, stream=None):
+    """Dense MHA under the index set's mask (idx None: causal only)."""
+    _check(lib().dsa_masked_mha_prefill(ctypes.byref(p), ctypes.byref(kv), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(idx), _ptr(out), _ptr(lse), _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_masked_mha_prefill")
 
 
 def forward(p, kv, q_idx, w, kidx_cache, k_scale, q, kv_cache, kv_row_stride, out, lse, idx_out,
