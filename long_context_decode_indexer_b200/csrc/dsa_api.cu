@@ -234,7 +234,7 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     }
     // chunks are whole ring stages; each group cuts its own span the same
     // way on the device (no larger than this)
-    const int64_t srows = 128 * DSA_K1_STAGE_TILES;
+    const int64_t srows = 128;
     chunk_max = chunk_max / srows * srows;
     const int64_t pc = p_cut > 0 ? p_cut : P;
     int64_t chunk = (sp + pc - 1) / pc;
@@ -264,7 +264,7 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
     // (the merge area reuses the ring once streaming is over)
     pl.stages = 0;
     if (mode != dsa::kModeTopk) {
-        int st = dsa::kK1WantStages;
+        int st = dsa::kK1MaxStages;
         while (st >= 2 &&
                dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st, !pl.parallel).total > 232448)
             --st;
@@ -527,8 +527,8 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.page_size = kv->page_table ? kv->page_size : 0;
     a.cache_rows = kv->cache_rows;
     CUtensorMap kmap;
-    // one box per ring stage, or one per page
-    const uint32_t box_rows = kv->page_table ? static_cast<uint32_t>(kv->page_size) : 128u * DSA_K1_STAGE_TILES;
+    // one box per 128-row tile, or one per page
+    const uint32_t box_rows = kv->page_table ? static_cast<uint32_t>(kv->page_size) : 128u;
     int rc = make_map_2d(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, kidx_cache, p->d_idx, kv->cache_rows,
                          p->d_idx, p->d_idx, box_rows,
                          p->d_idx == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);

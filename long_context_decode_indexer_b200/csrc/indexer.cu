@@ -52,9 +52,7 @@ namespace dsa {
 
 namespace {
 
-constexpr int kTileRows = 128;            // positions per MMA (M) and per epilogue tile
-constexpr int kStageTiles = DSA_K1_STAGE_TILES;  // tiles per TMA ring stage (one box)
-constexpr int kStageRows = kStageTiles * kTileRows;
+constexpr int kTileRows = 128;  // positions per ring stage, MMA (M) and epilogue tile
 
 struct K1Smem {
     uint64_t full[kK1MaxStages];
@@ -636,7 +634,6 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     int q0, nqg;
     group_queries(a, g, q0, nqg);
     constexpr int kTileBytes = kTileRows * DI;
-    constexpr int kStageBytes = kStageRows * DI;
     const int N = a.qg * HP;  // MMA N (columns per accumulator buffer)
 
     // ---- set-up
@@ -649,38 +646,37 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     }
     const int seq = nqg > 0 ? a.q_seq[q0] : 0;
     const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
-    const int chunk = min(a.chunk, ((span + Pg - 1) / Pg + kStageRows - 1) / kStageRows * kStageRows);
+    const int chunk = min(a.chunk, ((span + Pg - 1) / Pg + kTileRows - 1) / kTileRows * kTileRows);
     const int start = c * chunk;
     const int end = min(start + chunk, span);
     const int len = max(end - start, 0);
     const int ntiles = (len + kTileRows - 1) / kTileRows;
-    const int nst = (ntiles + kStageTiles - 1) / kStageTiles;  // ring stages of 256 rows
 
     // The producer (thread 0) fills the TMA ring as soon as its barriers
     // exist, so the first tiles are in flight during the rest of the set-up.
     const int64_t row0 = (a.page_table == nullptr && nqg > 0) ? a.seq_row0[seq] : 0;
-    // tests only: the first CTA never loads its first stage, so the MMA
+    // tests only: the first CTA never loads its first tile, so the MMA
     // issuer's wait for it runs out
     const bool skip_first = a.inject != 0 && blockIdx.x == 0;
-    // stage u holds tiles 2u and 2u + 1: one 256-row box (contiguous cache;
-    // a box past the end of the cache reads zeros), or one box per page
-    auto issue_stage = [&](int u, int s) {
-        if (skip_first && u == 0) return;
-        const int p0 = start + u * kStageRows;
-        uint8_t *dst = stages + s * kStageBytes;
+    // tile t: one 128-row box (contiguous cache; a box past the end of the
+    // cache reads zeros), or one box per page
+    auto issue_tile = [&](int t, int s) {
+        if (skip_first && t == 0) return;
+        const int p0 = start + t * kTileRows;
+        uint8_t *dst = stages + s * kTileBytes;
         if (a.page_table == nullptr) {
-            mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+            mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
             tma_load_2d(dst, &kmap, &sm.full[s], 0, static_cast<int32_t>(row0 + p0));
         } else {
             const int box = a.page_size;
             const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages + p0 / box;
             int n_box = 0;
-            for (int h = 0; h < kStageRows / box; ++h) n_box += (p0 + h * box < nmax);
+            for (int h = 0; h < kTileRows / box; ++h) n_box += (p0 + h * box < nmax);
             mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
             for (int h = 0; h < n_box; ++h, dst += box * DI) tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[h] * box);
         }
     };
-    const int n_pro = min(nst, a.stages);  // stages issued before the set-up barrier
+    const int n_pro = min(ntiles, a.stages);  // tiles issued before the set-up barrier
 
     if (tid == 0) {
         sm.abort = 0;
@@ -698,7 +694,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b % 2
         }
         fence_mbar_init();
-        for (int u = 0; u < n_pro; ++u) issue_stage(u, u);
+        for (int t = 0; t < n_pro; ++t) issue_tile(t, t);
         sm.chunk_c = c;
         sm.chunk_P = Pg;
     }
@@ -740,27 +736,27 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     if (ntiles > 0) {
         if (warp == 0) {
             if (lane == 0) {
-                // ring position (s, ph) advances by one per stage: no divisions
+                // ring position (s, ph) advances by one per tile: no divisions
                 // in this single-thread loop, which paces the whole stream
                 int s = n_pro == a.stages ? 0 : n_pro;
                 uint32_t ph = n_pro == a.stages ? 1u : 0u;
-                int u_end = n_pro;  // stages issued (or skipped) so far
-                for (int u = n_pro; u < nst; ++u) {
+                int t_end = n_pro;  // tiles issued (or skipped) so far
+                for (int t = n_pro; t < ntiles; ++t) {
                     if (!mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         break;
                     }
-                    issue_stage(u, s);
-                    u_end = u + 1;
+                    issue_tile(t, s);
+                    t_end = t + 1;
                     if (++s == a.stages) { s = 0; ph ^= 1; }
                 }
                 // before the CTA may exit, every load issued must have landed:
                 // wait (bounded) for the newest phase of each stage (a no-op
                 // when the MMA consumed them all)
-                for (int u = max(u_end - a.stages, 0); u < u_end; ++u)
-                    if (!(skip_first && u == 0) &&
-                        !mbar_wait(&sm.full[u % a.stages], static_cast<uint32_t>(u / a.stages) & 1u, a.wait_budget))
+                for (int t = max(t_end - a.stages, 0); t < t_end; ++t)
+                    if (!(skip_first && t == 0) &&
+                        !mbar_wait(&sm.full[t % a.stages], static_cast<uint32_t>(t / a.stages) & 1u, a.wait_budget))
                         record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else if (warp == 1) {
@@ -774,37 +770,27 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 const uint64_t bd0 = make_sdesc(smem_u32(qtile), 16, kSbo, kLayout);
                 int s = 0, b = 0;
                 uint32_t ph = 0, aph = 0;
-                bool failed = false;
-                for (int u = 0; u < nst && !failed; ++u) {
-                    const int nsub = min(kStageTiles, ntiles - kStageTiles * u);
-                    for (int sub = 0; sub < nsub; ++sub) {
-                        if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
-                            (sub == 0 && !mbar_wait(&sm.full[s], ph, a.wait_budget)) || sm.abort) {
-                            failed = true;
-                            break;
-                        }
-                        tc_fence_after();
-                        const uint64_t ad =
-                            ad0 + static_cast<uint64_t>((s * kStageBytes + sub * kTileBytes) >> 4);
-#pragma unroll
-                        for (int kk = 0; kk < DI / 32; ++kk)
-                            mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
-                        // release the ring slot first (its refill paces the
-                        // stream), then hand the accumulator over
-                        if (sub == nsub - 1) tc_commit(&sm.empty[s]);
-                        tc_commit(&sm.acc_full[b]);
-                        if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
+                for (int t = 0; t < ntiles; ++t) {
+                    if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
+                        !mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
+                        record_status(a.status, DSA_ERR_TIMEOUT);
+                        sm.abort = 1;
+                        // the MMAs already issued complete before TMEM is
+                        // freed (on success the epilogue waits for each)
+                        tc_commit(&sm.mma_done);
+                        if (!mbar_wait(&sm.mma_done, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
+                        break;
                     }
-                    if (failed) break;
+                    tc_fence_after();
+                    const uint64_t ad = ad0 + static_cast<uint64_t>(s * (kTileBytes >> 4));
+#pragma unroll
+                    for (int kk = 0; kk < DI / 32; ++kk)
+                        mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
+                    tc_commit(&sm.empty[s]);
+                    tc_commit(&sm.acc_full[b]);
                     if (++s == a.stages) { s = 0; ph ^= 1; }
+                    if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
                 }
-                if (failed) {
-                    record_status(a.status, DSA_ERR_TIMEOUT);
-                    sm.abort = 1;
-                }
-                // every MMA issued must complete before TMEM is freed
-                tc_commit(&sm.mma_done);
-                if (!mbar_wait(&sm.mma_done, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
             }
         } else {
             // epilogue: group 0 = warps 2..5 takes even tiles (buffer 0),

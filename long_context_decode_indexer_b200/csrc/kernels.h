@@ -21,17 +21,12 @@ constexpr int kModeFused = 0;   // scores stay on chip, TopK indices written
 constexpr int kModeScores = 1;  // scores written to HBM
 constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 
-// Indexer stream tuning: 128-row tiles per TMA ring stage (one box of
-// 128 * DSA_K1_STAGE_TILES rows), ring depth, and whether the SMs a batch of
-// equal chunk counts leaves idle give some groups one more chunk.
-#ifndef DSA_K1_STAGE_TILES
-#define DSA_K1_STAGE_TILES 1
-#endif
+// Indexer stream tuning: whether the SMs a batch of equal chunk counts
+// leaves idle give some groups one more chunk (parallel selection only).
 #ifndef DSA_K1_FILL_SMS
 #define DSA_K1_FILL_SMS 1
 #endif
 constexpr int kK1MaxStages = 12;     // TMA ring barriers
-constexpr int kK1WantStages = kK1MaxStages / DSA_K1_STAGE_TILES;  // ring depth used when shared memory allows
 constexpr int kK1MaxAcc = 4;         // TMEM accumulator buffers (even: one parity per epilogue group)
 constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
 constexpr int kK2Threads = 256;
@@ -106,7 +101,7 @@ __host__ __device__ inline K1Layout k1_layout(int mode, int di, int qg, int hp, 
     K1Layout L;
     uint32_t off = 0;
     L.stages = off;
-    if (mode != kModeTopk) off += static_cast<uint32_t>(stages) * 128u * DSA_K1_STAGE_TILES * static_cast<uint32_t>(di);
+    if (mode != kModeTopk) off += static_cast<uint32_t>(stages) * 128u * static_cast<uint32_t>(di);
     L.qtile = off;
     if (mode != kModeTopk) off += align_up(static_cast<uint32_t>(qg * hp * di), 1024);
     L.keys = off;
@@ -234,7 +229,7 @@ cudaError_t launch_kl_reduce(const MlaParams &a, cudaStream_t st);
 // Dense multi-head attention of 128-query tiles over 128-key tiles, the
 // index set applied as a membership mask.  One CTA per (query tile, head).
 constexpr int kMhaTile = 128;      // queries per CTA (MMA M) and keys per tile (MMA N)
-constexpr int kMhaThreads = 192;   // warp 0 TMA, warp 1 MMA, warps 2-5 softmax + epilogue
+constexpr int kMhaThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-9 softmax + epilogue (two per row)
 constexpr int kMhaMaxStages = 3;   // K ring depth limit (the V ring has 2 slots)
 constexpr int kMhaVStages = 2;
 
@@ -271,7 +266,7 @@ __host__ __device__ inline MhaLayout mha_layout(int d_qk, int d_v, int stages) {
     L.k_ring = L.k_stage;
     L.v_ring = L.k_ring + static_cast<uint32_t>(stages) * L.k_stage;
     L.misc = L.v_ring + kMhaVStages * L.v_stage;
-    L.total = L.misc + 1024 + 1024;  // barriers, alignment slack
+    L.total = L.misc + 4096 + 1024;  // barriers and the softmax exchange, alignment slack
     return L;
 }
 

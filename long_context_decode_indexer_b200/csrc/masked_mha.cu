@@ -14,7 +14,8 @@
 // that the CTAs running together share their K / V in L2.  Warp 0 streams Q
 // once and K / V tiles of 128 positions through a TMA ring (3-D tensor maps
 // over [row, head, dim], 128B swizzle); warp 1 issues the tcgen05 MMAs;
-// warps 2-5 (one thread per query row = TMEM lane) run the softmax.
+// warps 2-9 run the softmax, two warps per query row (= TMEM lane), each on
+// half of a tile's keys.
 //   S(j) = Q . K(j)^T      M = 128 queries, N = 128 keys, K = d_qk; two TMEM
 //                           buffers, so S(j+1) is computed during softmax(j)
 //   P(j) = 2^(S' - m)      S' = S * scale * log2(e), masked keys -inf; P goes
@@ -61,14 +62,33 @@ struct MhaSmem {
     uint32_t tmem_base;
     volatile int32_t abort;
     int32_t n_max;
+    float half_max[2][2][kMhaTile];  // [tile parity][column half][row]
+    float half_sum[2][kMhaTile];     // [column half][row]
 };
-static_assert(sizeof(MhaSmem) <= 1024, "MhaSmem must fit the reserve in mha_layout()");
+static_assert(sizeof(MhaSmem) <= 4096, "MhaSmem must fit the reserve in mha_layout()");
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
 __device__ __forceinline__ uint32_t bf16x2_bits(__nv_bfloat162 v) { return *reinterpret_cast<uint32_t *>(&v); }
+
+// Named barrier `id` over `count` threads.
+__device__ __forceinline__ void bar_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier `id` over `count` threads that also ANDs `pred` across them.
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
 
 }  // namespace
 
@@ -105,9 +125,9 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_free[b], 4);  // the four softmax warps
+            mbar_init(&sm.s_free[b], 8);  // the eight softmax warps
         }
-        mbar_init(&sm.p_full, 4);
+        mbar_init(&sm.p_full, 8);
         mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.mma_done, 1);
         fence_mbar_init();
@@ -242,46 +262,60 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             if (!mbar_wait(&sm.mma_done, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
         }
     } else {
-        // ------------------------------------- softmax (thread = query row)
-        const int qr = warp & 3;  // this warp's quarter of the TMEM lanes
+        // ------------------------------------- softmax: two warps per row
+        // A row (query) is TMEM lane r; warps w and w + 4 share the lane
+        // quarter w % 4 and take the key columns [0, 64) and [64, 128) of
+        // each tile (and halves of O's columns), exchanging their half-row
+        // maxima (and, at the end, row sums) through shared memory under a
+        // named barrier of the pair.
+        const int qr = warp & 3;              // this warp's quarter of the TMEM lanes
+        const int hf = (warp - 2) >> 2;       // which half of the columns
+        const int bar_id = 1 + ((warp - 2) & 3);
         const int r = qr * 32 + lane;
         const int t = t0 + r;
         const bool valid = r < nrows;
         const int n_t = valid ? min(a.q_n[t], a.max_n) : 0;
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(qr * 32) << 16);
         const uint32_t *mrow = (a.mask != nullptr && valid) ? a.mask + static_cast<int64_t>(t) * a.mask_words : nullptr;
-        float m_used = -INFINITY, l = 0.f;
+        const int oc0 = hf * (a.d_v / 2), oc1 = oc0 + a.d_v / 2;  // this warp's O columns
+        float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
         bool ok = true;
         for (int j = 0; j < nkt; ++j) {
             const int b = j & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], static_cast<uint32_t>(j >> 1) & 1u, a.wait_budget) &&
                                              !sm.abort);
+            ok = bar_and(bar_id, 64, ok);
             if (!ok) break;
             tc_fence_after();
-            uint32_t u[128];
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                tmem_ld32(lane_addr + kColS + b * 128 + c * 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32 * c));
+            uint32_t u[64];
+            tmem_ld32(lane_addr + kColS + b * 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
+            tmem_ld32(lane_addr + kColS + b * 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.s_free[b]);
-            // keys j*128 + c kept: below n_t and in the index set
-            uint32_t mw[4];
+            // keys j*128 + hf*64 + c kept: below n_t and in the index set
+            uint32_t mw[2];
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const int s0 = j * kMhaTile + w * 32;
+            for (int w = 0; w < 2; ++w) {
+                const int s0 = j * kMhaTile + hf * 64 + w * 32;
                 uint32_t bits = s0 >= n_t ? 0u : (n_t - s0 >= 32 ? 0xffffffffu : ((1u << (n_t - s0)) - 1u));
-                if (mrow != nullptr && bits != 0u) bits &= mrow[j * 4 + w];
+                if (mrow != nullptr && bits != 0u) bits &= mrow[j * 4 + hf * 2 + w];
                 mw[w] = bits;
             }
-            float x[128];
-            float mt = -INFINITY;
+            float x[64];
+            float mh = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 128; ++c) {
+            for (int c = 0; c < 64; ++c) {
                 x[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? __uint_as_float(u[c]) * a.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, x[c]);
+                mh = fmaxf(mh, x[c]);
             }
+            // the tile's row max from both halves (double-buffered slots: the
+            // partner reads slot b of tile j before either writes it again at
+            // tile j + 2, two barriers later)
+            sm.half_max[b][hf][r] = mh;
+            bar_sync(bar_id, 64);
+            const float mt = fmaxf(sm.half_max[b][0][r], sm.half_max[b][1][r]);
             float alpha = 1.f;
             bool rescale = false;  // O holds earlier tiles' products to scale by alpha
             if (mt > m_used + kRaiseLog2) {
@@ -294,12 +328,13 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             if (j > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, static_cast<uint32_t>(j - 1) & 1u, a.wait_budget) &&
                                                  !sm.abort);
+                ok = bar_and(bar_id, 64, ok);  // both warps of the pair leave together
                 if (!ok) break;
                 tc_fence_after();
             }
             if (__any_sync(0xffffffffu, rescale)) {
                 const float f = rescale ? alpha : 1.f;
-                for (int c = 0; c < a.d_v; c += 32) {
+                for (int c = oc0; c < oc1; c += 32) {
                     uint32_t o[32];
                     tmem_ld32(lane_addr + kColO + c, o);
                     tmem_wait_ld();
@@ -310,7 +345,7 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             }
             float lsum = 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
                 uint32_t hi[16], lo[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -319,12 +354,12 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
                     const float p1 = x1 == -INFINITY ? 0.f : fast_exp2(x1 - m_used);
                     lsum += p0 + p1;
                     const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                    const float2 hf = __bfloat1622float2(h2);
+                    const float2 hfl = __bfloat1622float2(h2);
                     hi[e] = bf16x2_bits(h2);
-                    lo[e] = bf16x2_bits(__floats2bfloat162_rn(p0 - hf.x, p1 - hf.y));
+                    lo[e] = bf16x2_bits(__floats2bfloat162_rn(p0 - hfl.x, p1 - hfl.y));
                 }
-                tmem_st16(lane_addr + kColPhi + c0 / 2, hi);
-                tmem_st16(lane_addr + kColPlo + c0 / 2, lo);
+                tmem_st16(lane_addr + kColPhi + hf * 32 + c0 / 2, hi);
+                tmem_st16(lane_addr + kColPlo + hf * 32 + c0 / 2, lo);
             }
             l += lsum;
             tmem_wait_st();
@@ -332,15 +367,18 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&sm.p_full);
         }
-        // epilogue: O / l as bf16, and the log-sum-exp (natural log)
+        // epilogue: O / l as bf16 (this warp's columns), and the log-sum-exp
         if (ok && nkt > 0)
             ok = __all_sync(0xffffffffu,
                             mbar_wait(&sm.pv_done, static_cast<uint32_t>(nkt - 1) & 1u, a.wait_budget) && !sm.abort);
+        sm.half_sum[hf][r] = l;
+        ok = bar_and(bar_id, 64, ok);
         if (ok) {
             tc_fence_after();
-            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            const float lrow = sm.half_sum[0][r] + sm.half_sum[1][r];
+            const float inv_l = lrow > 0.f ? 1.f / lrow : 0.f;
             uint16_t *dst = a.out + (static_cast<int64_t>(t) * a.h + head) * a.d_v;
-            for (int c = 0; c < a.d_v; c += 32) {
+            for (int c = oc0; c < oc1; c += 32) {
                 uint32_t o[32];
                 if (nkt > 0) {
                     tmem_ld32(lane_addr + kColO + c, o);
@@ -360,9 +398,9 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
                     for (int g = 0; g < 4; ++g) d4[g] = make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
                 }
             }
-            if (valid)
+            if (valid && hf == 0)
                 a.lse[static_cast<int64_t>(t) * a.h + head] =
-                    l > 0.f ? (m_used + log2f(l)) * 0.6931471805599453f : -INFINITY;
+                    lrow > 0.f ? (m_used + log2f(lrow)) * 0.6931471805599453f : -INFINITY;
         } else if (lane == 0) {
             record_status(a.status, DSA_ERR_TIMEOUT);
         }
