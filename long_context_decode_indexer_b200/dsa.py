@@ -98,7 +98,7 @@ def lib() -> ctypes.CDLL:
             L.dsa_indexer_topk_static.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, _P]
             jp = ctypes.POINTER(ProjectParams)
             L.dsa_project_workspace_size.argtypes = [jp, ctypes.POINTER(ctypes.c_size_t)]
-            L.dsa_indexer_project.argtypes = [jp, kp] + [_P] * 16 + [ctypes.c_size_t, _P]
+            L.dsa_indexer_project.argtypes = [jp, kp] + [_P] * 17 + [ctypes.c_size_t, _P]
             L.dsa_index_kl.argtypes = [pp, kp, _P, _P, ctypes.c_int64, _P, ctypes.c_int64, _P, _P, _P,
                                        _P, ctypes.c_size_t, _P]
             L.dsa_masked_mha_prefill.argtypes = [pp, kp, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]

@@ -34,6 +34,19 @@ def test_library_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_bindings_pass_every_declared_parameter(L):
+    """Each ctypes binding types as many arguments as its C declaration has
+    parameters: an argument past the typed ones would go through as a
+    32-bit int (the stream handle of the producer once did)."""
+    text = open(os.path.join(ROOT, "include", "dsa.h")).read()
+    decls = dict(re.findall(r"\n(?:int|const char \*)\s*(dsa_\w+)\(([^;]*?)\);", text, re.S))
+    assert set(decls) == set(dsa.ENTRY_POINTS)
+    for name, params in decls.items():
+        n = 0 if params.strip() in ("", "void") else params.count(",") + 1
+        types = getattr(L, name).argtypes
+        assert len(types or []) == n, "%s: %d parameters, %d argtypes" % (name, n, len(types or []))
+
+
 def _params(cfg=3, **kw):
     c = CONFIGS[cfg]
     base = dict(nq=c["nseq"], h_idx=c["h_idx"], d_idx=c["d_idx"], h=c["h"], topk=c["topk"],
