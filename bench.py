@@ -4,8 +4,9 @@ MLA attention over a 16 x 128K-context batch (one query per sequence).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--ragged] [--nseq S] [--L CTX]
-                    [--no-cpu-baseline] [--no-e2e] [--clocks-csv PATH]
+                    [--no-cpu-baseline] [--no-e2e] [--no-next-rows] [--clocks-csv PATH]
     python bench.py --profile [--workload NAME] [--nseq S] [--L CTX] [--warmup W] [--steps K]
+    python bench.py --profile-next ROW [--nseq S] [--L CTX] [--warmup W] [--steps K]
 
 Workloads: long_decode_16x128k (default: the headline), batched_decode_64x32k,
 paged_mtp_decode_128seq, causal_prefill_16k, tiny_decode_4k; --ragged draws
@@ -29,14 +30,21 @@ fused indexer), timed alone over the same workload; `stages` gives each
 stage's time and its fraction of the binding roofline; `e2e` repeats the step
 through the C ABI from pinned host buffers (query-side inputs in, outputs
 out; the caches are resident state); `cpu_baseline` is the fp64 oracle timed
-on a bounded sample on this host, on all cores and on one.
+on a bounded sample on this host, on all cores and on one.  `next_rows` (one
+GPU, decode workloads) times the rows after the decode path alone: the
+indexer's q/k/w producer for the batch's tokens, attention over an FP8
+latent cache, the distillation loss (sparse and dense stage) and the
+masked-MHA short prefill of 4096 tokens, each with its algorithmic bytes and
+FLOPs as fractions of the measured peaks.
 
 --profile runs warm-up + K forward steps with no timing and checks the
-device status: the command the ncu captures run.
+device status: the command the ncu captures run; --profile-next does the same
+for one of the next rows (after W forward steps that produce its indices).
 """
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import os
 import statistics
@@ -52,7 +60,8 @@ sys.path.insert(0, ROOT)
 
 from long_context_decode_indexer_b200 import dsa  # noqa: E402
 from long_context_decode_indexer_b200.batch import upload, workspace  # noqa: E402
-from long_context_decode_indexer_b200.synth import CONFIGS, make_inputs  # noqa: E402
+from long_context_decode_indexer_b200.synth import (CONFIGS, make_inputs, make_mha_inputs,  # noqa: E402
+                                                     make_project_inputs)
 
 METRIC = "DSA decode queries/s at 128K ctx (indexer+TopK+sparse MLA); % of HBM/TC roofline"
 WORKLOADS = {c["name"]: cid for cid, c in CONFIGS.items()}
@@ -354,6 +363,16 @@ def run_ours(args, world, rank):
         torch.cuda.synchronize()
         return sum(a.elapsed_time(b) for a, b in evs) / 1e3
 
+    if args.profile_next:
+        for _ in range(max(args.warmup, 1)):  # the indices the next rows read
+            step()
+        runs = {r[0]: r for r in next_row_runners(inp, db, p, kv, idx, st)}
+        name, fn, _, _, _, wss = runs[args.profile_next]
+        for _ in range(args.warmup + args.steps):
+            fn()
+        status = max((dsa.check_status(w_) for w_ in wss), key=abs)
+        print(json.dumps({"profile": name, "steps": args.warmup + args.steps, "device_status": status}))
+        return None, inp
     if args.profile:
         for _ in range(args.warmup + args.steps):
             step()
@@ -363,9 +382,11 @@ def run_ours(args, world, rank):
                           "device_status": status}))
         return None, inp
 
+    phase("warm-up")
     for _ in range(args.warmup):
         step()
     assert dsa.check_status(ws) == dsa.DSA_OK, dsa.last_error()
+    phase("timed steps")
     launches_per_step = count_our_launches(step)
     barrier(world)
     torch.cuda.synchronize()
@@ -384,7 +405,13 @@ def run_ours(args, world, rank):
     status = dsa.check_status(ws)
     t_max = max_over_ranks(t_total, world)
 
+    next_rows = None
+    phase("next rows")
+    if not args.no_next_rows and world == 1 and not prefill and not paged:
+        next_rows = measure_next_rows(next_row_runners(inp, db, p, kv, idx, st), timed, evict, *peaks()[:2])
+
     e2e = None
+    phase("end to end")
     if not args.no_e2e:
         e2e = run_e2e(args, world, inp, db, p, idx, out, lse, ws_idx, ws_mla, mla_fn, timed)
     for w_ in (ws, ws_idx, ws_mla):
@@ -465,11 +492,126 @@ def run_ours(args, world, rank):
         "input_gen_s": gen_s,
         "clocks": clk.summary(),
     }
+    if next_rows is not None:
+        res["next_rows"] = next_rows
     if e2e is not None:
         e2e["value"] = total_q / e2e.pop("t")
         e2e["eager_value"] = total_q / e2e.pop("t_eager")
         res["e2e"] = e2e
     return res, inp
+
+
+def next_row_runners(inp, db, p, kv, idx, st):
+    """The rows after the decode path, on this batch or (masked MHA) the
+    short-prefill shape: a list of (name, run, algorithmic bytes, FLOPs,
+    extra keys, workspaces).  The indexer's q/k/w producer for this batch's
+    tokens; attention over an FP8 latent cache (this batch's selected rows,
+    the cache cast to e4m3 on the device with unit row scales); the
+    distillation loss, sparse stage over the selected sets and dense stage
+    over every visible position; the masked-MHA short prefill of 4096 tokens
+    (128 heads, 192 / 128 wide) under the indexer's TopK."""
+    runs = []
+    d = lambda a, dt=None: (torch.from_numpy(np.ascontiguousarray(a)).view(dt) if dt is not None
+                            else torch.from_numpy(np.ascontiguousarray(a))).cuda()
+    # f1: the producer for nq tokens (decode: one token per query)
+    phase("set up the next rows")
+    nt = inp.nq
+    pi = make_project_inputs(np.arange(nt, dtype=np.int32), np.arange(nt, dtype=np.int32))
+    pp = dsa.make_project_params(nt=nt, hidden=pi.x.shape[1], q_lora_rank=pi.q_lora.shape[1],
+                                 h_idx=pi.h_idx, d_idx=pi.d_idx, rope_dim=pi.rope_dim)
+    pkeep = [d(pi.q_seq), d(np.zeros(nt, np.int64))]  # referenced as long as the runner lives
+    pkv = dsa.make_kv(q_seq=pkeep[0], q_n=None, seq_row0=pkeep[1], cache_rows=nt)
+    pws = workspace(dsa.project_workspace_size(pp))
+    H, dI = pi.h_idx, pi.d_idx
+    pargs = [d(pi.x, torch.int16), d(pi.q_lora, torch.int16), d(pi.w_qb, torch.int16),
+             d(pi.w_k, torch.int16), d(pi.w_proj, torch.int16), d(pi.ln_gamma), d(pi.ln_beta),
+             d(pi.positions), torch.empty((nt, H, dI), dtype=torch.uint8, device="cuda"),
+             torch.empty((nt, H), dtype=torch.float32, device="cuda"),
+             torch.empty((nt, H), dtype=torch.int16, device="cuda"),
+             torch.empty((nt, dI), dtype=torch.uint8, device="cuda"),
+             torch.empty((nt,), dtype=torch.float32, device="cuda")]
+    wsz = pi.w_qb.size + pi.w_k.size + pi.w_proj.size
+    runs.append(("f1_indexer_project",
+                 lambda: dsa.indexer_project(pp, pkv, *pargs, pws, stream=st),
+                 2 * wsz + 2 * (pi.x.size + pi.q_lora.size), 2 * nt * wsz,
+                 {"tokens": nt, "bound": "hbm", "_keep": (pkeep, pargs)}, [pws]))
+
+    # f4: attention over an FP8 latent cache (the same selected rows)
+    kv8 = db.kv.view(torch.bfloat16).to(torch.float8_e4m3fn).view(torch.uint8)
+    ksc = torch.ones(kv8.shape[0], dtype=torch.float32, device="cuda")
+    ws8 = workspace(dsa.workspace_size(p, kv, dsa.OP_SPARSE_MLA_DECODE))
+    out = torch.empty((inp.nq, inp.h, inp.d_v), dtype=torch.int16, device="cuda")
+    lse = torch.empty((inp.nq, inp.h), dtype=torch.float32, device="cuda")
+    sel = np.minimum(inp.q_n.astype(np.int64), inp.topk)
+    rows = int(sel.sum())
+    att_io = inp.nq * inp.h * (inp.d_qk * 2 + inp.d_v * 2 + 4) + inp.nq * inp.topk * 4
+    runs.append(("f4_sparse_mla_fp8",
+                 lambda: dsa.sparse_mla_decode_fp8(p, kv, db.q, kv8, kv8.stride(0), ksc, idx, out, lse, ws8,
+                                                   stream=st),
+                 rows * (inp.d_qk + 4) + att_io, 2 * rows * inp.h * (inp.d_qk + inp.d_v),
+                 {"rows": rows, "_keep": (kv8, ksc, out, lse)}, [ws8]))
+
+    # f3: distillation loss, sparse stage (the selected sets) and dense stage
+    ld = max(inp.max_n, 1)
+    scores = torch.zeros((inp.nq, ld), dtype=torch.float32, device="cuda")
+    wsc = workspace(dsa.workspace_size(p, kv, dsa.OP_INDEXER_SCORES))
+    dsa.indexer_scores(p, kv, db.q_idx, db.w, db.kidx, db.k_scale, scores, ld, wsc, stream=st)
+    kl = torch.empty((inp.nq,), dtype=torch.float32, device="cuda")
+    for name, ix, op in (("f3_index_kl_sparse", idx, dsa.OP_INDEX_KL_SPARSE),
+                         ("f3_index_kl_dense", None, dsa.OP_INDEX_KL_DENSE)):
+        wsk = workspace(dsa.workspace_size(p, kv, op))
+        r = rows if ix is not None else int(inp.q_n.astype(np.int64).sum())
+        # two passes of Q . K^T over the set; the rows read once from HBM
+        runs.append((name,
+                     (lambda ix=ix, wsk=wsk: dsa.index_kl(p, kv, db.q, db.kv, db.kv_row_stride, scores, ld, ix,
+                                                          kl, None, wsk, stream=st)),
+                     r * inp.d_qk * 2 + r * 4 + (inp.nq * ld * 4 if ix is None else 0),
+                     2 * 2 * r * inp.h * inp.d_qk, {"rows": r, "_keep": (scores, kl)}, [wsk, wsc]))
+
+    # f2: masked-MHA short prefill, 4096 tokens, the indexer's TopK as the mask
+    L = 4096
+    pin = make_inputs(4, L=L, with_attention=False)
+    pdb = upload(pin)
+    ipar, ikv = pdb.params(), pdb.kvdesc()
+    pidx = torch.empty((L, pin.topk), dtype=torch.int32, device="cuda")
+    wsi = workspace(dsa.workspace_size(ipar, ikv, dsa.OP_INDEXER_TOPK))
+    dsa.indexer_topk(ipar, ikv, pdb.q_idx, pdb.w, pdb.kidx, pdb.k_scale, pidx, None, wsi, stream=st)
+    m = make_mha_inputs(L)
+    mkeep = [d(m.q, torch.int16), d(m.k, torch.int16), d(m.v, torch.int16), d(m.q_seq), d(m.q_n),
+             d(m.seq_row0)]
+    hq, dq, dv = m.q.shape[1], m.q.shape[2], m.v.shape[2]
+    pm = dsa.make_params(nq=L, h_idx=1, d_idx=64, h=hq, topk=pin.topk, max_n=L, q_per_seq=L, scale=m.scale,
+                         d_qk=dq, d_v=dv)
+    kvm = dsa.make_kv(q_seq=mkeep[3], q_n=mkeep[4], seq_row0=mkeep[5], cache_rows=L)
+    wsm = workspace(dsa.workspace_size(pm, kvm, dsa.OP_MASKED_MHA))
+    mout = torch.empty((L, hq, dv), dtype=torch.int16, device="cuda")
+    mlse = torch.empty((L, hq), dtype=torch.float32, device="cuda")
+    runs.append(("f2_masked_mha_prefill_4k",
+                 lambda: dsa.masked_mha_prefill(pm, kvm, mkeep[0], mkeep[1], mkeep[2], pidx, mout, mlse, wsm,
+                                                stream=st),
+                 2 * L * hq * (2 * dq + 2 * dv),                            # q, k, v, out
+                 2 * hq * float(m.q_n.astype(np.int64).sum()) * (dq + dv),  # causal dense
+                 {"tokens": L, "bound": "tensor", "_keep": (mkeep, pdb, pidx, mout, mlse)}, [wsm, wsi]))
+    return runs
+
+
+def measure_next_rows(runs, timed, evict, hbm, bf16, iters=20):
+    """Each next row timed alone (CUDA events on the launching stream, L2
+    evicted before every run), with its algorithmic bytes and FLOPs as
+    fractions of the measured peaks."""
+    res = {}
+    for name, fn, bytes_, flops, extra, wss in runs:
+        phase(name)
+        fn()
+        t = timed(fn, iters, before=evict) / iters
+        for w_ in wss:
+            assert dsa.check_status(w_) == dsa.DSA_OK, dsa.last_error()
+        r = {"us": t * 1e6, "gbs": bytes_ / t / 1e9, "tflops": flops / t / 1e12,
+             "frac_hbm": bytes_ / t / 1e9 / hbm, "frac_bf16": flops / t / 1e12 / bf16,
+             "algorithmic_bytes": bytes_, "flops": flops}
+        r.update({k: v for k, v in extra.items() if not k.startswith("_")})
+        res[name] = r
+    return res
 
 
 def run_e2e(args, world, inp, db, p, idx, out, lse, ws_idx, ws_mla, mla_fn, timed):
@@ -650,17 +792,30 @@ def parse_args(argv=None):
     ap.add_argument("--L", type=int, default=None, help="resize: context length (median for paged)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the next rows' timings (producer, FP8 attention, distillation loss, masked MHA)")
     ap.add_argument("--profile", action="store_true",
                     help="run warm-up + steps forward calls untimed (for profiler captures)")
+    ap.add_argument("--profile-next", default=None,
+                    choices=["f1_indexer_project", "f2_masked_mha_prefill_4k", "f3_index_kl_sparse",
+                             "f3_index_kl_dense", "f4_sparse_mla_fp8"],
+                    help="run warm-up forward steps, then warm-up + steps calls of one next row untimed")
     ap.add_argument("--clocks-csv", default=None,
                     help="also record nvidia-smi clock samples (CSV) during the timed loops")
     args = ap.parse_args(argv)
-    if not args.profile:
+    if not args.profile and not args.profile_next:
         args.warmup = max(args.warmup, 3)
     return args
 
 
+def phase(name: str):
+    """A progress line on stderr (where a crash happened, with faulthandler's
+    traceback)."""
+    print("bench: %s" % name, file=sys.stderr, flush=True)
+
+
 def main():
+    faulthandler.enable()
     args = parse_args()
     world, rank, _ = dist_init() if args.impl == "ours" else (
         int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
@@ -672,6 +827,7 @@ def main():
     res, inp = run_ours(args, world, rank)
     if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
+            phase("cpu baseline")
             res["cpu_baseline"] = cpu_baseline(inp)
         print(json.dumps(res))
     if world > 1:
