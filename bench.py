@@ -78,7 +78,7 @@ K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
               "long_context_decode_indexer_b200/csrc/select.cuh",
               "long_context_decode_indexer_b200/csrc/ptx.cuh",
               "long_context_decode_indexer_b200/csrc/kernels.h")
-K1_PROFILED = {"sha256_16": "8a4b7d790e67b55e", "bytes_per_position": 131.10498046875}
+K1_PROFILED = {"sha256_16": "c0b39042a1523559", "bytes_per_position": 132.142333984375}
 
 
 def k1_sources_hash() -> str:
@@ -532,7 +532,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
              torch.empty((nt,), dtype=torch.float32, device="cuda")]
     wsz = pi.w_qb.size + pi.w_k.size + pi.w_proj.size
     runs.append(("f1_indexer_project",
-                 lambda: dsa.indexer_project(pp, pkv, *pargs, pws, stream=st),
+                 lambda: dsa.indexer_project(pp, pkv, *pargs, pws),
                  2 * wsz + 2 * (pi.x.size + pi.q_lora.size), 2 * nt * wsz,
                  {"tokens": nt, "bound": "hbm", "_keep": (pkeep, pargs)}, [pws]))
 
@@ -546,8 +546,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
     rows = int(sel.sum())
     att_io = inp.nq * inp.h * (inp.d_qk * 2 + inp.d_v * 2 + 4) + inp.nq * inp.topk * 4
     runs.append(("f4_sparse_mla_fp8",
-                 lambda: dsa.sparse_mla_decode_fp8(p, kv, db.q, kv8, kv8.stride(0), ksc, idx, out, lse, ws8,
-                                                   stream=st),
+                 lambda: dsa.sparse_mla_decode_fp8(p, kv, db.q, kv8, kv8.stride(0), ksc, idx, out, lse, ws8),
                  rows * (inp.d_qk + 4) + att_io, 2 * rows * inp.h * (inp.d_qk + inp.d_v),
                  {"rows": rows, "_keep": (kv8, ksc, out, lse)}, [ws8]))
 
@@ -555,7 +554,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
     ld = max(inp.max_n, 1)
     scores = torch.zeros((inp.nq, ld), dtype=torch.float32, device="cuda")
     wsc = workspace(dsa.workspace_size(p, kv, dsa.OP_INDEXER_SCORES))
-    dsa.indexer_scores(p, kv, db.q_idx, db.w, db.kidx, db.k_scale, scores, ld, wsc, stream=st)
+    dsa.indexer_scores(p, kv, db.q_idx, db.w, db.kidx, db.k_scale, scores, ld, wsc)
     kl = torch.empty((inp.nq,), dtype=torch.float32, device="cuda")
     for name, ix, op in (("f3_index_kl_sparse", idx, dsa.OP_INDEX_KL_SPARSE),
                          ("f3_index_kl_dense", None, dsa.OP_INDEX_KL_DENSE)):
@@ -564,7 +563,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
         # two passes of Q . K^T over the set; the rows read once from HBM
         runs.append((name,
                      (lambda ix=ix, wsk=wsk: dsa.index_kl(p, kv, db.q, db.kv, db.kv_row_stride, scores, ld, ix,
-                                                          kl, None, wsk, stream=st)),
+                                                          kl, None, wsk)),
                      r * inp.d_qk * 2 + r * 4 + (inp.nq * ld * 4 if ix is None else 0),
                      2 * 2 * r * inp.h * inp.d_qk, {"rows": r, "_keep": (scores, kl)}, [wsk, wsc]))
 
@@ -575,7 +574,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
     ipar, ikv = pdb.params(), pdb.kvdesc()
     pidx = torch.empty((L, pin.topk), dtype=torch.int32, device="cuda")
     wsi = workspace(dsa.workspace_size(ipar, ikv, dsa.OP_INDEXER_TOPK))
-    dsa.indexer_topk(ipar, ikv, pdb.q_idx, pdb.w, pdb.kidx, pdb.k_scale, pidx, None, wsi, stream=st)
+    dsa.indexer_topk(ipar, ikv, pdb.q_idx, pdb.w, pdb.kidx, pdb.k_scale, pidx, None, wsi)
     m = make_mha_inputs(L)
     mkeep = [d(m.q, torch.int16), d(m.k, torch.int16), d(m.v, torch.int16), d(m.q_seq), d(m.q_n),
              d(m.seq_row0)]
@@ -587,8 +586,7 @@ def next_row_runners(inp, db, p, kv, idx, st):
     mout = torch.empty((L, hq, dv), dtype=torch.int16, device="cuda")
     mlse = torch.empty((L, hq), dtype=torch.float32, device="cuda")
     runs.append(("f2_masked_mha_prefill_4k",
-                 lambda: dsa.masked_mha_prefill(pm, kvm, mkeep[0], mkeep[1], mkeep[2], pidx, mout, mlse, wsm,
-                                                stream=st),
+                 lambda: dsa.masked_mha_prefill(pm, kvm, mkeep[0], mkeep[1], mkeep[2], pidx, mout, mlse, wsm),
                  2 * L * hq * (2 * dq + 2 * dv),                            # q, k, v, out
                  2 * hq * float(m.q_n.astype(np.int64).sum()) * (dq + dv),  # causal dense
                  {"tokens": L, "bound": "tensor", "_keep": (mkeep, pdb, pidx, mout, mlse)}, [wsm, wsi]))
@@ -596,17 +594,42 @@ def next_row_runners(inp, db, p, kv, idx, st):
 
 
 def measure_next_rows(runs, timed, evict, hbm, bf16, iters=20):
-    """Each next row timed alone (CUDA events on the launching stream, L2
-    evicted before every run), with its algorithmic bytes and FLOPs as
-    fractions of the measured peaks."""
+    """Each next row timed alone, L2 evicted before every run: replayed as a
+    CUDA graph (device time: the library's host-side set-up, e.g. tensor-map
+    encoding, runs once at capture) and as eager calls (device time plus
+    whatever host time the calls leave the GPU idle).  The algorithmic bytes
+    and FLOPs are given as fractions of the measured peaks at the graph
+    time."""
     res = {}
     for name, fn, bytes_, flops, extra, wss in runs:
         phase(name)
         fn()
-        t = timed(fn, iters, before=evict) / iters
+        t_eager = timed(fn, iters, before=evict) / iters
         for w_ in wss:
             assert dsa.check_status(w_) == dsa.DSA_OK, dsa.last_error()
-        r = {"us": t * 1e6, "gbs": bytes_ / t / 1e9, "tflops": flops / t / 1e12,
+        t, launch = t_eager, "eager"
+        try:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                fn()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g):
+                fn()
+            g.replay()
+            torch.cuda.synchronize()
+            t = timed(g.replay, iters, before=evict) / iters
+            launch = "cuda_graph"
+            del g
+        except RuntimeError as exc:
+            print("next row %s: graph capture failed (%s); eager time reported" % (name, exc),
+                  file=sys.stderr)
+        for w_ in wss:
+            assert dsa.check_status(w_) == dsa.DSA_OK, dsa.last_error()
+        r = {"us": t * 1e6, "us_eager": t_eager * 1e6, "launch": launch,
+             "gbs": bytes_ / t / 1e9, "tflops": flops / t / 1e12,
              "frac_hbm": bytes_ / t / 1e9 / hbm, "frac_bf16": flops / t / 1e12 / bf16,
              "algorithmic_bytes": bytes_, "flops": flops}
         r.update({k: v for k, v in extra.items() if not k.startswith("_")})
