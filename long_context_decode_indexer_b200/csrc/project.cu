@@ -76,15 +76,19 @@ __device__ __forceinline__ uint32_t e4m3(float x) {
     return static_cast<uint32_t>(__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3));
 }
 
-// RoPE of the pair (v0, v1) at dims (2i, 2i+1): angle pos * theta^(-2i/rope_dim)
-// in double (positions reach 2^27; an fp32 angle would lose the fraction).
-__device__ __forceinline__ void rope_pair(float &v0, float &v1, int i, int rope_dim, int pos, float theta) {
+// The rotation of pair i (dims 2i, 2i+1) at position pos: angle
+// pos * theta^(-2i/rope_dim) in double (positions reach 2^27; an fp32 angle
+// would lose the fraction).  A token's pairs are the same for its k^I and
+// every q^I head, so each CTA computes them once (rope_table).
+__device__ __forceinline__ void rope_angle(int i, int rope_dim, int pos, float theta, double &s, double &c) {
     const double inv = pow(static_cast<double>(theta), -2.0 * static_cast<double>(i) / static_cast<double>(rope_dim));
-    double s, c;
     sincos(static_cast<double>(pos) * inv, &s, &c);
+}
+
+__device__ __forceinline__ void rope_pair(float &v0, float &v1, const double2 &sc) {
     const double x0 = v0, x1 = v1;
-    v0 = static_cast<float>(x0 * c - x1 * s);
-    v1 = static_cast<float>(x0 * s + x1 * c);
+    v0 = static_cast<float>(x0 * sc.y - x1 * sc.x);
+    v1 = static_cast<float>(x0 * sc.x + x1 * sc.y);
 }
 
 }  // namespace
@@ -234,10 +238,17 @@ __global__ void __launch_bounds__(192, 1)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
     __shared__ float wraw[64];
+    __shared__ double2 rope_table[64];  // (sin, cos) of each rotated pair at this token's position
     const int t = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int d = a.d_idx, H = a.h_idx, per = a.d_idx / 32;
     const int pos = a.positions[t];
+    for (int i = threadIdx.x; i < a.rope_dim / 2; i += blockDim.x) {
+        double sn, cs;
+        rope_angle(i, a.rope_dim, pos, a.rope_theta, sn, cs);
+        rope_table[i] = make_double2(sn, cs);
+    }
+    __syncthreads();
 
     if (warp == 0) {
         // ---- k^I: LayerNorm, RoPE, FP8 with a power-of-two scale, cache append
@@ -261,7 +272,7 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
         }
         for (int i = 0; i < per; i += 2) {
             const int o = lane * per + i;
-            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], o / 2, a.rope_dim, pos, a.rope_theta);
+            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], rope_table[o / 2]);
         }
         float amax = 0.f;
         for (int i = 0; i < per; ++i) amax = fmaxf(amax, fabsf(v[i]));
@@ -310,7 +321,7 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
         }
         for (int i = 0; i < per; i += 2) {
             const int o = lane * per + i;
-            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], o / 2, a.rope_dim, pos, a.rope_theta);
+            if (o < a.rope_dim) rope_pair(v[i], v[i + 1], rope_table[o / 2]);
         }
         float amax = 0.f;
         for (int i = 0; i < per; ++i) amax = fmaxf(amax, fabsf(v[i]));
