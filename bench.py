@@ -78,15 +78,22 @@ K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
               "long_context_decode_indexer_b200/csrc/select.cuh",
               "long_context_decode_indexer_b200/csrc/ptx.cuh",
               "long_context_decode_indexer_b200/csrc/kernels.h")
-K1_PROFILED = {"sha256_16": "c0b39042a1523559", "bytes_per_position": 132.142333984375}
+# kernels.h holds every kernel's parameters: only its indexer part (up to
+# this line) belongs to k1
+K1_HEADER_END = "// ------------------------------------------------------ sparse MLA attention"
+K1_PROFILED = {"sha256_16": "592551061317433e", "bytes_per_position": 132.142333984375}
 
 
 def k1_sources_hash() -> str:
+    """Hash of the indexer kernel's sources (the k1 part of kernels.h)."""
     import hashlib
     h = hashlib.sha256()
     for f in K1_SOURCES:
         with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+            data = fh.read()
+        if f.endswith("kernels.h"):
+            data = data[:data.index(K1_HEADER_END.encode())]
+        h.update(data)
     return h.hexdigest()[:16]
 
 

@@ -617,7 +617,8 @@ int check_mla_inputs(const dsa_params *p, const void *q, const void *kv_cache, i
 
 // ------------------------------------------------------- indexer producer
 struct ProjPlan {
-    int m_tiles, k_steps[2], n_cols[2], n_tiles[2], splits[2], ld[2];
+    int n_tok, t_tiles, m_tiles[2], k_steps[2], splits[2], ld[2], stages;
+    uint32_t stage_bytes;
     size_t part_off[2], total;
 };
 
@@ -639,26 +640,33 @@ int check_project(const dsa_project_params *pp) {
 // proportion to each problem's weight bytes (decode streams the weights).
 ProjPlan plan_project(const dsa_project_params *pp) {
     ProjPlan pl;
-    pl.m_tiles = (pp->nt + 127) / 128;
+    // token tiles of up to 256 (the MMA N), a multiple of 16
+    int nt16 = (pp->nt + 15) / 16 * 16;
+    pl.n_tok = nt16 < 16 ? 16 : (nt16 > 256 ? 256 : nt16);
+    pl.t_tiles = (pp->nt + pl.n_tok - 1) / pl.n_tok;
+    pl.m_tiles[0] = (pp->d_idx + pp->h_idx + 127) / 128;
+    pl.m_tiles[1] = (pp->h_idx * pp->d_idx + 127) / 128;
     pl.k_steps[0] = (pp->hidden + 63) / 64;
     pl.k_steps[1] = (pp->q_lora_rank + 63) / 64;
-    pl.n_cols[0] = (pp->d_idx + pp->h_idx + 15) / 16 * 16;
-    pl.n_cols[1] = 128;
-    pl.n_tiles[0] = 1;
-    pl.n_tiles[1] = (pp->h_idx * pp->d_idx + 127) / 128;
     pl.ld[0] = (pp->d_idx + pp->h_idx + 3) & ~3;
     pl.ld[1] = pp->h_idx * pp->d_idx;
+    // K slices fill the SMs in proportion to each problem's weight bytes
     const double b0 = static_cast<double>(pp->d_idx + pp->h_idx) * pp->hidden;
     const double b1 = static_cast<double>(pp->h_idx) * pp->d_idx * pp->q_lora_rank;
     const int sms = num_sms();
-    const int base0 = pl.m_tiles, base1 = pl.m_tiles * pl.n_tiles[1];
+    const int base0 = pl.m_tiles[0] * pl.t_tiles, base1 = pl.m_tiles[1] * pl.t_tiles;
     int s0 = 1, s1 = 1;
-    if (pl.m_tiles > 0 && base0 + base1 < sms) {
+    if (pl.t_tiles > 0 && base0 + base1 < sms) {
         s0 = static_cast<int>(sms * b0 / (b0 + b1) / base0);
         s1 = static_cast<int>(sms * b1 / (b0 + b1) / base1);
     }
     pl.splits[0] = s0 < 1 ? 1 : (s0 > pl.k_steps[0] ? pl.k_steps[0] : s0);
     pl.splits[1] = s1 < 1 ? 1 : (s1 > pl.k_steps[1] ? pl.k_steps[1] : s1);
+    // ring: 16 KB of weights + n_tok x 128 B of activations per stage
+    pl.stage_bytes = (16384u + static_cast<uint32_t>(pl.n_tok) * 128u + 1023u) & ~1023u;
+    int st = dsa::kProjMaxStages;
+    while (st > 2 && static_cast<size_t>(st) * pl.stage_bytes + 1024 + 1024 > 232448) --st;
+    pl.stages = st;
     size_t off = 256;  // status word
     for (int q = 0; q < 2; ++q) {
         pl.part_off[q] = off;
@@ -1000,9 +1008,12 @@ int dsa_indexer_project(const dsa_project_params *pp, const dsa_kv *kv, const vo
     CUtensorMap xm, qm, km, pm, wm;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    rc = make_map_2d(&xm, bf, x, pp->hidden, pp->nt, pp->hidden * 2ull, 64, 128, sw);
-    if (!rc) rc = make_map_2d(&qm, bf, q_lora, pp->q_lora_rank, pp->nt, pp->q_lora_rank * 2ull, 64, 128, sw);
-    if (!rc) rc = make_map_2d(&km, bf, w_k, pp->hidden, pp->d_idx, pp->hidden * 2ull, 64, pp->d_idx, sw);
+    // weights as 64-row (W_k, W_proj) / 128-row (W_qb) boxes, activations as
+    // boxes of one token tile
+    const uint32_t ntok = static_cast<uint32_t>(pl.n_tok);
+    rc = make_map_2d(&xm, bf, x, pp->hidden, pp->nt, pp->hidden * 2ull, 64, ntok, sw);
+    if (!rc) rc = make_map_2d(&qm, bf, q_lora, pp->q_lora_rank, pp->nt, pp->q_lora_rank * 2ull, 64, ntok, sw);
+    if (!rc) rc = make_map_2d(&km, bf, w_k, pp->hidden, pp->d_idx, pp->hidden * 2ull, 64, 64, sw);
     if (!rc) rc = make_map_2d(&pm, bf, w_proj, pp->hidden, pp->h_idx, pp->hidden * 2ull, 64, pp->h_idx, sw);
     if (!rc) rc = make_map_2d(&wm, bf, w_qb, pp->q_lora_rank, static_cast<uint64_t>(pp->h_idx) * pp->d_idx,
                               pp->q_lora_rank * 2ull, 64, 128, sw);
@@ -1010,16 +1021,18 @@ int dsa_indexer_project(const dsa_project_params *pp, const dsa_kv *kv, const vo
     dsa::ProjGemmParams g;
     memset(&g, 0, sizeof g);
     g.nt = pp->nt;
-    g.m_tiles = pl.m_tiles;
+    g.n_tok = pl.n_tok;
+    g.t_tiles = pl.t_tiles;
     for (int q = 0; q < 2; ++q) {
+        g.m_tiles[q] = pl.m_tiles[q];
         g.k_steps[q] = pl.k_steps[q];
-        g.n_cols[q] = pl.n_cols[q];
-        g.n_tiles[q] = pl.n_tiles[q];
         g.splits[q] = pl.splits[q];
         g.part[q] = at<float>(ws, pl.part_off[q]);
         g.ld[q] = pl.ld[q];
     }
-    g.items0 = pl.m_tiles * pl.n_tiles[0] * pl.splits[0];
+    g.items0 = pl.m_tiles[0] * pl.t_tiles * pl.splits[0];
+    g.stages = pl.stages;
+    g.stage_bytes = pl.stage_bytes;
     g.d_idx = pp->d_idx;
     g.h_idx = pp->h_idx;
     g.status = at<int>(ws, 0);

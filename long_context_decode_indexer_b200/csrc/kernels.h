@@ -276,19 +276,21 @@ cudaError_t launch_masked_mha(const CUtensorMap &qmap, const CUtensorMap &kmap, 
                               const MhaParams &a, int grid, cudaStream_t st);
 
 // ------------------------------------------------ indexer producer (q^I, k^I, w)
-constexpr int kProjStages = 4;  // TMA ring depth of the projection GEMM
+constexpr int kProjMaxStages = 12;  // TMA ring depth limit of the projection GEMM
 
 // Split-K GEMM of both projections: problem 0 = x . [W_k; W_proj]^T
 // (N = d_I + H_I), problem 1 = q_lora . W_qb^T (N tiles of 128 rows).
 struct ProjGemmParams {
     int32_t nt;              // tokens
-    int32_t m_tiles;         // 128-token tiles
+    int32_t n_tok;           // tokens per tile (MMA N, a multiple of 16, <= 256)
+    int32_t t_tiles;         // token tiles
+    int32_t m_tiles[2];      // 128-output tiles per problem (MMA M: weight rows)
     int32_t k_steps[2];      // 64-wide K steps per problem
-    int32_t n_cols[2];       // MMA N of a tile (a multiple of 16)
-    int32_t n_tiles[2];      // tiles along N (1 for problem 0)
     int32_t splits[2];       // K slices per problem
     int32_t items0;          // work items of problem 0 (they come first in the grid)
     int32_t d_idx, h_idx;
+    int32_t stages;          // TMA ring depth
+    uint32_t stage_bytes;    // one stage: 128 weight rows + n_tok token rows, 64 K each
     float *part[2];          // [splits, nt, ld] fp32 partial sums per K slice
     int32_t ld[2];           // row lengths of part
     int *status;

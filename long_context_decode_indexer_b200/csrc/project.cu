@@ -9,13 +9,14 @@
 // pos * theta^(-2i / rope_dim); the FP8 scales are powers of two (the e8m0
 // k_s of section 4.3; the same for q, so folding it into w is exact).
 //
-// k5_proj_gemm: both contractions in one launch, on the tensor cores.  A work
-// item is (problem, 128-token tile, N tile, K slice); a TMA ring feeds
-// tcgen05.mma kind::f16 (M = 128 tokens, N = d_I + H_I for the x problem, 128
-// for the q_lora problem, K = 64 per stage) into TMEM, and the epilogue warps
-// write the fp32 partial sums of the slice.  Few tokens (decode) leave most
-// SMs without a token tile, so K is split into slices until the grid fills
-// the SMs, in proportion to each problem's weight bytes.
+// k5_proj_gemm: both contractions in one launch, on the tensor cores, with
+// the weights as the MMA's M operand (128 output rows per tile) and the
+// tokens as N (16 to 256 per tile): at decode a tile then streams 16 KB of
+// weights and only N x 128 bytes of activations per 64-wide K step, so a
+// deep TMA ring keeps many weight bytes in flight.  A work item is
+// (problem, 128-output tile, token tile, K slice); K is split into slices
+// until the grid fills the SMs, in proportion to each problem's weight
+// bytes; the epilogue writes the slice's fp32 partial sums.
 // k6_proj_epilogue: one CTA per token sums the slices in a fixed order and
 // applies LayerNorm, RoPE, the quantisation, the weight folding and the
 // cache append.
@@ -33,15 +34,13 @@ namespace dsa {
 
 namespace {
 
-constexpr int kPBm = 128;                 // tokens per tile (MMA M)
+constexpr int kPBm = 128;                 // weight rows per tile (MMA M)
 constexpr int kPBk = 64;                  // K per stage (128 bytes of bf16: one swizzle span)
-constexpr int kPABytes = kPBm * kPBk * 2; // 16 KB
-constexpr int kPBMaxRows = 256;           // B rows per tile (MMA N <= 256)
-constexpr int kPStageBytes = kPABytes + kPBMaxRows * kPBk * 2;
+constexpr int kPABytes = kPBm * kPBk * 2; // 16 KB of weights per stage
 
 struct ProjSmem {
-    uint64_t full[kProjStages];
-    uint64_t empty[kProjStages];
+    uint64_t full[kProjMaxStages];
+    uint64_t empty[kProjMaxStages];
     uint64_t acc_full;
     uint32_t tmem_base;
     volatile int32_t abort;
@@ -94,8 +93,11 @@ __device__ __forceinline__ void rope_pair(float &v0, float &v1, const double2 &s
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// k5: split-K tcgen05 GEMM of both projections.  192 threads: warp 0 TMA,
-// warp 1 MMA, warps 2-5 epilogue (TMEM lane quarter = warp % 4).
+// k5: split-K tcgen05 GEMM of both projections, D[output, token].  192
+// threads: warp 0 TMA, warp 1 MMA, warps 2-5 epilogue (TMEM lane quarter =
+// warp % 4; a lane is an output row, a column a token).
+// Problem 0 stacks W_k (rows 0..d_I-1) and W_proj (rows d_I..d_I+H_I-1), in
+// 64-row pieces; problem 1 is W_qb.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(192, 1)
     k5_proj_gemm(const __grid_constant__ CUtensorMap x_map, const __grid_constant__ CUtensorMap ql_map,
@@ -103,26 +105,36 @@ __global__ void __launch_bounds__(192, 1)
                  const __grid_constant__ CUtensorMap wq_map, const ProjGemmParams a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    ProjSmem &sm = *reinterpret_cast<ProjSmem *>(base + kProjStages * kPStageBytes);
+    ProjSmem &sm = *reinterpret_cast<ProjSmem *>(base + static_cast<uint32_t>(a.stages) * a.stage_bytes);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int prob = static_cast<int>(blockIdx.x) < a.items0 ? 0 : 1;
     const int it = prob ? static_cast<int>(blockIdx.x) - a.items0 : static_cast<int>(blockIdx.x);
     const int split = it % a.splits[prob];
     const int rest = it / a.splits[prob];
-    const int n_tile = rest % a.n_tiles[prob];
-    const int m_tile = rest / a.n_tiles[prob];
+    const int t_tile = rest % a.t_tiles;
+    const int m_tile = rest / a.t_tiles;
     const int k_begin = static_cast<int>(static_cast<int64_t>(split) * a.k_steps[prob] / a.splits[prob]);
     const int k_end = static_cast<int>(static_cast<int64_t>(split + 1) * a.k_steps[prob] / a.splits[prob]);
     const int nk = k_end - k_begin;
-    const int N = a.n_cols[prob];
-    const uint32_t b_bytes = prob == 0 ? static_cast<uint32_t>(a.d_idx + a.h_idx) * kPBk * 2u
-                                       : static_cast<uint32_t>(kPBm) * kPBk * 2u;
-    const uint32_t tmem_cols = N <= 128 ? 128u : 256u;
+    const int N = a.n_tok;
+    const uint32_t tmem_cols = N <= 32 ? 32u : (N <= 64 ? 64u : (N <= 128 ? 128u : 256u));
+    // problem 0: the two 64-row pieces of this tile come from W_k or W_proj
+    const int n_out = prob == 0 ? a.d_idx + a.h_idx : a.h_idx * a.d_idx;
+    uint32_t piece_bytes[2] = {0u, 0u};
+    if (prob == 0) {
+        for (int pc = 0; pc < 2; ++pc) {
+            const int r0 = m_tile * kPBm + 64 * pc;
+            if (r0 < a.d_idx) piece_bytes[pc] = 64u * kPBk * 2u;
+            else if (r0 < a.d_idx + a.h_idx) piece_bytes[pc] = static_cast<uint32_t>(a.h_idx) * kPBk * 2u;
+        }
+    }
+    const uint32_t a_bytes = prob == 0 ? piece_bytes[0] + piece_bytes[1] : static_cast<uint32_t>(kPABytes);
+    const uint32_t b_bytes = static_cast<uint32_t>(N) * kPBk * 2u;
 
     if (tid == 0) {
         sm.abort = 0;
-        for (int s = 0; s < kProjStages; ++s) {
+        for (int s = 0; s < a.stages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -149,23 +161,27 @@ __global__ void __launch_bounds__(192, 1)
                     sm.abort = 1;
                     break;
                 }
-                uint8_t *st = base + s * kPStageBytes;
+                uint8_t *st = base + static_cast<uint32_t>(s) * a.stage_bytes;
                 const int k0 = (k_begin + t) * kPBk;
-                mbar_arrive_expect_tx(&sm.full[s], kPABytes + b_bytes);
+                mbar_arrive_expect_tx(&sm.full[s], a_bytes + b_bytes);
                 if (prob == 0) {
-                    tma_load_2d(st, &x_map, &sm.full[s], k0, m_tile * kPBm);
-                    tma_load_2d(st + kPABytes, &wk_map, &sm.full[s], k0, 0);
-                    tma_load_2d(st + kPABytes + a.d_idx * kPBk * 2, &wp_map, &sm.full[s], k0, 0);
+                    for (int pc = 0; pc < 2; ++pc) {
+                        const int r0 = m_tile * kPBm + 64 * pc;
+                        if (r0 < a.d_idx) tma_load_2d(st + pc * 64 * 128, &wk_map, &sm.full[s], k0, r0);
+                        else if (r0 < a.d_idx + a.h_idx)
+                            tma_load_2d(st + pc * 64 * 128, &wp_map, &sm.full[s], k0, r0 - a.d_idx);
+                    }
+                    tma_load_2d(st + kPABytes, &x_map, &sm.full[s], k0, t_tile * N);
                 } else {
-                    tma_load_2d(st, &ql_map, &sm.full[s], k0, m_tile * kPBm);
-                    tma_load_2d(st + kPABytes, &wq_map, &sm.full[s], k0, n_tile * kPBm);
+                    tma_load_2d(st, &wq_map, &sm.full[s], k0, m_tile * kPBm);
+                    tma_load_2d(st + kPABytes, &ql_map, &sm.full[s], k0, t_tile * N);
                 }
                 t_end = t + 1;
-                if (++s == kProjStages) { s = 0; ph ^= 1; }
+                if (++s == a.stages) { s = 0; ph ^= 1; }
             }
             // every load issued lands before the CTA may exit
-            for (int t = max(t_end - kProjStages, 0); t < t_end; ++t)
-                mbar_wait(&sm.full[t % kProjStages], static_cast<uint32_t>(t / kProjStages) & 1u, a.wait_budget);
+            for (int t = max(t_end - a.stages, 0); t < t_end; ++t)
+                mbar_wait(&sm.full[t % a.stages], static_cast<uint32_t>(t / a.stages) & 1u, a.wait_budget);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -179,7 +195,7 @@ __global__ void __launch_bounds__(192, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t aa = smem_u32(base + s * kPStageBytes);
+                const uint32_t aa = smem_u32(base + static_cast<uint32_t>(s) * a.stage_bytes);
                 const uint32_t ba = aa + kPABytes;
 #pragma unroll
                 for (int kk = 0; kk < kPBk / 16; ++kk) {
@@ -188,37 +204,30 @@ __global__ void __launch_bounds__(192, 1)
                     mma_bf16_ss(tmem, ad, bd, idesc, (t > 0 || kk > 0) ? 1u : 0u);
                 }
                 tc_commit(&sm.empty[s]);
-                if (++s == kProjStages) { s = 0; ph ^= 1; }
+                if (++s == a.stages) { s = 0; ph ^= 1; }
             }
             // completes once every MMA issued above has (also when none was)
             tc_commit(&sm.acc_full);
         }
     } else {
-        // epilogue: TMEM lane = token row of the tile
+        // epilogue: TMEM lane = output row, column = token of the tile
         const int quarter = warp & 3;
-        const int m = m_tile * kPBm + quarter * 32 + lane;
+        const int col = m_tile * kPBm + quarter * 32 + lane;  // output index (column of part)
         const bool ok = warp_wait(&sm.acc_full, 0, &sm.abort, a.wait_budget);
         if (ok) {
             tc_fence_after();
-            // valid columns of this tile
-            const int ncol = prob == 0 ? a.d_idx + a.h_idx : min(kPBm, a.ld[1] - n_tile * kPBm);
-            float *row = a.part[prob] + (static_cast<int64_t>(split) * a.nt + m) * a.ld[prob] +
-                         static_cast<int64_t>(n_tile) * kPBm;
             const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+            float *p = a.part[prob] + static_cast<int64_t>(split) * a.nt * a.ld[prob] + col;
             for (int c0 = 0; c0 < N; c0 += 32) {
                 uint32_t v[32];
                 tmem_ld32(lane_addr + c0, v);
                 tmem_wait_ld();
-                if (m < a.nt) {
+                if (col < n_out) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        if (c0 + j + 3 < ncol)
-                            *reinterpret_cast<float4 *>(row + c0 + j) =
-                                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                            __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                        else
-                            for (int e = 0; e < 4; ++e)
-                                if (c0 + j + e < ncol) row[c0 + j + e] = __uint_as_float(v[j + e]);
+                    for (int j = 0; j < 32; ++j) {
+                        const int token = t_tile * N + c0 + j;
+                        if (c0 + j < N && token < a.nt) p[static_cast<int64_t>(token) * a.ld[prob]] = __uint_as_float(v[j]);
+                    }
                 }
             }
         } else if (lane == 0) {
@@ -349,11 +358,11 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
 cudaError_t launch_project(const CUtensorMap &x_map, const CUtensorMap &ql_map, const CUtensorMap &wk_map,
                            const CUtensorMap &wp_map, const CUtensorMap &wq_map, const ProjGemmParams &g,
                            const ProjEpiParams &e, cudaStream_t st) {
-    const size_t smem = static_cast<size_t>(kProjStages) * kPStageBytes + sizeof(ProjSmem) + 1024;
+    const size_t smem = static_cast<size_t>(g.stages) * g.stage_bytes + sizeof(ProjSmem) + 1024;
     cudaError_t err = cudaFuncSetAttribute(k5_proj_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(smem));
     if (err != cudaSuccess) return err;
-    const int grid = g.items0 + g.m_tiles * g.n_tiles[1] * g.splits[1];
+    const int grid = g.items0 + g.m_tiles[1] * g.t_tiles * g.splits[1];
     if (grid == 0 || g.nt == 0) return cudaSuccess;
     k5_proj_gemm<<<grid, 192, smem, st>>>(x_map, ql_map, wk_map, wp_map, wq_map, g);
     err = cudaGetLastError();
