@@ -70,10 +70,10 @@ L2_BYTES = 126 * 1024 * 1024
 STAGE_ITERS = 200  # iterations of each stage-alone timing loop (more clock samples)
 
 
-# DRAM traffic of the fused indexer from one ncu capture of the 16 x 98304
+# DRAM traffic of the fused indexer from one ncu capture of the 16 x 65536
 # decode case (dram__bytes_read.sum + dram__bytes_write.sum per launch over
-# the scored positions), valid only while the kernel sources hash to the
-# captured build; the capture is summarised under profiles/.
+# the scored positions), valid only while the indexer's sources hash to the
+# captured build.
 K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
               "long_context_decode_indexer_b200/csrc/select.cuh",
               "long_context_decode_indexer_b200/csrc/ptx.cuh",

@@ -47,6 +47,16 @@ bool inject_timeout(const char *kernel) {
     return v != nullptr && strcmp(v, kernel) == 0;
 }
 
+// Test hook for callers' error handling: DSA_TEST_INJECT_HOST_ERROR=<step>
+// (indexer, attention, index_kl, masked_mha, project, or all) makes that
+// step fail on the host with DSA_ERR_CUDA after its arguments were
+// validated, before anything is enqueued.  Unset, it does nothing.
+int host_fault(const char *step) {
+    const char *v = getenv("DSA_TEST_INJECT_HOST_ERROR");
+    if (v == nullptr || (strcmp(v, step) != 0 && strcmp(v, "all") != 0)) return DSA_OK;
+    return fail(DSA_ERR_CUDA, "injected host failure in %s (DSA_TEST_INJECT_HOST_ERROR)", step);
+}
+
 size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ---------------------------------------------------------------- TMA maps
@@ -489,6 +499,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
     a.nsel = nsel;
     a.status = at<int>(ws, wl.status);
     a.wait_budget = dsa::kWaitBudgetCycles;
+    if (int rc = host_fault("indexer")) return rc;
     if (mode != dsa::kModeTopk && inject_timeout("indexer")) {
         a.wait_budget = kTestWaitBudget;
         a.inject = 1;
@@ -542,6 +553,7 @@ int run_mla(const dsa_params *p, const dsa_kv *kv, const void *q, const void *kv
             int64_t kv_row_stride, const int32_t *idx, void *out, float *lse, void *ws,
             const WsLayout &wl, const MlaPlan &m, cudaStream_t st, const float *kv_scale = nullptr) {
     if (p->nq == 0) return DSA_OK;
+    if (int rc = host_fault("attention")) return rc;
     CUtensorMap qmap;
     const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
     int rc = make_map_2d(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, dsa::kDqk,
@@ -803,6 +815,7 @@ int dsa_index_kl(const dsa_params *p, const dsa_kv *kv, const void *q, const voi
     if (!rc) rc = check_ws(ws, ws_bytes, wl);
     if (rc) return rc;
     if (p->nq == 0) return DSA_OK;
+    if (int frc = host_fault("index_kl")) return frc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     CUtensorMap qmap;
     const uint32_t hbox = p->h < 128 ? static_cast<uint32_t>(p->h) : 128u;
@@ -864,6 +877,7 @@ int dsa_masked_mha_prefill(const dsa_params *p, const dsa_kv *kv, const void *q,
     if (!rc) rc = check_ws(ws, ws_bytes, wl);
     if (rc) return rc;
     if (p->nq == 0) return DSA_OK;
+    if (int frc = host_fault("masked_mha")) return frc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const uint64_t H = static_cast<uint64_t>(p->h);
     CUtensorMap qmap, kmap, vmap;
@@ -1005,6 +1019,7 @@ int dsa_indexer_project(const dsa_project_params *pp, const dsa_kv *kv, const vo
         !aligned(w_proj, 16) || !aligned(q_idx, 4) || !aligned(kidx_cache, 4))
         return fail(DSA_ERR_INVALID_ARG, "x, q_lora and the weights must be 16-byte aligned, q_idx and "
                                          "kidx_cache 4-byte aligned");
+    if (int frc = host_fault("project")) return frc;
     CUtensorMap xm, qm, km, pm, wm;
     const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;

@@ -16,13 +16,16 @@
 // over [row, head, dim], 128B swizzle); warp 1 issues the tcgen05 MMAs;
 // warps 2-9 run the softmax, two warps per query row (= TMEM lane), each on
 // half of a tile's keys.
-//   S(j) = Q . K(j)^T      M = 128 queries, N = 128 keys, K = d_qk; two TMEM
-//                           buffers, so S(j+1) is computed during softmax(j)
+//   S(j) = Q . K(j)^T      M = 128 queries, N = 128 keys, K = d_qk; one TMEM
+//                           buffer, which the softmax reads first thing, so
+//                           S(j+1) is computed during softmax(j)
 //   P(j) = 2^(S' - m)      S' = S * scale * log2(e), masked keys -inf; P goes
-//                           to TMEM as a pair of bf16 tiles P_hi + P_lo
-//                           (together exact to ~2^-16, as in the decode
-//                           attention) and is the A operand of
-//   O   += P(j) . V(j)      V(j) MN-major from shared memory, O in TMEM.
+//                           to TMEM (two buffers) as a pair of bf16 tiles
+//                           P_hi + P_lo (together exact to ~2^-16, as in the
+//                           decode attention) and is the A operand of
+//   O   += P(j) . V(j)      V(j) MN-major from shared memory, O in TMEM; with
+//                           two P buffers P(j+1) is written while P(j) . V(j)
+//                           runs.
 // The running max m is raised only when a tile's max exceeds it by more than
 // 2^8 (then O and the row sum are rescaled once); otherwise P <= 2^8 and
 // nothing is rescaled.  O / l and the log-sum-exp are exact either way.
@@ -42,10 +45,10 @@ namespace dsa {
 namespace {
 
 constexpr uint32_t kChunkBytes = kMhaTile * 128u;  // 128 rows x 64 bf16 columns
-constexpr uint32_t kColS = 0;                       // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;                     // O: d_v <= 128 columns
-constexpr uint32_t kColPhi = 384;                   // P_hi: 128 keys as 64 columns of bf16 pairs
-constexpr uint32_t kColPlo = 448;                   // P_lo
+constexpr uint32_t kColS = 0;                       // S: 128 columns
+constexpr uint32_t kColO = 128;                     // O: d_v <= 128 columns
+constexpr uint32_t kColP = 256;                     // two P buffers of 128 columns: P_hi (128 keys as 64
+                                                    // columns of bf16 pairs), then P_lo
 constexpr float kRaiseLog2 = 8.f;                   // raise the running max only past 2^8
 
 struct MhaSmem {
@@ -54,10 +57,10 @@ struct MhaSmem {
     uint64_t k_empty[kMhaMaxStages];
     uint64_t v_full[kMhaVStages];
     uint64_t v_empty[kMhaVStages];
-    uint64_t s_full[2];
-    uint64_t s_free[2];
-    uint64_t p_full;
-    uint64_t pv_done;
+    uint64_t s_full;
+    uint64_t s_free;
+    uint64_t p_full[2];
+    uint64_t pv_done[2];
     uint64_t mma_done;
     uint32_t tmem_base;
     volatile int32_t abort;
@@ -123,12 +126,12 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             mbar_init(&sm.v_full[s], 1);
             mbar_init(&sm.v_empty[s], 1);
         }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.s_free, 8);  // the eight softmax warps
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&sm.s_full[b], 1);
-            mbar_init(&sm.s_free[b], 8);  // the eight softmax warps
+            mbar_init(&sm.p_full[b], 8);
+            mbar_init(&sm.pv_done[b], 1);
         }
-        mbar_init(&sm.p_full, 8);
-        mbar_init(&sm.pv_done, 1);
         mbar_init(&sm.mma_done, 1);
         fence_mbar_init();
     }
@@ -208,12 +211,12 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
             const uint32_t idesc_s = make_idesc(1, 1, 0, 0, 128, 128);
             const uint32_t idesc_pv = make_idesc(1, 1, 0, 1, 128, static_cast<uint32_t>(a.d_v));
             const uint32_t qa = smem_u32(base + L.q);
-            // S(j) into buffer j % 2 once softmax has read S(j - 2) from it
+            // S(j) once the softmax has read S(j - 1) (it does so first thing)
             auto issue_s = [&](int j) -> bool {
-                const int st = j % a.stages, b = j & 1;
+                const int st = j % a.stages;
                 if (!mbar_wait(&sm.k_full[st], static_cast<uint32_t>(j / a.stages) & 1u, a.wait_budget) || sm.abort)
                     return false;
-                if (j >= 2 && !mbar_wait(&sm.s_free[b], static_cast<uint32_t>((j - 2) >> 1) & 1u, a.wait_budget))
+                if (j >= 1 && !mbar_wait(&sm.s_free, static_cast<uint32_t>(j - 1) & 1u, a.wait_budget))
                     return false;
                 tc_fence_after();
                 const uint32_t ka = smem_u32(base + L.k_ring + st * L.k_stage);
@@ -222,17 +225,17 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t ad = make_sdesc(qa + c * kChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
                         const uint64_t bd = make_sdesc(ka + c * kChunkBytes + kk * 32, 16, 1024, kSwizzle128B);
-                        mma_bf16_ss(tmem + kColS + b * 128, ad, bd, idesc_s, (c > 0 || kk > 0) ? 1u : 0u);
+                        mma_bf16_ss(tmem + kColS, ad, bd, idesc_s, (c > 0 || kk > 0) ? 1u : 0u);
                     }
                 tc_commit(&sm.k_empty[st]);
-                tc_commit(&sm.s_full[b]);
+                tc_commit(&sm.s_full);
                 return true;
             };
             bool ok = mbar_wait(&sm.q_full, 0, a.wait_budget) && !sm.abort;
             if (ok) ok = issue_s(0);
             for (int j = 0; j < nkt && ok; ++j) {
                 if (j + 1 < nkt && !(ok = issue_s(j + 1))) break;
-                if (!mbar_wait(&sm.p_full, static_cast<uint32_t>(j) & 1u, a.wait_budget) ||
+                if (!mbar_wait(&sm.p_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, a.wait_budget) ||
                     !mbar_wait(&sm.v_full[j % kMhaVStages], static_cast<uint32_t>(j / kMhaVStages) & 1u,
                                a.wait_budget) ||
                     sm.abort) {
@@ -247,11 +250,12 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
 #pragma unroll
                 for (int ks = 0; ks < kMhaTile / 16; ++ks) {
                     const uint64_t bd = make_sdesc(va + ks * 2048, kChunkBytes, 1024, kSwizzle128B);
-                    mma_bf16_ts(tmem + kColO, tmem + kColPhi + ks * 8, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-                    mma_bf16_ts(tmem + kColO, tmem + kColPlo + ks * 8, bd, idesc_pv, 1u);
+                    const uint32_t pcol = kColP + (j & 1) * 128 + ks * 8;
+                    mma_bf16_ts(tmem + kColO, tmem + pcol, bd, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+                    mma_bf16_ts(tmem + kColO, tmem + pcol + 64, bd, idesc_pv, 1u);
                 }
                 tc_commit(&sm.v_empty[j % kMhaVStages]);
-                tc_commit(&sm.pv_done);
+                tc_commit(&sm.pv_done[j & 1]);
             }
             if (!ok) {
                 record_status(a.status, DSA_ERR_TIMEOUT);
@@ -281,19 +285,19 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
         float m_used = -INFINITY, l = 0.f;  // l: this half's share of the row sum
         bool ok = true;
         for (int j = 0; j < nkt; ++j) {
-            const int b = j & 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[b], static_cast<uint32_t>(j >> 1) & 1u, a.wait_budget) &&
+            const int b = j & 1;  // P buffer; also the slot of the half-max exchange
+            ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full, static_cast<uint32_t>(j) & 1u, a.wait_budget) &&
                                              !sm.abort);
             ok = bar_and(bar_id, 64, ok);
             if (!ok) break;
             tc_fence_after();
             uint32_t u[64];
-            tmem_ld32(lane_addr + kColS + b * 128 + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
-            tmem_ld32(lane_addr + kColS + b * 128 + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
+            tmem_ld32(lane_addr + kColS + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(u));
+            tmem_ld32(lane_addr + kColS + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(u + 32));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_free[b]);
+            if (lane == 0) mbar_arrive(&sm.s_free);
             // keys j*128 + hf*64 + c kept: below n_t and in the index set
             uint32_t mw[2];
 #pragma unroll
@@ -324,15 +328,23 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
                 m_used = mt;
                 l *= alpha;
             }
-            // P(j) replaces P(j - 1), and O must hold every tile before j
-            if (j > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(&sm.pv_done, static_cast<uint32_t>(j - 1) & 1u, a.wait_budget) &&
-                                                 !sm.abort);
+            // P(j) goes to buffer j % 2, which P(j - 2) . V(j - 2) must be done
+            // reading; a rescale of O needs every tile before j in O.  (The
+            // two warps of a pair hold the same rows: same decisions, same
+            // waits.)
+            const bool need_o = __any_sync(0xffffffffu, rescale) && j >= 1;
+            if (j >= 2 || need_o) {
+                bool w = true;
+                if (need_o)
+                    w = mbar_wait(&sm.pv_done[(j - 1) & 1], static_cast<uint32_t>((j - 1) >> 1) & 1u, a.wait_budget);
+                if (w && j >= 2)
+                    w = mbar_wait(&sm.pv_done[b], static_cast<uint32_t>((j - 2) >> 1) & 1u, a.wait_budget);
+                ok = __all_sync(0xffffffffu, w && !sm.abort);
                 ok = bar_and(bar_id, 64, ok);  // both warps of the pair leave together
                 if (!ok) break;
                 tc_fence_after();
             }
-            if (__any_sync(0xffffffffu, rescale)) {
+            if (need_o) {
                 const float f = rescale ? alpha : 1.f;
                 for (int c = oc0; c < oc1; c += 32) {
                     uint32_t o[32];
@@ -358,19 +370,21 @@ __global__ void __launch_bounds__(kMhaThreads, 1)
                     hi[e] = bf16x2_bits(h2);
                     lo[e] = bf16x2_bits(__floats2bfloat162_rn(p0 - hfl.x, p1 - hfl.y));
                 }
-                tmem_st16(lane_addr + kColPhi + hf * 32 + c0 / 2, hi);
-                tmem_st16(lane_addr + kColPlo + hf * 32 + c0 / 2, lo);
+                tmem_st16(lane_addr + kColP + b * 128 + hf * 32 + c0 / 2, hi);
+                tmem_st16(lane_addr + kColP + b * 128 + 64 + hf * 32 + c0 / 2, lo);
             }
             l += lsum;
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.p_full);
+            if (lane == 0) mbar_arrive(&sm.p_full[b]);
         }
         // epilogue: O / l as bf16 (this warp's columns), and the log-sum-exp
         if (ok && nkt > 0)
             ok = __all_sync(0xffffffffu,
-                            mbar_wait(&sm.pv_done, static_cast<uint32_t>(nkt - 1) & 1u, a.wait_budget) && !sm.abort);
+                            mbar_wait(&sm.pv_done[(nkt - 1) & 1], static_cast<uint32_t>((nkt - 1) >> 1) & 1u,
+                                      a.wait_budget) &&
+                                !sm.abort);
         sm.half_sum[hf][r] = l;
         ok = bar_and(bar_id, 64, ok);
         if (ok) {

@@ -241,14 +241,20 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------------------
-// k6: per token, sum the K slices (in slice order) and finish the producer.
-// 256 threads; lane l of a warp holds dims [l * per, (l + 1) * per) of a
+// k6: sum the K slices (in slice order) and finish the producer.  Grid
+// (token, 1 + H_I / 8): block y = 0 produces the token's k^I (warp 0) and
+// the raw head weights (warp 1); block y >= 1 produces q^I heads
+// 8 (y - 1) .. 8 (y - 1) + 7, one per warp, each warp summing its own head
+// weight.  Lane l of a warp holds dims [l * per, (l + 1) * per) of a
 // d_I-wide vector (per = d_I / 32: 4 or 2), so every RoPE pair is in-lane.
+// Spreading a token over several CTAs keeps the dependent chains (partial
+// loads, reductions, quantisation) short: one CTA per token ran them head
+// after head.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
-    __shared__ float wraw[64];
     __shared__ double2 rope_table[64];  // (sin, cos) of each rotated pair at this token's position
     const int t = blockIdx.x;
+    const int hgroup = static_cast<int>(blockIdx.y) - 1;  // -1: the k^I block
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int d = a.d_idx, H = a.h_idx, per = a.d_idx / 32;
     const int pos = a.positions[t];
@@ -259,7 +265,7 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
     }
     __syncthreads();
 
-    if (warp == 0) {
+    if (hgroup < 0 && warp == 0) {
         // ---- k^I: LayerNorm, RoPE, FP8 with a power-of-two scale, cache append
         float v[4];
         for (int i = 0; i < per; ++i) {
@@ -309,18 +315,19 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
         }
         if (a.k_f32)
             for (int i = 0; i < per; ++i) a.k_f32[static_cast<int64_t>(t) * d + lane * per + i] = v[i];
-    } else if (warp == 1) {
-        // ---- the raw head weights W_proj . x
-        for (int j = lane; j < H; j += 32) {
-            float acc = 0.f;
-            for (int s = 0; s < a.splits0; ++s) acc += a.part0[(static_cast<int64_t>(s) * a.nt + t) * a.ld0 + d + j];
-            wraw[j] = acc;
-            if (a.w_f32) a.w_f32[static_cast<int64_t>(t) * H + j] = acc;
-        }
+    } else if (hgroup < 0 && warp == 1) {
+        // ---- the raw head weights W_proj . x (optional fp32 output)
+        if (a.w_f32)
+            for (int j = lane; j < H; j += 32) {
+                float acc = 0.f;
+                for (int s = 0; s < a.splits0; ++s) acc += a.part0[(static_cast<int64_t>(s) * a.nt + t) * a.ld0 + d + j];
+                a.w_f32[static_cast<int64_t>(t) * H + j] = acc;
+            }
     }
-    __syncthreads();
-    // ---- q^I heads: RoPE, FP8 with a power-of-two scale; w folds the scale
-    for (int h = warp; h < H; h += 8) {
+    // ---- q^I head h of this block: RoPE, FP8 with a power-of-two scale; w
+    // folds the scale
+    const int h = hgroup * 8 + warp;
+    if (hgroup >= 0 && h < H) {
         float v[4];
         const int64_t col0 = static_cast<int64_t>(h) * d + lane * per;
         for (int i = 0; i < per; ++i) {
@@ -346,9 +353,11 @@ __global__ void __launch_bounds__(256) k6_proj_epilogue(const ProjEpiParams a) {
         if (lane == 0) {
             const int64_t th = static_cast<int64_t>(t) * H + h;
             if (a.q_scale) a.q_scale[th] = scale;
+            float wraw = 0.f;  // W_proj . x for head h, slices summed in order
+            for (int s = 0; s < a.splits0; ++s) wraw += a.part0[(static_cast<int64_t>(s) * a.nt + t) * a.ld0 + d + h];
             // the same operations, in the same order, as the definition:
             // w / sqrt(H_I) / sqrt(d_I) * q_scale, then bf16 (ties to even)
-            const double wv = static_cast<double>(wraw[h]) / sqrt(static_cast<double>(H)) /
+            const double wv = static_cast<double>(wraw) / sqrt(static_cast<double>(H)) /
                               sqrt(static_cast<double>(d)) * static_cast<double>(scale);
             a.w[th] = __bfloat16_as_ushort(__double2bfloat16(wv));
         }
@@ -367,7 +376,7 @@ cudaError_t launch_project(const CUtensorMap &x_map, const CUtensorMap &ql_map, 
     k5_proj_gemm<<<grid, 192, smem, st>>>(x_map, ql_map, wk_map, wp_map, wq_map, g);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    k6_proj_epilogue<<<g.nt, 256, 0, st>>>(e);
+    k6_proj_epilogue<<<dim3(g.nt, 1 + (g.h_idx + 7) / 8), 256, 0, st>>>(e);
     return cudaGetLastError();
 }
 

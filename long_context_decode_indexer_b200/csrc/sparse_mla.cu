@@ -126,71 +126,86 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return a | (b << 16);
 }
 
-// Eight e4m3 codes (one 8-byte load) times a power-of-two row scale as eight
-// bf16 values (a 16-byte shared-memory piece).  e4m3 -> f16 is exact, the
-// power-of-two product is exact in fp32 and a value with 4 significant bits
-// is exact in bf16: the piece equals the cache's value, with no rounding.
-__device__ __forceinline__ uint4 fp8x8_to_bf16x8(uint2 codes, float sc) {
-    const uint32_t w[2] = {codes.x, codes.y};
-    uint32_t o[4];
+// Sixteen e4m3 codes (one 16-byte load) times a power-of-two row scale as
+// sixteen bf16 values (two 16-byte shared-memory pieces).  e4m3 -> f16 is
+// exact, the power-of-two product is exact in fp32 and a value with 4
+// significant bits is exact in bf16: the pieces equal the cache's values.
+__device__ __forceinline__ void fp8x16_to_bf16x16(uint4 codes, float sc, uint4 &lo, uint4 &hi) {
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    uint32_t o[8];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
         const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFFFFu);
         const __half2 h = __half2(__nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3));
         const float2 f = __half22float2(h);
         o[i] = pack_bf16x2(f.x * sc, f.y * sc);
     }
-    return make_uint4(o[0], o[1], o[2], o[3]);
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-__device__ __forceinline__ uint2 ldg_u2(const uint8_t *p) {
-    return __ldg(reinterpret_cast<const uint2 *>(p));
+__device__ __forceinline__ uint4 ldg_u4(const uint8_t *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
 }
 
-// Pass-1 gathers from an FP8 cache: the same piece ownership as the bf16
-// gather below, with the 8 codes of a piece loaded into registers two
-// chunks ahead, converted, and stored into the swizzled stage; a chunk is
-// published once this thread's stores of it are done.
+constexpr int kFp8Rows = kMlaMaxRows / (kPass1Threads / 4);  // pass-1 rows per gather thread (FP8)
+
+// Pass-1 gathers from an FP8 cache.  Gather thread gt owns the 16-byte code
+// piece j4 = gt % 4 (codes 16 j4 .. 16 j4 + 15 of each 64-column chunk, two
+// bf16 pieces of the swizzled stage) of rows gt / 4 + 64 k; its loads run
+// two chunks ahead in registers; a chunk is published once this thread's
+// stores of it are done.
 __device__ bool gather_pass1_fp8(const MlaParams &a, MlaSmem &sm, uint8_t *ring, int gt, int Rp) {
-    const int j = gt & 7, r0 = gt >> 3, lane = threadIdx.x & 31;
-    const uint8_t *src[kPass1Rows];
-    uint32_t dst[kPass1Rows];
-    float sc[kPass1Rows];
+    const int j4 = gt & 3, r0 = gt >> 2, lane = threadIdx.x & 31;
+    const uint8_t *src[kFp8Rows];
+    uint32_t dst0[kFp8Rows], dst1[kFp8Rows];
+    float sc[kFp8Rows];
 #pragma unroll
-    for (int k = 0; k < kPass1Rows; ++k) {
-        const int r = r0 + 32 * k;
-        src[k] = a.kv8 + static_cast<int64_t>(sm.rows[r]) * a.kv8_row_bytes + j * 8;
-        dst[k] = static_cast<uint32_t>(r * 128 + ((j ^ (r & 7)) << 4));
+    for (int k = 0; k < kFp8Rows; ++k) {
+        const int r = r0 + 64 * k;
+        src[k] = a.kv8 + static_cast<int64_t>(sm.rows[r]) * a.kv8_row_bytes + j4 * 16;
+        dst0[k] = static_cast<uint32_t>(r * 128 + (((2 * j4) ^ (r & 7)) << 4));
+        dst1[k] = static_cast<uint32_t>(r * 128 + (((2 * j4 + 1) ^ (r & 7)) << 4));
         sc[k] = sm.valid[r] ? a.kv_scale[sm.rows[r]] : 0.f;
     }
-    constexpr int kAhead = 2;
-    uint2 buf[kAhead + 1][kPass1Rows];
-    auto load = [&](int c, uint2 (&b)[kPass1Rows]) {
+    // registers two chunks ahead, shifted down each chunk (a rolled loop:
+    // the unrolled one stalled on instruction fetch)
+    uint4 b0[kFp8Rows], b1[kFp8Rows], b2[kFp8Rows];
+    auto load = [&](int c, uint4 (&b)[kFp8Rows]) {
 #pragma unroll
-        for (int k = 0; k < kPass1Rows; ++k)
-            b[k] = (r0 + 32 * k < Rp) ? ldg_u2(src[k] + c * 64) : make_uint2(0u, 0u);
+        for (int k = 0; k < kFp8Rows; ++k)
+            b[k] = (r0 + 64 * k < Rp) ? ldg_u4(src[k] + c * 64) : make_uint4(0u, 0u, 0u, 0u);
     };
-#pragma unroll
-    for (int c = 0; c < kAhead; ++c) load(c, buf[c]);
+    load(0, b0);
+    load(1, b1);
     bool ok = true;
-#pragma unroll
+#pragma unroll 1
     for (int c = 0; c < kNumKChunks; ++c) {
-        if (c + kAhead < kNumKChunks) load(c + kAhead, buf[(c + kAhead) % (kAhead + 1)]);
+        if (c + 2 < kNumKChunks) load(c + 2, b2);
         const int s = c % kMlaStages;
         const uint32_t ph = (c / kMlaStages) & 1;
         ok = ok && __all_sync(0xffffffffu, mbar_wait(&sm.empty[s], ph ^ 1, a.wait_budget) && !sm.abort);
         if (ok) {
             uint8_t *kst = ring + s * kStageBytes + kQChunkBytes;
 #pragma unroll
-            for (int k = 0; k < kPass1Rows; ++k)
-                if (r0 + 32 * k < Rp)
-                    *reinterpret_cast<uint4 *>(kst + dst[k]) = fp8x8_to_bf16x8(buf[c % (kAhead + 1)][k], sc[k]);
+            for (int k = 0; k < kFp8Rows; ++k)
+                if (r0 + 64 * k < Rp) {
+                    uint4 lo, hi;
+                    fp8x16_to_bf16x16(b0[k], sc[k], lo, hi);
+                    *reinterpret_cast<uint4 *>(kst + dst0[k]) = lo;
+                    *reinterpret_cast<uint4 *>(kst + dst1[k]) = hi;
+                }
         }
         fence_proxy_async_smem();
         __syncwarp();
         // tests only: the first CTA never publishes chunk 0
         const bool skip = a.inject != 0 && blockIdx.x == 0 && c == 0;
         if (lane == 0 && !skip) mbar_arrive(&sm.full[s]);
+#pragma unroll
+        for (int k = 0; k < kFp8Rows; ++k) {
+            b0[k] = b1[k];
+            b1[k] = b2[k];
+        }
     }
     return ok;
 }
@@ -461,16 +476,18 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                 const int vr = gt >> 2, vu = gt & 3;
                 const int nvt = (Rp + kMlaVRows - 1) / kMlaVRows;
                 if constexpr (KV8) {
-                    // FP8 rows: this thread's 16 pieces of row vr of a tile,
-                    // loaded into registers one tile ahead and converted
-                    uint2 cur[16], nxt[16];
+                    // FP8 rows: this thread's 8 code pieces of 16 bytes
+                    // (u = vu + 4 m: value columns 16 u .. 16 u + 15, the bf16
+                    // pieces 2u and 2u + 1) of row vr of a tile, loaded into
+                    // registers one tile ahead and converted
+                    uint4 cur[8], nxt[8];
                     float csc = 0.f, nsc = 0.f;
-                    auto vload = [&](int vt, uint2 (&b)[16], float &sc) {
+                    auto vload = [&](int vt, uint4 (&b)[8], float &sc) {
                         const int rr = vt * kMlaVRows + vr;
                         const uint8_t *vsrc = a.kv8 + static_cast<int64_t>(sm.rows[rr]) * a.kv8_row_bytes;
                         sc = sm.valid[rr] ? a.kv_scale[sm.rows[rr]] : 0.f;
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) b[m] = ldg_u2(vsrc + (vu + 4 * m) * 8);
+                        for (int m = 0; m < 8; ++m) b[m] = ldg_u4(vsrc + (vu + 4 * m) * 16);
                     };
                     if (nvt > 0) vload(0, cur, csc);
                     for (int vt = 0; vt < nvt; ++vt) {
@@ -481,18 +498,20 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
                         if (ok) {
                             uint8_t *vdst = vring + v * kVTileBytes + vr * 128;
 #pragma unroll
-                            for (int m = 0; m < 16; ++m) {
-                                const int pc = vu + 4 * m;
-                                const int blk = pc >> 3, j = pc & 7;
-                                *reinterpret_cast<uint4 *>(vdst + blk * kVBlockBytes + ((j ^ (vr & 7)) << 4)) =
-                                    fp8x8_to_bf16x8(cur[m], csc);
+                            for (int m = 0; m < 8; ++m) {
+                                const int u = vu + 4 * m;
+                                const int pc0 = 2 * u, pc1 = 2 * u + 1;  // bf16 pieces (8 columns each)
+                                uint4 lo, hi;
+                                fp8x16_to_bf16x16(cur[m], csc, lo, hi);
+                                *reinterpret_cast<uint4 *>(vdst + (pc0 >> 3) * kVBlockBytes + (((pc0 & 7) ^ (vr & 7)) << 4)) = lo;
+                                *reinterpret_cast<uint4 *>(vdst + (pc1 >> 3) * kVBlockBytes + (((pc1 & 7) ^ (vr & 7)) << 4)) = hi;
                             }
                         }
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(&sm.v_full[v]);
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) cur[m] = nxt[m];
+                        for (int m = 0; m < 8; ++m) cur[m] = nxt[m];
                         csc = nsc;
                     }
                 } else {
@@ -766,27 +785,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1)
     __syncthreads();
     tc_fence_after();
     if (warp == 5) tmem_dealloc(tmem, 512);
+
 }
 
-// Merge the splits of one (query, head): out = sum_s w_s o_s / sum_s w_s with
-// w_s = exp(lse_s - max lse); lse = max + ln sum_s w_s.  A split's stored
-// half row is o_s * 2^-e_s (fp16), so it enters with the weight w_s * 2^e_s.  One warp covers 256
-// value columns of one head (8 per lane, 16-byte loads and stores), so a
-// head takes two warps and a 128-thread CTA two heads.  Every warp reads the
-// head's split log-sum-exps itself (lane s holds split s; splits <= 32) and
-// gets the weights by shuffles: no shared memory, no CTA barrier.  The
-// partial loads of all splits are issued before any is used.
-__global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_slots) {
-    grid_dependency_wait();  // the partials come from the preceding attention kernel
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int head_slot = blockIdx.x * 2 + (warp >> 1);  // (query in wave) * h + head
-    if (head_slot >= n_slots) return;                     // whole warp: odd head count
-    const int wq = head_slot / a.h, hh = head_slot % a.h;
+// Merge the splits of one (query, head), value columns [256 half, 256 half +
+// 256), by one warp: out = sum_s w_s o_s / sum_s w_s with w_s = exp(lse_s -
+// max lse); lse = max + ln sum_s w_s.  A split's stored half row is
+// o_s * 2^-e_s (fp16), so it enters with the weight w_s * 2^e_s.  Lane s
+// reads split s's log-sum-exp (splits <= 32) and the weights are shuffled
+// from it; 8 columns per lane, 16-byte loads and stores, the partial loads
+// of 8 splits issued before any is used.
+__device__ void combine_half_head(const MlaParams &a, int wq, int hh, int half) {
+    const int lane = threadIdx.x & 31;
     const int q = a.q0 + wq;
     const int64_t row0 = static_cast<int64_t>(wq) * a.splits * 128 + hh;  // split s: row0 + 128 s
-    const int d = (warp & 1) * 256 + lane * 8;
-    const float ls = lane < a.splits ? a.part_lse[row0 + 128 * lane] : -INFINITY;
-    const float sc = lane < a.splits ? a.part_scale[(row0 + 128 * lane) * 2 + (warp & 1)] : 0.f;
+    const int d = half * 256 + lane * 8;
+    const float ls = lane < a.splits ? __ldcg(&a.part_lse[row0 + 128 * lane]) : -INFINITY;
+    const float sc = lane < a.splits ? __ldcg(&a.part_scale[(row0 + 128 * lane) * 2 + half]) : 0.f;
     float mx = ls;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -798,7 +813,7 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_s
     uint16_t *o = a.out + (static_cast<int64_t>(q) * a.h + hh) * kDv + d;
     if (mx == -INFINITY) {
         *reinterpret_cast<uint4 *>(o) = make_uint4(0, 0, 0, 0);
-        if (lane == 0 && (warp & 1) == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
+        if (lane == 0 && half == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = -INFINITY;
         return;
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -807,7 +822,7 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_s
 #pragma unroll
         for (int u = 0; u < 8; ++u)
             raw[u] = s0 + u < a.splits
-                         ? *reinterpret_cast<const uint4 *>(a.part_o + (row0 + 128 * (s0 + u)) * kDv + d)
+                         ? __ldcg(reinterpret_cast<const uint4 *>(a.part_o + (row0 + 128 * (s0 + u)) * kDv + d))
                          : make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -828,7 +843,17 @@ __global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_s
     res.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
     res.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
     *reinterpret_cast<uint4 *>(o) = res;
-    if (lane == 0 && (warp & 1) == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
+    if (lane == 0 && half == 0) a.lse[static_cast<int64_t>(q) * a.h + hh] = mx + logf(tot);
+}
+
+// The split combine as its own kernel: one warp per half head, two heads per
+// 128-thread CTA, no shared memory, no CTA barrier.
+__global__ void __launch_bounds__(128) k4_mla_combine(const MlaParams a, int n_slots) {
+    grid_dependency_wait();  // the partials come from the preceding attention kernel
+    const int warp = threadIdx.x >> 5;
+    const int head_slot = blockIdx.x * 2 + (warp >> 1);  // (query in wave) * h + head
+    if (head_slot >= n_slots) return;                     // whole warp: odd head count
+    combine_half_head(a, head_slot / a.h, head_slot % a.h, warp & 1);
 }
 
 // Each head's log-sum-exp over the whole set from its splits' (one warp per

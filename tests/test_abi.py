@@ -169,3 +169,26 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(dsa, "_lib", None)
     with pytest.raises(dsa.DsaError):
         dsa.lib()
+
+
+def test_host_fault_hook_fails_a_step_before_any_launch(L, monkeypatch):
+    """DSA_TEST_INJECT_HOST_ERROR=<step> makes that step return DSA_ERR_CUDA
+    after its arguments were validated and before anything is enqueued (no
+    GPU needed: the failure comes first); other steps are unaffected."""
+    p = _params(3)
+    kv = _kv()
+    fake = 1 << 40  # never dereferenced
+    need_idx = dsa.workspace_size(p, kv, dsa.OP_INDEXER_TOPK)
+    need_att = dsa.workspace_size(p, kv, dsa.OP_SPARSE_MLA_DECODE)
+    monkeypatch.setenv("DSA_TEST_INJECT_HOST_ERROR", "indexer")
+    rc = L.dsa_indexer_topk(ctypes.byref(p), ctypes.byref(kv), fake, fake, fake, None, fake, None,
+                            fake, need_idx, None)
+    assert rc == dsa.DSA_ERR_CUDA and "injected host failure in indexer" in dsa.last_error()
+    monkeypatch.setenv("DSA_TEST_INJECT_HOST_ERROR", "all")
+    rc = L.dsa_sparse_mla_decode(ctypes.byref(p), ctypes.byref(kv), fake, fake, 576, fake, fake, fake,
+                                 fake, need_att, None)
+    assert rc == dsa.DSA_ERR_CUDA and "injected host failure in attention" in dsa.last_error()
+    # validation still comes first: a bad workspace is reported as such
+    rc = L.dsa_indexer_topk(ctypes.byref(p), ctypes.byref(kv), fake, fake, fake, None, fake, None,
+                            fake, need_idx - 256, None)
+    assert rc == dsa.DSA_ERR_WORKSPACE
