@@ -637,6 +637,26 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     const int N = a.qg * HP;  // MMA N (columns per accumulator buffer)
 
     // ---- set-up
+    // The q^I tile and the weights are loaded first, into registers: issued
+    // before the TMA ring fills, they do not queue behind it.
+    constexpr int kQPieces = (kMaxGroupQueries * HP * (DI / 16) + kK1Threads - 1) / kK1Threads;
+    static_assert(kMaxGroupQueries * HP <= kK1Threads, "one weight per thread");
+    uint4 qv[kQPieces];
+#pragma unroll
+    for (int u = 0; u < kQPieces; ++u) {
+        const int i = tid + u * kK1Threads;
+        const int r = i / (DI / 16), ch = i % (DI / 16);
+        const int qi = r / HP, j = r % HP;
+        qv[u] = make_uint4(0, 0, 0, 0);
+        if (r < N && qi < nqg && j < a.h_idx)
+            qv[u] = *reinterpret_cast<const uint4 *>(a.q_idx + (static_cast<int64_t>(q0 + qi) * a.h_idx + j) * DI + ch * 16);
+    }
+    float wv = 0.f;
+    if (tid < N) {
+        const int qi = tid / HP, j = tid % HP;
+        if (qi < nqg && j < a.h_idx) wv = bf16_bits_to_float(a.w[static_cast<int64_t>(q0 + qi) * a.h_idx + j]);
+    }
+
     // ---- span of positions this CTA covers (every thread, from global q_n)
     int nmax = 0, nscored = 0;
     for (int i = 0; i < nqg; ++i) {
@@ -660,20 +680,23 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     const bool skip_first = a.inject != 0 && blockIdx.x == 0;
     // tile t: one 128-row box (contiguous cache; a box past the end of the
     // cache reads zeros), or one box per page
+    // k^I is read once per call: its lines go first when L2 needs room
+    const uint64_t stream_policy = l2_policy_evict_first();
     auto issue_tile = [&](int t, int s) {
         if (skip_first && t == 0) return;
         const int p0 = start + t * kTileRows;
         uint8_t *dst = stages + s * kTileBytes;
         if (a.page_table == nullptr) {
             mbar_arrive_expect_tx(&sm.full[s], kTileBytes);
-            tma_load_2d(dst, &kmap, &sm.full[s], 0, static_cast<int32_t>(row0 + p0));
+            tma_load_2d_hint(dst, &kmap, &sm.full[s], 0, static_cast<int32_t>(row0 + p0), stream_policy);
         } else {
             const int box = a.page_size;
             const int32_t *pt = a.page_table + static_cast<int64_t>(seq) * a.max_pages + p0 / box;
             int n_box = 0;
             for (int h = 0; h < kTileRows / box; ++h) n_box += (p0 + h * box < nmax);
             mbar_arrive_expect_tx(&sm.full[s], static_cast<uint32_t>(n_box * box * DI));
-            for (int h = 0; h < n_box; ++h, dst += box * DI) tma_load_2d(dst, &kmap, &sm.full[s], 0, pt[h] * box);
+            for (int h = 0; h < n_box; ++h, dst += box * DI)
+                tma_load_2d_hint(dst, &kmap, &sm.full[s], 0, pt[h] * box, stream_policy);
         }
     };
     const int n_pro = min(ntiles, a.stages);  // tiles issued before the set-up barrier
@@ -700,19 +723,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     }
     if (tid < kMaxGroupQueries) sm.n_q[tid] = tid < nqg ? a.q_n[q0 + tid] : 0;
     // q^I tile (B operand, K-major, swizzled like the TMA tiles) and weights
-    for (int i = tid; i < N * (DI / 16); i += blockDim.x) {
+#pragma unroll
+    for (int u = 0; u < kQPieces; ++u) {
+        const int i = tid + u * kK1Threads;
         const int r = i / (DI / 16), ch = i % (DI / 16);
-        const int qi = r / HP, j = r % HP;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (qi < nqg && j < a.h_idx)
-            v = *reinterpret_cast<const uint4 *>(a.q_idx + (static_cast<int64_t>(q0 + qi) * a.h_idx + j) * DI + ch * 16);
         const int sw = (DI == 128) ? (ch ^ (r & 7)) : (ch ^ ((r >> 1) & 3));
-        *reinterpret_cast<uint4 *>(qtile + r * DI + sw * 16) = v;
+        if (r < N) *reinterpret_cast<uint4 *>(qtile + r * DI + sw * 16) = qv[u];
     }
-    for (int i = tid; i < N; i += blockDim.x) {
-        const int qi = i / HP, j = i % HP;
-        wts[i] = (qi < nqg && j < a.h_idx) ? bf16_bits_to_float(a.w[static_cast<int64_t>(q0 + qi) * a.h_idx + j]) : 0.f;
-    }
+    if (tid < N) wts[tid] = wv;
     if (MODE == kModeFused)
         for (int i = tid; i < a.qg * kSelBins; i += blockDim.x) lhist[i] = 0;
     if (warp == 1) {
