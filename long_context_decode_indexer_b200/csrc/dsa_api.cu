@@ -278,8 +278,17 @@ int plan_indexer(const dsa_params *p, int mode, int64_t span, IndexerPlan &pl) {
         while (st >= 2 &&
                dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, st, !pl.parallel).total > 232448)
             --st;
+        // the two MMA threads take alternate tiles: an even ring, at least
+        // as deep as the accumulator ring (the epilogue's wait on a stage's
+        // commit relies on it)
+        st &= ~1;
         if (st < 2) return fail(DSA_ERR_UNSUPPORTED, "indexer shared memory plan too large");
         pl.stages = st;
+        if (pl.stages < pl.acc_bufs) {
+            pl.acc_bufs = 2;
+            pl.tmem_cols = 32;
+            while (pl.tmem_cols < static_cast<uint32_t>(pl.acc_bufs * pl.qg * pl.hp)) pl.tmem_cols <<= 1;
+        }
     }
     const dsa::K1Layout L = dsa::k1_layout(mode, p->d_idx, pl.qg, pl.hp, pl.chunk, pl.P, p->topk, pl.stages,
                                            !pl.parallel);

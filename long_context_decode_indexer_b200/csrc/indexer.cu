@@ -56,8 +56,7 @@ constexpr int kTileRows = 128;  // positions per ring stage, MMA (M) and epilogu
 
 struct K1Smem {
     uint64_t full[kK1MaxStages];
-    uint64_t empty[kK1MaxStages];
-    uint64_t acc_full[kK1MaxAcc];
+    uint64_t empty[kK1MaxStages];        // also the epilogue's "accumulator ready": one commit per tile
     uint64_t acc_empty[kK1MaxAcc];
     uint32_t tmem_base;
     volatile int32_t abort;
@@ -76,7 +75,7 @@ struct K1Smem {
     unsigned long long t_exact;          // parallel: the need-th largest listed composite
     uint64_t merge_bar;                  // merge: bulk copies of the candidate lists
     uint32_t merge_phase;
-    uint64_t mma_done;                   // every MMA issued by this CTA has completed
+    uint64_t mma_done[2];                // every MMA issued by MMA thread i has completed
     SelectScratch sel;
 };
 
@@ -706,14 +705,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
         sm.is_last = 0;
         for (int i = 0; i < kMaxGroupQueries; ++i) sm.g_complete[i] = 0;
         mbar_init(&sm.merge_bar, 1);
-        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.mma_done[0], 1);
+        mbar_init(&sm.mma_done[1], 1);
         sm.merge_phase = 0;
         for (int s = 0; s < a.stages; ++s) {
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < a.acc_bufs; ++b) {
-            mbar_init(&sm.acc_full[b], 1);
             mbar_init(&sm.acc_empty[b], 4);  // the four warps of epilogue group b % 2
         }
         fence_mbar_init();
@@ -777,8 +776,14 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                         !mbar_wait(&sm.full[t % a.stages], static_cast<uint32_t>(t / a.stages) & 1u, a.wait_budget))
                         record_status(a.status, DSA_ERR_TIMEOUT);
             }
-        } else if (warp == 1) {
+        } else if (warp == 1 || warp == 10) {
+            // two MMA threads: warp 1 issues the even tiles, warp 10 the odd
+            // ones (each tcgen05 instruction holds its issuing thread for
+            // tens of cycles; one thread issuing every tile paced the
+            // stream).  One commit per tile: empty[s] frees the ring stage
+            // and tells the epilogue that buffer b holds tile t.
             if (lane == 0) {
+                const int r0 = warp == 1 ? 0 : 1;
                 const uint32_t idesc = make_idesc(0, 0, 0, 0, kTileRows, N);
                 constexpr uint32_t kSbo = 8 * DI;
                 constexpr uint32_t kLayout = (DI == 128) ? kSwizzle128B : kSwizzle64B;
@@ -786,17 +791,19 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 // K step) is a fixed offset in the 16-byte address field
                 const uint64_t ad0 = make_sdesc(smem_u32(stages), 16, kSbo, kLayout);
                 const uint64_t bd0 = make_sdesc(smem_u32(qtile), 16, kSbo, kLayout);
-                int s = 0, b = 0;
+                // ring stage and accumulator of tile t = r0, r0 + 2, ...: both
+                // advance by two per tile (a.stages even, a.acc_bufs even)
+                int s = r0, b = r0;
                 uint32_t ph = 0, aph = 0;
-                for (int t = 0; t < ntiles; ++t) {
+                for (int t = r0; t < ntiles; t += 2) {
                     if (!mbar_wait(&sm.acc_empty[b], aph ^ 1, a.wait_budget) ||
                         !mbar_wait(&sm.full[s], ph, a.wait_budget) || sm.abort) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
                         sm.abort = 1;
                         // the MMAs already issued complete before TMEM is
                         // freed (on success the epilogue waits for each)
-                        tc_commit(&sm.mma_done);
-                        if (!mbar_wait(&sm.mma_done, 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
+                        tc_commit(&sm.mma_done[r0]);
+                        if (!mbar_wait(&sm.mma_done[r0], 0, a.wait_budget)) record_status(a.status, DSA_ERR_TIMEOUT);
                         break;
                     }
                     tc_fence_after();
@@ -805,9 +812,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                     for (int kk = 0; kk < DI / 32; ++kk)
                         mma_f8_ss(tmem + b * N, ad + 2 * kk, bd0 + 2 * kk, idesc, kk > 0 ? 1u : 0u);
                     tc_commit(&sm.empty[s]);
-                    tc_commit(&sm.acc_full[b]);
-                    if (++s == a.stages) { s = 0; ph ^= 1; }
-                    if (++b == a.acc_bufs) { b = 0; aph ^= 1; }
+                    s += 2;
+                    if (s >= a.stages) { s -= a.stages; ph ^= 1; }
+                    b += 2;
+                    if (b >= a.acc_bufs) { b -= a.acc_bufs; aph ^= 1; }
                 }
             }
         } else {
@@ -817,16 +825,20 @@ __global__ void __launch_bounds__(kK1Threads, 1)
             const int grp = (warp - 2) >> 2;
             const int r = quarter * 32 + lane;
             // this group's tiles t = grp, grp + 2, ... use buffers grp, grp + 2, ...
-            int b = grp;
-            uint32_t aph = 0;
+            // and ring stages grp, grp + 2, ... (whose commit marks the tile's
+            // MMAs complete)
+            int b = grp, se = grp;
+            uint32_t eph = 0;
             for (int t = grp; t < ntiles; t += 2) {
                 // lane 0 polls (eight warps polling with every lane would
                 // steal issue slots from the producer and MMA threads); then
                 // every lane observes the completed phase itself -- its own
-                // acquire, which cannot fail: the buffer's next phase needs
-                // this warp's release below.  The warp proceeds only if all
-                // lanes saw it (tcgen05.ld below is warp-collective).
-                const bool ok = warp_wait(&sm.acc_full[b], aph, &sm.abort, a.wait_budget);
+                // acquire, which cannot fail: the stage's next phase is the
+                // commit of tile t + a.stages, which the same MMA thread
+                // issues after tile t + a.acc_bufs, whose buffer needs this
+                // warp's release below.  The warp proceeds only if all lanes
+                // saw it (tcgen05.ld below is warp-collective).
+                const bool ok = warp_wait(&sm.empty[se], eph, &sm.abort, a.wait_budget);
                 if (!ok) {
                     if (lane == 0) {
                         record_status(a.status, DSA_ERR_TIMEOUT);
@@ -884,7 +896,9 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.acc_empty[b]);
                 b += 2;
-                if (b >= a.acc_bufs) { b -= a.acc_bufs; aph ^= 1; }
+                if (b >= a.acc_bufs) b -= a.acc_bufs;
+                se += 2;
+                if (se >= a.stages) { se -= a.stages; eph ^= 1; }
             }
         }
     }

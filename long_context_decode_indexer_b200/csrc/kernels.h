@@ -28,7 +28,7 @@ constexpr int kModeTopk = 2;    // TopK of scores read from HBM
 #endif
 constexpr int kK1MaxStages = 12;     // TMA ring barriers
 constexpr int kK1MaxAcc = 4;         // TMEM accumulator buffers (even: one parity per epilogue group)
-constexpr int kK1Threads = 320;      // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9: two epilogue groups
+constexpr int kK1Threads = 352;      // warp 0 TMA, warps 1 and 10 MMA (even / odd tiles), warps 2-5 and 6-9: epilogue
 constexpr int kK2Threads = 256;
 constexpr int kMaxGroupQueries = 2;  // queries sharing one k^I tile (N <= 2 * 64)
 constexpr int kMaxChunks = 32;       // chunks per query group (merge bookkeeping)
