@@ -792,7 +792,11 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                 const uint64_t ad0 = make_sdesc(smem_u32(stages), 16, kSbo, kLayout);
                 const uint64_t bd0 = make_sdesc(smem_u32(qtile), 16, kSbo, kLayout);
                 // ring stage and accumulator of tile t = r0, r0 + 2, ...: both
-                // advance by two per tile (a.stages even, a.acc_bufs even)
+                // advance by two per tile (a.stages even, a.acc_bufs even).
+                // The parity waits below cannot alias an older phase because
+                // tiles t - a.acc_bufs and t - a.stages (same parity) went
+                // through this same thread first: a third issuer breaks that
+                // (tried: it let a tile into a buffer still in use).
                 int s = r0, b = r0;
                 uint32_t ph = 0, aph = 0;
                 for (int t = r0; t < ntiles; t += 2) {
