@@ -29,7 +29,8 @@ Printed: one JSON line (rank 0).  `roofline` is for the dominant kernel (the
 fused indexer), timed alone over the same workload; `stages` gives each
 stage's time and its fraction of the binding roofline; `e2e` repeats the step
 through the C ABI from pinned host buffers (query-side inputs in, outputs
-out; the caches are resident state); `cpu_baseline` is the fp64 oracle timed
+out; the caches are resident state), steps pipelined over two buffer sets
+so that each step's copies overlap its neighbours' kernels; `cpu_baseline` is the fp64 oracle timed
 on a bounded sample on this host, on all cores and on one.  `next_rows` (one
 GPU, decode workloads) times the rows after the decode path alone: the
 indexer's q/k/w producer for the batch's tokens, attention over an FP8
@@ -504,6 +505,8 @@ def run_ours(args, world, rank):
     if e2e is not None:
         e2e["value"] = total_q / e2e.pop("t")
         e2e["eager_value"] = total_q / e2e.pop("t_eager")
+        t_graph = e2e.pop("t_graph")
+        e2e["graph_value"] = total_q / t_graph if t_graph else None
         res["e2e"] = e2e
     return res, inp
 
@@ -644,84 +647,108 @@ def measure_next_rows(runs, timed, evict, hbm, bf16, iters=20):
     return res
 
 
+E2E_SLOTS = 2        # device buffer sets: step k uses slot k % 2
+E2E_GRAPH_STEPS = 8  # steps recorded in one CUDA graph (pipelined inside it)
+
+
 def run_e2e(args, world, inp, db, p, idx, out, lse, ws_idx, ws_mla, mla_fn, timed):
-    """The step end to end through the C ABI from pinned host buffers: the
-    query-side inputs go up, the indices and the attention output come back,
-    every step (the caches are resident state)."""
+    """The step end to end through the C ABI from pinned host buffers: every
+    step uploads its query-side inputs and downloads its indices, attention
+    output and LSE (the caches are resident state).  Steps are pipelined over
+    two buffer sets and three streams, as a server runs independent batches:
+    the uploads of step k + 1 (copy engine, host to device) and the downloads
+    of step k - 1 (device to host) run while step k computes."""
     st = torch.cuda.current_stream()
     h_qidx = torch.from_numpy(inp.q_idx).pin_memory()
     h_w = torch.from_numpy(inp.w.view(np.int16)).pin_memory()
     h_q = torch.from_numpy(inp.q.view(np.int16)).pin_memory()
     h_qn = torch.from_numpy(inp.q_n).pin_memory()
     h_qseq = torch.from_numpy(inp.q_seq).pin_memory()
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    h_idx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    d_qidx, d_w, d_q = torch.empty_like(db.q_idx), torch.empty_like(db.w), torch.empty_like(db.q)
-    d_qn, d_qseq = torch.empty_like(db.q_n), torch.empty_like(db.q_seq)
-    kv_e = dsa.make_kv(q_seq=d_qseq, q_n=d_qn, seq_row0=db.seq_row0, page_table=db.page_table,
-                       page_size=inp.page_size, cache_rows=db.kidx.shape[0])
+    slots = []
+    for j in range(E2E_SLOTS):
+        sl = {"d_qidx": torch.empty_like(db.q_idx), "d_w": torch.empty_like(db.w), "d_q": torch.empty_like(db.q),
+              "d_qn": torch.empty_like(db.q_n), "d_qseq": torch.empty_like(db.q_seq),
+              "idx": torch.empty_like(idx), "out": torch.empty_like(out), "lse": torch.empty_like(lse),
+              "h_out": torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+              "h_lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory(),
+              "h_idx": torch.empty(idx.shape, dtype=idx.dtype).pin_memory()}
+        sl["kv"] = dsa.make_kv(q_seq=sl["d_qseq"], q_n=sl["d_qn"], seq_row0=db.seq_row0,
+                               page_table=db.page_table, page_size=inp.page_size, cache_rows=db.kidx.shape[0])
+        slots.append(sl)
     h2d = sum(t.numel() * t.element_size() for t in (h_qidx, h_w, h_q, h_qn, h_qseq))
-    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_idx))
+    d2h = sum(slots[0][k].numel() * slots[0][k].element_size() for k in ("h_out", "h_lse", "h_idx"))
 
     ref_out = out.clone()  # the device-resident path's result, for the check below
-    copy_stream = torch.cuda.Stream()
+    up_stream, down_stream = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def e2e_step():
-        # The same two stages through the public entry points (dsa_indexer_topk,
-        # then the sparse attention, which is what dsa_forward runs), with the
-        # copies overlapped on a second stream: the attention query goes up
-        # while the indexer runs, the indices come down while the attention
-        # runs.  `cur` is the capture stream while a graph is recorded.
+    def run_steps(n):
+        """n consecutive steps; `cur` is the capture stream while a graph is
+        recorded (the side streams fork from it and join it at the end)."""
         cur = torch.cuda.current_stream()
-        copy_stream.wait_stream(cur)                 # the previous step is done with d_q
-        with torch.cuda.stream(copy_stream):
-            d_q.copy_(h_q, non_blocking=True)
-        for d, h in ((d_qidx, h_qidx), (d_w, h_w), (d_qn, h_qn), (d_qseq, h_qseq)):
-            d.copy_(h, non_blocking=True)
-        dsa.indexer_topk(p, kv_e, d_qidx, d_w, db.kidx, db.k_scale, idx, None, ws_idx)
-        cur.wait_stream(copy_stream)                 # the query is on the device
-        copy_stream.wait_stream(cur)                 # the indices are final
-        with torch.cuda.stream(copy_stream):
-            h_idx.copy_(idx, non_blocking=True)
-        mla_fn(p, kv_e, d_q, db.kv, db.kv_row_stride, idx, out, lse, ws_mla)
-        h_out.copy_(out, non_blocking=True)
-        h_lse.copy_(lse, non_blocking=True)
-        cur.wait_stream(copy_stream)                 # join the copy stream
+        up_stream.wait_stream(cur)
+        down_stream.wait_stream(cur)
+        # fresh events: a wait on one not yet recorded is a no-op, and no wait
+        # reaches an event recorded outside the run (or outside a capture)
+        for sl in slots:
+            sl["up"], sl["comp"], sl["down"] = torch.cuda.Event(), torch.cuda.Event(), torch.cuda.Event()
+        for k in range(n):
+            sl = slots[k % E2E_SLOTS]
+            with torch.cuda.stream(up_stream):
+                up_stream.wait_event(sl["comp"])      # step k - 2 is done with the inputs
+                for d, h in (("d_qidx", h_qidx), ("d_w", h_w), ("d_q", h_q), ("d_qn", h_qn), ("d_qseq", h_qseq)):
+                    sl[d].copy_(h, non_blocking=True)
+                sl["up"].record(up_stream)
+            cur.wait_event(sl["up"])
+            cur.wait_event(sl["down"])                # step k - 2's results are on the host
+            dsa.indexer_topk(p, sl["kv"], sl["d_qidx"], sl["d_w"], db.kidx, db.k_scale, sl["idx"], None, ws_idx)
+            mla_fn(p, sl["kv"], sl["d_q"], db.kv, db.kv_row_stride, sl["idx"], sl["out"], sl["lse"], ws_mla)
+            sl["comp"].record(cur)
+            with torch.cuda.stream(down_stream):
+                down_stream.wait_event(sl["comp"])
+                sl["h_idx"].copy_(sl["idx"], non_blocking=True)
+                sl["h_out"].copy_(sl["out"], non_blocking=True)
+                sl["h_lse"].copy_(sl["lse"], non_blocking=True)
+                sl["down"].record(down_stream)
+        cur.wait_stream(up_stream)
+        cur.wait_stream(down_stream)
 
-    for _ in range(args.warmup):
-        e2e_step()
+    run_steps(max(args.warmup, E2E_SLOTS))
     torch.cuda.synchronize()
     barrier(world)
-    t_eager = max_over_ranks(timed(e2e_step, args.steps), world)
-    # The same step recorded once as a CUDA graph (copies from the pinned
-    # buffers, the two stages' launches, copies back, both streams) and
-    # replayed: one host launch per step, as a decode loop would run it.
-    launch = "cuda_graph"
+    t_eager = max_over_ranks(timed(lambda: run_steps(args.steps), 1), world)
+    # E2E_GRAPH_STEPS pipelined steps recorded once as a CUDA graph and
+    # replayed: one host launch per group of steps, as a decode loop would
+    # run it; the time per step is the replays' time over the steps they ran.
     try:
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(st)
         with torch.cuda.stream(side):
-            e2e_step()
+            run_steps(E2E_SLOTS)
         st.wait_stream(side)
         torch.cuda.synchronize()
         with torch.cuda.graph(graph):
-            e2e_step()
-        for _ in range(args.warmup):
+            run_steps(E2E_GRAPH_STEPS)
+        for _ in range(max(1, args.warmup // E2E_GRAPH_STEPS)):
             graph.replay()
         torch.cuda.synchronize()
         barrier(world)
-        t = max_over_ranks(timed(graph.replay, args.steps), world)
+        reps = max(1, args.steps // E2E_GRAPH_STEPS)
+        t_graph = max_over_ranks(timed(graph.replay, reps), world) / (reps * E2E_GRAPH_STEPS) * args.steps
         del graph
     except RuntimeError as exc:  # capture refused: report the eager loop
         print("e2e graph capture failed (%s); reporting the eager loop" % exc, file=sys.stderr)
-        launch, t = "eager", t_eager
+        t_graph = None
+    # the faster of the two launch modes (both reported); on the boxes
+    # measured the copies set the pace and the eager loop overlapped them better
+    t, launch = (t_graph, "cuda_graph") if t_graph is not None and t_graph <= t_eager else (t_eager, "eager")
     torch.cuda.synchronize()
-    same = bool(torch.equal(h_out, ref_out.cpu()))  # host copy == device-resident result
-    return {"t": t, "t_eager": t_eager, "unit": "queries/s", "h2d_bytes_per_step": h2d,
+    same = all(bool(torch.equal(sl["h_out"], ref_out.cpu())) for sl in slots)  # host copies == device result
+    return {"t": t, "t_eager": t_eager, "t_graph": t_graph, "unit": "queries/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "launch": launch,
-            "copies": "overlapped with the kernels on a second stream",
+            "copies": "pipelined: uploads of the next step and downloads of the previous one run "
+                      "during each step's kernels (two buffer sets, three streams)",
+            "graph_steps": E2E_GRAPH_STEPS,
             "matches_device_result": same}
 
 

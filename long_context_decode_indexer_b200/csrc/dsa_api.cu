@@ -527,11 +527,18 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
         a.cand_stride = cand_stride(p);
         a.cand_cnt = at<int32_t>(ws, wl.cand_cnt);
         a.cand_above = at<int32_t>(ws, wl.cand_above);
-        cudaError_t e = cudaMemsetAsync(static_cast<uint8_t *>(ws) + wl.zero_begin, 0,
-                                        wl.zero_end - wl.zero_begin, st);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
     }
     if (p->nq == 0) return DSA_OK;
+    // the cross-chunk counters start at zero: a clearing kernel right before
+    // the indexer, which starts as its programmatic dependent and waits for
+    // it only after streaming (not the TopK-only kernel, which reads scores
+    // a preceding kernel may still be writing)
+    bool pdl = false;
+    if (mode != dsa::kModeScores && pl.P > 1 && wl.zero_end > wl.zero_begin) {
+        cudaError_t e = dsa::launch_clear(static_cast<uint8_t *>(ws) + wl.zero_begin, wl.zero_end - wl.zero_begin, st);
+        if (e != cudaSuccess) return cuda_fail(e, "counter clear launch");
+        pdl = mode != dsa::kModeTopk;
+    }
     cudaError_t e;
     if (mode == dsa::kModeTopk) {
         a.q_n = kv ? kv->q_n : nullptr;
@@ -553,7 +560,7 @@ int run_indexer(const dsa_params *p, const dsa_kv *kv, int mode, const void *q_i
                          p->d_idx, p->d_idx, box_rows,
                          p->d_idx == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
-    e = dsa::launch_indexer(mode, pl.hp, p->d_idx, kmap, a, st);
+    e = dsa::launch_indexer(mode, pl.hp, p->d_idx, kmap, a, st, pdl);
     if (e != cudaSuccess) return cuda_fail(e, "indexer launch");
     return DSA_OK;
 }

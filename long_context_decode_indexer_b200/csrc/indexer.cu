@@ -909,6 +909,10 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // The cross-chunk counters below were cleared by k0_clear, which may
+    // still have been running while this grid streamed (launched as its
+    // programmatic dependent); long finished by now, this waits for nothing.
+    grid_dependency_wait();
     // the attention kernel may start launching on SMs this grid frees up
     // (it waits for this grid's completion before reading the indices)
     if (tid == 0) grid_launch_dependents();
@@ -1004,8 +1008,19 @@ __global__ void __launch_bounds__(kK2Threads, 1) k2_topk(const K1Params a) {
 // ---------------------------------------------------------------------------
 // host-side launchers
 // ---------------------------------------------------------------------------
+// Clears the indexer's cross-chunk counters of one call (16-byte units).
+// It lets the next kernel in the stream (k1, launched as its programmatic
+// dependent) start at once: k1 streams its keys meanwhile and waits for this
+// grid only before it touches the counters.
+__global__ void __launch_bounds__(256) k0_clear(uint4 *p, long long n16) {
+    grid_launch_dependents();
+    const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride)
+        p[i] = make_uint4(0, 0, 0, 0);
+}
+
 template <int MODE, int HP, int DI>
-static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaStream_t st) {
+static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaStream_t st, bool pdl) {
     const K1Layout L = k1_layout(MODE, DI, a.qg, HP, a.chunk, a.P, a.topk, a.stages, !a.parallel);
     const size_t smem = smem_for_tmem(L.total, a.tmem_cols);
     auto kern = k1_indexer<MODE, HP, DI>;
@@ -1013,14 +1028,38 @@ static cudaError_t launch_k1_t(const CUtensorMap &kmap, const K1Params &a, cudaS
     if (e != cudaSuccess) return e;
     const int grid = a.n_big * a.P + (a.n_groups - a.n_big) * (a.P - 1);
     if (grid == 0) return cudaSuccess;
-    kern<<<grid, kK1Threads, smem, st>>>(kmap, a);
+    if (!pdl) {
+        kern<<<grid, kK1Threads, smem, st>>>(kmap, a);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kK1Threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, kmap, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_clear(void *p, size_t bytes, cudaStream_t st) {
+    const long long n16 = static_cast<long long>(bytes / 16);
+    if (n16 == 0) return cudaSuccess;
+    long long grid = (n16 + 255) / 256;
+    if (grid > 1184) grid = 1184;
+    k0_clear<<<static_cast<int>(grid), 256, 0, st>>>(static_cast<uint4 *>(p), n16);
     return cudaGetLastError();
 }
 
 cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, const K1Params &a,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool pdl) {
 #define DSA_K1_CASE(M, H, D) \
-    if (mode == M && hp == H && di == D) return launch_k1_t<M, H, D>(kmap, a, st);
+    if (mode == M && hp == H && di == D) return launch_k1_t<M, H, D>(kmap, a, st, pdl);
     DSA_K1_CASE(kModeFused, 64, 128)
     DSA_K1_CASE(kModeFused, 16, 128)
     DSA_K1_CASE(kModeFused, 64, 64)

@@ -134,8 +134,13 @@ inline size_t smem_for_tmem(size_t want, uint32_t tmem_cols) {
     return want > floor_bytes ? want : floor_bytes;
 }
 
+// pdl: launched as the programmatic dependent of launch_clear (which must
+// directly precede it in the stream)
 cudaError_t launch_indexer(int mode, int hp, int di, const CUtensorMap &kmap, const K1Params &a,
-                           cudaStream_t st);
+                           cudaStream_t st, bool pdl);
+// zero `bytes` (a multiple of 16, 16-byte aligned) at p with a kernel that
+// lets its programmatic dependent start at once
+cudaError_t launch_clear(void *p, size_t bytes, cudaStream_t st);
 cudaError_t launch_topk(const K1Params &a, cudaStream_t st);
 
 // ------------------------------------------------------ sparse MLA attention
