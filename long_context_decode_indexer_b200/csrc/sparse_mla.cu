@@ -802,6 +802,14 @@ __device__ void combine_half_head(const MlaParams &a, int wq, int hh, int half) 
     const int d = half * 256 + lane * 8;
     const float ls = lane < a.splits ? __ldcg(&a.part_lse[row0 + 128 * lane]) : -INFINITY;
     const float sc = lane < a.splits ? __ldcg(&a.part_scale[(row0 + 128 * lane) * 2 + half]) : 0.f;
+    // the first kFirst splits' partial rows are loaded together with the
+    // statistics (one L2 round trip for the usual split counts)
+    constexpr int kFirst = 16;
+    uint4 raw0[kFirst];
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u)
+        raw0[u] = u < a.splits ? __ldcg(reinterpret_cast<const uint4 *>(a.part_o + (row0 + 128 * u) * kDv + d))
+                               : make_uint4(0, 0, 0, 0);
     float mx = ls;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -817,7 +825,18 @@ __device__ void combine_half_head(const MlaParams &a, int wq, int hh, int half) 
         return;
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int s0 = 0; s0 < a.splits; s0 += 8) {
+#pragma unroll
+    for (int u = 0; u < kFirst; ++u) {
+        const float wgt = __shfl_sync(0xffffffffu, wsc, u);
+        const uint32_t r4[4] = {raw0[u].x, raw0[u].y, raw0[u].z, raw0[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&r4[e]));
+            acc[2 * e] = fmaf(wgt, f.x, acc[2 * e]);
+            acc[2 * e + 1] = fmaf(wgt, f.y, acc[2 * e + 1]);
+        }
+    }
+    for (int s0 = kFirst; s0 < a.splits; s0 += 8) {
         uint4 raw[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
