@@ -82,7 +82,7 @@ K1_SOURCES = ("long_context_decode_indexer_b200/csrc/indexer.cu",
 # kernels.h holds every kernel's parameters: only its indexer part (up to
 # this line) belongs to k1
 K1_HEADER_END = "// ------------------------------------------------------ sparse MLA attention"
-K1_PROFILED = {"sha256_16": "74c477295bb3c3a2", "bytes_per_position": 131.636962890625}
+K1_PROFILED = {"sha256_16": "d9af3af125c4e33f", "bytes_per_position": 131.944580078125}
 
 
 def k1_sources_hash() -> str:

@@ -494,6 +494,7 @@ __device__ void chunk_select(const K1Params &a, K1Smem &sm, int q, int qi, int n
 __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32_t *hist,
                             uint64_t *list, int list_cap) {
     const int K = a.topk;
+    const int P = sm.chunk_P;  // this group's chunks (the lists' layout keeps a.P slots)
     uint32_t dstar, above;
     if (sm.g_complete[qi]) {
         // this CTA's snapshot already held every chunk's histogram
@@ -517,34 +518,34 @@ __device__ void group_merge(const K1Params &a, K1Smem &sm, int q, int qi, uint32
         // one lane per chunk (P <= 32): the counts are loaded in parallel,
         // the offsets are a warp scan of the padded counts
         const int c = threadIdx.x;
-        const int m = c < a.P ? min(__ldcg(&cnt[c]), K) : 0;
+        const int m = c < P ? min(__ldcg(&cnt[c]), K) : 0;
         const int padded = (m + 1) & ~1;
         const int incl = static_cast<int>(warp_incl_scan(static_cast<uint32_t>(padded)));
-        if (c < a.P) {
+        if (c < P) {
             sm.cand_off[c] = incl - padded;
             sm.cand_n[c] = m;
         }
         const int off = __shfl_sync(0xffffffffu, incl, 31);
         if (c == 0) {
-            sm.cand_off[a.P] = off;
+            sm.cand_off[P] = off;
             if (off <= list_cap) mbar_arrive_expect_tx(&sm.merge_bar, static_cast<uint32_t>(off) * 8u);
         }
     }
     __syncthreads();
-    const int total = sm.cand_off[a.P];
+    const int total = sm.cand_off[P];
     if (total > list_cap) {
         if (threadIdx.x == 0) record_status(a.status, DSA_ERR_DEVICE_CHECK);
         __syncthreads();
         return;
     }
-    if (threadIdx.x < a.P) {
+    if (threadIdx.x < P) {
         const int c = threadIdx.x, m = sm.cand_n[c];
         if (m > 0)
             bulk_load(list + sm.cand_off[c], cand + static_cast<int64_t>(c) * a.cand_stride,
                       static_cast<uint32_t>((m + 1) & ~1) * 8u, &sm.merge_bar);
     }
     const bool staged = __syncthreads_and(mbar_wait(&sm.merge_bar, sm.merge_phase, a.wait_budget));
-    if (threadIdx.x < a.P && (sm.cand_n[threadIdx.x] & 1)) list[sm.cand_off[threadIdx.x] + sm.cand_n[threadIdx.x]] = 0ull;
+    if (threadIdx.x < P && (sm.cand_n[threadIdx.x] & 1)) list[sm.cand_off[threadIdx.x] + sm.cand_n[threadIdx.x]] = 0ull;
     if (threadIdx.x == 0) sm.merge_phase ^= 1u;
     __syncthreads();
     if (!staged) {
@@ -586,7 +587,7 @@ __device__ bool arrive_group(const K1Params &a, K1Smem &sm, int g) {
     __syncthreads();
     if (threadIdx.x == 0) {
         const uint32_t prev = atomicAdd(&a.done[g], 1u);
-        sm.is_last = (prev == static_cast<uint32_t>(a.P - 1));
+        sm.is_last = (prev == static_cast<uint32_t>(sm.chunk_P - 1));
     }
     __syncthreads();
     if (sm.is_last) __threadfence();
@@ -665,6 +666,17 @@ __global__ void __launch_bounds__(kK1Threads, 1)
     }
     const int seq = nqg > 0 ? a.q_seq[q0] : 0;
     const int span = (MODE == kModeScores) ? static_cast<int>(a.ld) : nscored;
+    // With the merge selection a group uses only the chunks its own span
+    // needs (a.chunk positions at most, the plan's size for the longest
+    // span): the launch has a.P per group, and a batch of short and long
+    // histories would otherwise pay a.P chunks' fixed costs (set-up,
+    // histogram exchange, arrival) for every short one.  The CTAs past a
+    // group's count leave before touching anything shared.
+    if (MODE == kModeFused && !a.parallel) {
+        const int need = max(1, (span + a.chunk - 1) / a.chunk);
+        if (need < Pg) Pg = need;
+        if (c >= Pg) return;
+    }
     const int chunk = min(a.chunk, ((span + Pg - 1) / Pg + kTileRows - 1) / kTileRows * kTileRows);
     const int start = c * chunk;
     const int end = min(start + chunk, span);
@@ -931,7 +943,7 @@ __global__ void __launch_bounds__(kK1Threads, 1)
                          lhist + qi * kSelBins, hist, below_keys, below_cap);
             __syncthreads();
         }
-        if (a.P > 1 && !a.parallel) {
+        if (sm.chunk_P > 1 && !a.parallel) {
             bool any = false;
             for (int qi = 0; qi < nqg; ++qi) any |= sm.n_q[qi] > a.topk;
             if (any && arrive_group(a, sm, g)) {
